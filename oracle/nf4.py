@@ -1,0 +1,246 @@
+"""Oracle: blockwise NF4 quantization with double quantization (CPU, numpy).
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring.  Every step follows the
+pages' description in their order; where the pages are silent the reading used
+is stated at the function.
+
+Data layout (the same contract the CUDA library implements independently):
+  * W is taken as one flat row-major sequence of ``numel`` fp32 values.
+  * block  = 64 consecutive flat elements (last block may be partial);
+  * group  = 256 consecutive blocks (last group may be partial);
+  * codes  = ceil(numel/2) bytes, flat element 2j in the LOW nibble of byte j,
+             element 2j+1 in the HIGH nibble; an unused final high nibble is 0;
+  * absmax_q    = one uint8 per block;
+  * group_scale = one fp32 per group.
+
+Precision: all scalar steps are IEEE fp32 round-to-nearest-even (numpy float32
+arithmetic, no fused multiply-add), written ``fl32(.)`` below; bf16(.) is
+fp32 -> bf16 round-to-nearest-even.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import mpmath
+
+BLOCK = 64          # weights per absmax block
+GROUP = 256         # blocks per double-quantization group
+NLEVELS = 16
+
+
+# ---------------------------------------------------------------------------
+# Codebook
+# ---------------------------------------------------------------------------
+
+def nf4_levels_exact(dps: int = 50):
+    """The 16 NF4 levels as high-precision mpmath numbers, ascending.
+
+    [Blog-nf4]: NF4 places its 16 levels at quantiles of a normal distribution
+    so that each level covers an equal share of normally distributed weights;
+    [QLoRA-abs] (a): information-theoretically optimal for normal weights;
+    [Cap-nf4]: combined with block-wise absmax scaling.
+
+    Reading (the pages give no formula): the levels must span [-1, 1] (absmax
+    scaling maps every block into that interval) and contain an exact zero (so
+    a zero weight and an all-zero block survive).  16 = 1 zero + 8 positive +
+    7 negative quantiles.  The positive levels are the standard-normal
+    quantiles Phi^-1(p) at the 8 points p = d + (1/2 - d) i / 8, i = 0..7, the
+    negative ones are -Phi^-1(p) at p = d + (1/2 - d) i / 7, i = 0..6, with the
+    outer probability d = 1 - (1/32 + 1/30)/2 (finite quantile at the edge,
+    the midpoint of the 1/32 and 1/30 tail masses of 16 and 15 equal slices).
+    The set is divided by its largest magnitude so both ends land on +-1.
+    """
+    mp = mpmath.mp.clone()
+    mp.dps = dps
+    d = 1 - (mp.mpf(1) / 32 + mp.mpf(1) / 30) / 2
+
+    def phi_inv(p):
+        return mp.sqrt(2) * mp.erfinv(2 * p - 1)
+
+    pos = [phi_inv(d + (mp.mpf(1) / 2 - d) * i / 8) for i in range(8)]
+    neg = [-phi_inv(d + (mp.mpf(1) / 2 - d) * i / 7) for i in range(7)]
+    vals = sorted(pos + neg + [mp.mpf(0)])
+    top = max(abs(v) for v in vals)
+    return [v / top for v in vals]
+
+
+def nf4_codebook() -> np.ndarray:
+    """The 16 levels rounded to fp32 (round-to-nearest), ascending."""
+    return np.array([float(v) for v in nf4_levels_exact()], dtype=np.float64).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# bf16 helpers (bit patterns carried as uint16)
+# ---------------------------------------------------------------------------
+
+def bf16_rne_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 round-to-nearest-even, returned as uint16 bit patterns.
+
+    Definition: keep the upper 16 bits of the fp32 pattern, rounding the
+    discarded 16 bits to nearest with ties to an even kept part.  Inputs must be
+    finite (the quantizer rejects non-finite weights).
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    keep = u >> 16
+    rest = u & 0xFFFF
+    up = (rest > 0x8000) | ((rest == 0x8000) & ((keep & 1) == 1))
+    return (keep + up.astype(np.uint64)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# Quantization steps
+# ---------------------------------------------------------------------------
+
+def num_blocks(numel: int) -> int:
+    return -(-numel // BLOCK)
+
+
+def num_groups(numel: int) -> int:
+    return -(-num_blocks(numel) // GROUP)
+
+
+def footprint_bytes(numel: int) -> int:
+    """Bytes of the packed representation: codes + u8 constants + fp32 scales."""
+    return -(-numel // 2) + num_blocks(numel) + 4 * num_groups(numel)
+
+
+def block_absmax(w_flat: np.ndarray) -> np.ndarray:
+    """a_b = max |w| over each block of 64 consecutive flat elements (fp32, exact).
+
+    [Blog-nf4] (one scaling constant per block of weights), [Cap-nf4]
+    (block-wise absmax scaling), [Cap-qlora] (absmax tracking).
+    """
+    w = np.asarray(w_flat, dtype=np.float32).ravel()
+    nb = num_blocks(w.size)
+    pad = nb * BLOCK - w.size
+    a = np.abs(w)
+    if pad:
+        a = np.concatenate([a, np.zeros(pad, np.float32)])
+    return a.reshape(nb, BLOCK).max(axis=1).astype(np.float32)
+
+
+def normalize(w_flat: np.ndarray, absmax: np.ndarray) -> np.ndarray:
+    """n = fl32(w / a_b) for each element; n = 0 where a_b = 0 (all-zero block)."""
+    w = np.asarray(w_flat, dtype=np.float32).ravel()
+    a = np.repeat(absmax, BLOCK)[: w.size]
+    n = np.zeros_like(w)
+    nz = a != 0
+    n[nz] = w[nz] / a[nz]          # float32 / float32: IEEE RN
+    return n
+
+
+def nearest_code(n: np.ndarray, levels: np.ndarray, chunk: int = 1 << 20) -> np.ndarray:
+    """code = argmin_i |n - v_i| with ties broken to the LOWER index.
+
+    Distances are taken in fp64; for fp32 n and fp32 levels they are exact
+    wherever two distances can be close to a tie (every midpoint between
+    adjacent levels has magnitude >= 0.039), so the argmin is exact.
+    numpy's argmin returns the first minimum, i.e. the lower index.
+    """
+    n = np.asarray(n, dtype=np.float32).ravel()
+    v = np.asarray(levels, dtype=np.float32).astype(np.float64)
+    out = np.empty(n.size, dtype=np.uint8)
+    for s in range(0, n.size, chunk):
+        x = n[s:s + chunk].astype(np.float64)
+        dist = np.abs(x[:, None] - v[None, :])
+        out[s:s + chunk] = np.argmin(dist, axis=1).astype(np.uint8)
+    return out
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte: element 2j -> low nibble, 2j+1 -> high nibble."""
+    c = np.asarray(codes, dtype=np.uint8).ravel()
+    if c.size % 2:
+        c = np.concatenate([c, np.zeros(1, np.uint8)])
+    return (c[0::2] & 0xF) | ((c[1::2] & 0xF) << 4)
+
+
+def unpack_nibbles(packed: np.ndarray, numel: int) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8).ravel()
+    c = np.empty(p.size * 2, dtype=np.uint8)
+    c[0::2] = p & 0xF
+    c[1::2] = p >> 4
+    return c[:numel]
+
+
+def double_quantize(absmax: np.ndarray):
+    """Quantize the fp32 block constants to 8 bits with one fp32 scale per group.
+
+    [Blog-nf4] (double quantization stores the per-block constants in 8-bit
+    with a second, coarser set of constants above them), [QLoRA-abs] (b),
+    [Cap-nf4].  Reading (the 8-bit format is not given): unsigned linear
+    8-bit codes with no offset, group = 256 consecutive blocks:
+        c_g = max_b a_b,   S_g = fl32(c_g / 255),
+        q_b = min(255, round_half_even(fl32(a_b / S_g)))   (q_b = 0 if S_g == 0).
+    Returns (q uint8 [nblocks], S float32 [ngroups]).
+    """
+    a = np.asarray(absmax, dtype=np.float32).ravel()
+    nb = a.size
+    ng = -(-nb // GROUP)
+    pad = ng * GROUP - nb
+    ap = np.concatenate([a, np.zeros(pad, np.float32)]) if pad else a
+    c = ap.reshape(ng, GROUP).max(axis=1).astype(np.float32)
+    S = (c / np.float32(255.0)).astype(np.float32)
+    Sb = np.repeat(S, GROUP)[:nb]
+    q = np.zeros(nb, dtype=np.uint8)
+    nz = Sb != 0
+    ratio = (a[nz] / Sb[nz]).astype(np.float32)           # fl32(a_b / S_g)
+    r = np.rint(ratio)                                      # half-to-even
+    q[nz] = np.minimum(r, 255.0).astype(np.uint8)
+    return q, S
+
+
+def dequantize_absmax(q: np.ndarray, S: np.ndarray) -> np.ndarray:
+    """a'_b = fl32(q_b * S_g)."""
+    q = np.asarray(q, dtype=np.uint8).ravel()
+    Sb = np.repeat(np.asarray(S, np.float32), GROUP)[: q.size]
+    return (q.astype(np.float32) * Sb).astype(np.float32)
+
+
+def quantize_nf4(W: np.ndarray):
+    """Quantize fp32 weights once, up front ([Blog-mem]: the base never changes,
+    so it is quantized once).
+
+    Steps in the pages' order: block absmax -> normalise -> nearest NF4 level
+    -> pack 4-bit codes -> double-quantize the block constants.  The codes use
+    the exact fp32 block absmax (the constants are quantized afterwards, as a
+    separate second level).  Raises ValueError on non-finite input.
+
+    Returns dict(codes=uint8[ceil(numel/2)], absmax_q=uint8[nblocks],
+    group_scale=float32[ngroups], shape=W.shape).
+    """
+    W = np.asarray(W, dtype=np.float32)
+    if not np.all(np.isfinite(W)):
+        raise ValueError("non-finite weight")
+    flat = W.ravel()
+    a = block_absmax(flat)
+    n = normalize(flat, a)
+    codes = nearest_code(n, nf4_codebook())
+    q, S = double_quantize(a)
+    return {"codes": pack_nibbles(codes), "absmax_q": q, "group_scale": S,
+            "shape": tuple(W.shape)}
+
+
+def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np.ndarray,
+                        shape) -> np.ndarray:
+    """W' = bf16(fl32(v_code * a'_b)) with a'_b = fl32(q_b * S_g); bf16 bit patterns.
+
+    [Blog-mem]: the 4-bit base is dequantized on the fly to 16-bit for each
+    forward and backward pass.  Reading: the 16-bit type is bf16, the product
+    is formed in fp32 then rounded once to bf16.
+    """
+    numel = int(np.prod(shape))
+    c = unpack_nibbles(codes, numel)
+    v = nf4_codebook()[c]
+    ap = np.repeat(dequantize_absmax(absmax_q, group_scale), BLOCK)[:numel]
+    w32 = (v * ap).astype(np.float32)
+    return bf16_rne_bits(w32).reshape(shape)
+
+
+def dequantize_nf4(q: dict) -> np.ndarray:
+    """Convenience: dequantize a quantize_nf4() result to bf16 bit patterns."""
+    return dequantize_nf4_bits(q["codes"], q["absmax_q"], q["group_scale"], q["shape"])
