@@ -1,0 +1,200 @@
+"""Thin Python binding of libqlora.so (NF4 + double quantization + LoRA linear, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  Tensors are torch CUDA tensors (device memory and streams come
+from PyTorch); each call enqueues on ``torch.cuda.current_stream()``.
+
+The library must be built (``python -m bit_quantized_lora_nf4_b200.build``);
+there is no fallback: a missing or unloadable library raises at first use.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QLORA_OP_FWD = 0
+QLORA_OP_BWD = 1
+
+STATUS_NAMES = {
+    0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED_SHAPE", 3: "QLORA_ERR_MISALIGNED",
+    4: "QLORA_ERR_NONFINITE", 5: "QLORA_ERR_DEVICE_TIMEOUT", 6: "QLORA_ERR_CUDA", 7: "QLORA_ERR_WORKSPACE",
+}
+
+# Every symbol include/qlora.h declares.
+EXPORTS = (
+    "qlora_codes_bytes", "qlora_absmax_bytes", "qlora_group_scale_bytes", "qlora_quantize_nf4", "qlora_dequantize",
+    "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
+    "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout",
+)
+
+
+class QloraError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class Nf4WeightC(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p),
+                ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libqlora.so once and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libqlora.so not built at {path}; run python -m bit_quantized_lora_nf4_b200.build")
+    lib = ctypes.CDLL(path)
+    vp, i64, sz, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+    wp = ctypes.POINTER(Nf4WeightC)
+    sig = {
+        "qlora_codes_bytes": (sz, [i64, i64]),
+        "qlora_absmax_bytes": (sz, [i64, i64]),
+        "qlora_group_scale_bytes": (sz, [i64, i64]),
+        "qlora_quantize_nf4": (i32, [vp, wp, vp]),
+        "qlora_dequantize": (i32, [wp, vp, vp]),
+        "qlora_workspace_bytes": (sz, [i32, i64, i64, i64, i32]),
+        "qlora_linear_fwd": (i32, [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_linear_bwd": (i32, [wp, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
+        "qlora_nf4_codebook": (i32, [ctypes.POINTER(ctypes.c_float)]),
+        "qlora_device_status": (i32, [vp]),
+        "qlora_status_string": (ctypes.c_char_p, [i32]),
+        "qlora_set_wait_limit": (ctypes.c_uint64, [ctypes.c_uint64]),
+        "qlora_selftest_wait_timeout": (i32, [ctypes.c_uint64, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise QloraError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+@dataclass
+class NF4Weight:
+    """Frozen base weight [rows, cols] in NF4 with double-quantized constants (device tensors)."""
+    rows: int
+    cols: int
+    codes: torch.Tensor        # uint8 [ceil(rows*cols/2)]
+    absmax_q: torch.Tensor     # uint8 [ceil(rows*cols/64)]
+    group_scale: torch.Tensor  # float32 [ceil(rows*cols/16384)]
+
+    def c_struct(self) -> Nf4WeightC:
+        return Nf4WeightC(self.rows, self.cols, self.codes.data_ptr(), self.absmax_q.data_ptr(),
+                          self.group_scale.data_ptr())
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "NF4Weight":
+        lib = load()
+        return NF4Weight(rows, cols,
+                         torch.empty(lib.qlora_codes_bytes(rows, cols), dtype=torch.uint8, device=device),
+                         torch.empty(lib.qlora_absmax_bytes(rows, cols), dtype=torch.uint8, device=device),
+                         torch.empty(lib.qlora_group_scale_bytes(rows, cols) // 4, dtype=torch.float32,
+                                     device=device))
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.absmax_q.numel() + 4 * self.group_scale.numel()
+
+
+def codebook() -> list:
+    lib = load()
+    out = (ctypes.c_float * 16)()
+    _check(lib.qlora_nf4_codebook(out), "qlora_nf4_codebook")
+    return list(out)
+
+
+def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
+    return int(load().qlora_workspace_bytes(op, M, N, K, r))
+
+
+def device_status() -> int:
+    return int(load().qlora_device_status(_stream()))
+
+
+def set_wait_limit(cycles: int) -> int:
+    return int(load().qlora_set_wait_limit(cycles))
+
+
+def selftest_wait_timeout(cycles: int) -> int:
+    lib = load()
+    _check(lib.qlora_selftest_wait_timeout(cycles, _stream()), "qlora_selftest_wait_timeout")
+    return device_status()
+
+
+def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None) -> NF4Weight:
+    """Quantize a contiguous fp32 CUDA tensor [rows, cols] (flat row-major)."""
+    lib = load()
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    rows, cols = (W.shape[0], W[0].numel()) if W.dim() >= 2 else (1, W.numel())
+    w = out if out is not None else NF4Weight.empty(rows, cols, W.device)
+    s = w.c_struct()
+    _check(lib.qlora_quantize_nf4(_ptr(W), ctypes.byref(s), _stream()), "qlora_quantize_nf4")
+    return w
+
+
+def dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:
+    lib = load()
+    if out is None:
+        out = torch.empty((w.rows, w.cols), dtype=torch.bfloat16, device=w.codes.device)
+    s = w.c_struct()
+    _check(lib.qlora_dequantize(ctypes.byref(s), _ptr(out), _stream()), "qlora_dequantize")
+    return out
+
+
+def linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float, save_h: bool = True,
+               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Y = X W'^T + s (X A^T) B^T.  Returns (Y bf16 [M,N], H fp32 [M,r] or None)."""
+    lib = load()
+    M, r = X.shape[0], A.shape[0]
+    Y = out if out is not None else torch.empty((M, w.rows), dtype=torch.bfloat16, device=X.device)
+    H = torch.empty((M, r), dtype=torch.float32, device=X.device) if save_h else None
+    need = lib.qlora_workspace_bytes(QLORA_OP_FWD, M, w.rows, w.cols, r)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
+    st = w.c_struct()
+    _check(lib.qlora_linear_fwd(ctypes.byref(st), _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(Y), _ptr(H), _ptr(ws),
+                                ws.numel(), _stream()), "qlora_linear_fwd")
+    return Y, H
+
+
+def linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float,
+               H: torch.Tensor | None = None, outs=None, workspace: torch.Tensor | None = None):
+    """Returns (dX bf16 [M,K], dA fp32 [r,K], dB fp32 [N,r]); the frozen W' gets no gradient."""
+    lib = load()
+    M, r = X.shape[0], A.shape[0]
+    if outs is None:
+        dX = torch.empty((M, w.cols), dtype=torch.bfloat16, device=X.device)
+        dA = torch.empty((r, w.cols), dtype=torch.float32, device=X.device)
+        dB = torch.empty((w.rows, r), dtype=torch.float32, device=X.device)
+    else:
+        dX, dA, dB = outs
+    need = lib.qlora_workspace_bytes(QLORA_OP_BWD, M, w.rows, w.cols, r)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
+    st = w.c_struct()
+    _check(lib.qlora_linear_bwd(ctypes.byref(st), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, s, _ptr(H), _ptr(dX),
+                                _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream()), "qlora_linear_bwd")
+    return dX, dA, dB

@@ -1,0 +1,383 @@
+// C ABI of libqlora.so: argument validation, workspace planning and the
+// launch order of the quantizer, the dequantizer and the LoRA linear.
+#include <cmath>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+
+#include "internal.h"
+
+namespace qlora {
+
+// ----------------------------------------------------------------- NF4 table
+namespace {
+
+// Standard normal quantile by Newton's method on the complementary error
+// function, in extended precision.
+long double normal_quantile(long double p) {
+  long double x = 0.0L;
+  const long double rt2 = sqrtl(2.0L);
+  const long double inv_sqrt_2pi = 0.398942280401432677939946059934381868L;
+  for (int it = 0; it < 200; ++it) {
+    const long double f = 0.5L * erfcl(-x / rt2) - p;
+    const long double d = inv_sqrt_2pi * expl(-0.5L * x * x);
+    const long double step = f / d;
+    x -= step;
+    if (fabsl(step) < 1e-19L * (1.0L + fabsl(x))) break;
+  }
+  return x;
+}
+
+Nf4Table build_nf4_table() {
+  // 8 positive quantiles at p = d + (1/2 - d) i / 8 and 7 negative ones at
+  // p = d + (1/2 - d) i / 7 (i from 0), an exact zero, scaled so the
+  // extreme levels are -1 and +1.
+  const long double d = 1.0L - (1.0L / 32.0L + 1.0L / 30.0L) / 2.0L;
+  long double v[16];
+  int k = 0;
+  for (int i = 0; i < 7; ++i) v[k++] = -normal_quantile(d + (0.5L - d) * i / 7.0L);
+  v[k++] = 0.0L;
+  for (int i = 7; i >= 0; --i) v[k++] = normal_quantile(d + (0.5L - d) * i / 8.0L);
+  long double top = 0.0L;
+  for (int i = 0; i < 16; ++i) top = fmaxl(top, fabsl(v[i]));
+  Nf4Table t{};
+  for (int i = 0; i < 16; ++i) t.level[i] = static_cast<float>(v[i] / top);
+  // thresholds: exact midpoint (representable in double) rounded toward -inf to fp32
+  for (int i = 0; i < 15; ++i) {
+    const double mid = (static_cast<double>(t.level[i]) + static_cast<double>(t.level[i + 1])) * 0.5;
+    float f = static_cast<float>(mid);
+    if (static_cast<double>(f) > mid) f = nextafterf(f, -INFINITY);
+    t.thresh[i] = f;
+  }
+  return t;
+}
+
+std::atomic<uint64_t> g_wait_limit{2000000000ull};
+
+__global__ void selftest_wait_kernel(uint64_t limit, int *status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the bounded wait must give up.
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit)) latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
+}
+
+}  // namespace
+
+const Nf4Table &nf4_table() {
+  static const Nf4Table t = build_nf4_table();
+  return t;
+}
+
+uint64_t wait_limit() { return g_wait_limit.load(); }
+
+// ----------------------------------------------------------------- device status word
+__device__ int g_device_status;
+
+int *device_status_ptr() {
+  static int *ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int *>(p);
+  }
+  return ptrs[dev];
+}
+
+// ----------------------------------------------------------------- tensor maps
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap *tm, const void *base, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- workspace plan
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+  // byte offsets into the workspace
+  size_t part = 0, H = 0, sH = 0, Hs = 0, Gb = 0, Gs = 0, total = 0;
+  int spH = 1, spG = 1, spB = 1, spA = 1;
+  int64_t kpsH = 0, kpsG = 0, kpsB = 0, kpsA = 0;
+  bool gemv = false;
+};
+
+Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r) {
+  Plan p;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up(bytes);
+    return o;
+  };
+  const size_t Mr = static_cast<size_t>(M) * r;
+  if (op == QLORA_OP_FWD && M <= kGemvMaxTokens && gemv_enabled()) {
+    p.gemv = true;
+    p.H = take(Mr * 4);
+    p.total = off < kAlign ? kAlign : off;
+    return p;
+  }
+  skinny_plan(M, r, K, &p.spH, &p.kpsH);
+  size_t part = static_cast<size_t>(p.spH) * Mr;
+  if (op == QLORA_OP_BWD) {
+    skinny_plan(M, r, N, &p.spG, &p.kpsG);
+    skinny_plan(N, 2 * r, M, &p.spB, &p.kpsB);
+    skinny_plan(2 * r, K, M, &p.spA, &p.kpsA);
+    part = std::max(part, static_cast<size_t>(p.spG) * Mr);
+    part = std::max(part, static_cast<size_t>(p.spB) * N * 2 * r);
+    part = std::max(part, static_cast<size_t>(p.spA) * 2 * r * K);
+  }
+  p.part = take(part * 4);
+  p.H = take(Mr * 4);
+  if (op == QLORA_OP_FWD) {
+    p.sH = take(Mr * 2);
+  } else {
+    p.Hs = take(Mr * 2 * 2);
+    p.Gb = take(Mr * 2);
+    p.Gs = take(Mr * 2 * 2);
+  }
+  p.total = off;
+  return p;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+qlora_status check_weight(const qlora_nf4_weight *w) {
+  if (!w || !w->codes || !w->absmax_q || !w->group_scale) return QLORA_ERR_INVALID_ARG;
+  if (w->rows < 1 || w->cols < 1) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+// Shape, pointer and alignment checks shared by the linear calls (no workspace).
+qlora_status check_linear(const qlora_nf4_weight *w, int64_t M, int r, float s, const void *X, const void *A,
+                          const void *B, const void *out) {
+  qlora_status st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || !out) return QLORA_ERR_INVALID_ARG;
+  if (M < 1 || r < 8 || r > 256 || !std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (r % 8 != 0 || w->cols % 64 != 0 || w->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 31) - 1 || w->rows > (int64_t(1) << 31) - 1 || w->cols > (int64_t(1) << 31) - 1)
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(out)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+qlora_status check_ws(const void *ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+#define QL_CUDA(expr)                                 \
+  do {                                                \
+    if ((expr) != cudaSuccess) return QLORA_ERR_CUDA; \
+  } while (0)
+#define QL_TRY(expr)                          \
+  do {                                        \
+    const qlora_status _s = (expr);           \
+    if (_s != QLORA_OK) return _s;            \
+  } while (0)
+
+// H = X A^T into H (fp32) and bf16(s*H) into sH; optional hi/lo copy into Hs.
+qlora_status run_h(const Plan &p, void *ws, const uint16_t *X, const uint16_t *A, int64_t M, int64_t K, int r,
+                   float s, float *H, uint16_t *sH, uint16_t *Hs, cudaStream_t st) {
+  SkinnyArgs a{X, K, true, A, K, true, M, r, K, p.spH, p.kpsH, at<float>(ws, p.part)};
+  QL_CUDA(launch_skinny(a, st));
+  QL_CUDA(launch_finalize_h(at<float>(ws, p.part), p.spH, M, r, s, H, sH, Hs, st));
+  return QLORA_OK;
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+size_t qlora_codes_bytes(int64_t rows, int64_t cols) {
+  return rows < 1 || cols < 1 ? 0 : static_cast<size_t>((rows * cols + 1) / 2);
+}
+size_t qlora_absmax_bytes(int64_t rows, int64_t cols) {
+  return rows < 1 || cols < 1 ? 0 : static_cast<size_t>((rows * cols + kBlock - 1) / kBlock);
+}
+size_t qlora_group_scale_bytes(int64_t rows, int64_t cols) {
+  const int64_t nb = (rows * cols + kBlock - 1) / kBlock;
+  return rows < 1 || cols < 1 ? 0 : static_cast<size_t>((nb + kGroup - 1) / kGroup) * 4;
+}
+
+const char *qlora_status_string(qlora_status st) {
+  switch (st) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "QLORA_ERR_UNSUPPORTED_SHAPE";
+    case QLORA_ERR_MISALIGNED: return "QLORA_ERR_MISALIGNED";
+    case QLORA_ERR_NONFINITE: return "QLORA_ERR_NONFINITE";
+    case QLORA_ERR_DEVICE_TIMEOUT: return "QLORA_ERR_DEVICE_TIMEOUT";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+    case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE";
+  }
+  return "QLORA_ERR_UNKNOWN";
+}
+
+qlora_status qlora_nf4_codebook(float *out) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(out, nf4_table().level, sizeof(float) * 16);
+  return QLORA_OK;
+}
+
+uint64_t qlora_set_wait_limit(uint64_t cycles) { return g_wait_limit.exchange(cycles); }
+
+qlora_status qlora_selftest_wait_timeout(uint64_t cycles, void *stream) {
+  int *status = device_status_ptr();
+  if (!status) return QLORA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(cycles, status);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_device_status(void *stream) {
+  int *p = device_status_ptr();
+  if (!p) return QLORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return QLORA_ERR_CUDA;
+  }
+  return static_cast<qlora_status>(v);
+}
+
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
+  if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || M < 1 || N < 1 || K < 1 || r < 1) return 0;
+  return make_plan(op, M, N, K, r).total;
+}
+
+qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream) {
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_weight(out));
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  int *status = device_status_ptr();
+  if (!status) return QLORA_ERR_CUDA;
+  QL_CUDA(launch_quantize(W, out->rows * out->cols, out->codes, out->absmax_q, out->group_scale, status,
+                          static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream) {
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_weight(w));
+  if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
+  QL_CUDA(launch_dequantize(w->codes, w->absmax_q, w->group_scale, w->rows * w->cols, W_out,
+                            static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
+                              const uint16_t *B, int r, float s, uint16_t *Y, float *H_out, void *ws,
+                              size_t ws_bytes, void *stream) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear(w, M, r, s, X, A, B, Y));
+  const int64_t N = w->rows, K = w->cols;
+  const Plan p = make_plan(QLORA_OP_FWD, M, N, K, r);
+  QL_TRY(check_ws(ws, ws_bytes, p.total));
+  if (H_out && !aligned16(H_out)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *H = H_out ? H_out : at<float>(ws, p.H);
+  if (p.gemv) {
+    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<float>(ws, p.H)};
+    return launch_gemv(g, st);
+  }
+  QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
+  QGemmArgs g{false, M, N, K, X, w->codes, w->absmax_q, w->group_scale, at<uint16_t>(ws, p.sH), B, r, Y};
+  return launch_qgemm(g, st);
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
+                              const uint16_t *A, const uint16_t *B, int r, float s, const float *H_saved,
+                              uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream) {
+  if (!w || !dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear(w, M, r, s, X, A, B, dX));
+  const int64_t N = w->rows, K = w->cols;
+  const Plan p = make_plan(QLORA_OP_BWD, M, N, K, r);
+  QL_TRY(check_ws(ws, ws_bytes, p.total));
+  if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_MISALIGNED;
+  if (H_saved && !aligned16(H_saved)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *part = at<float>(ws, p.part);
+  uint16_t *Hs = at<uint16_t>(ws, p.Hs);
+  uint16_t *Gb = at<uint16_t>(ws, p.Gb);
+  uint16_t *Gs = at<uint16_t>(ws, p.Gs);
+
+  // H (recomputed when not saved) as a hi/lo bf16 pair for dB.
+  if (H_saved) {
+    QL_CUDA(launch_split_hilo(H_saved, M, r, Hs, st));
+  } else {
+    float *H = at<float>(ws, p.H);
+    SkinnyArgs a{X, K, true, A, K, true, M, r, K, p.spH, p.kpsH, part};
+    QL_CUDA(launch_skinny(a, st));
+    QL_CUDA(launch_finalize_h(part, p.spH, M, r, s, H, Gb /* scratch for s*H, overwritten below */, Hs, st));
+  }
+  // G = s dY B  -> Gb (dgrad operand) and Gs (hi/lo, for dA)
+  {
+    SkinnyArgs a{dY, N, true, B, r, false, M, r, N, p.spG, p.kpsG, part};
+    QL_CUDA(launch_skinny(a, st));
+    QL_CUDA(launch_finalize_g(part, p.spG, M, r, s, Gb, Gs, st));
+  }
+  // dB = s dY^T H
+  {
+    SkinnyArgs a{dY, N, false, Hs, 2 * static_cast<int64_t>(r), false, N, 2 * static_cast<int64_t>(r), M, p.spB,
+                 p.kpsB, part};
+    QL_CUDA(launch_skinny(a, st));
+    QL_CUDA(launch_finalize_cols(part, p.spB, N, r, s, dB, st));
+  }
+  // dA = G^T X
+  {
+    SkinnyArgs a{Gs, 2 * static_cast<int64_t>(r), false, X, K, false, 2 * static_cast<int64_t>(r), K, M, p.spA,
+                 p.kpsA, part};
+    QL_CUDA(launch_skinny(a, st));
+    QL_CUDA(launch_finalize_rows(part, p.spA, r, K, dA, st));
+  }
+  // dX = dY W' + Gb A
+  QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX};
+  return launch_qgemm(g, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,109 @@
+// Host-side declarations shared by the translation units of libqlora.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "qlora.h"
+
+namespace qlora {
+
+// NF4 table computed once on the host (normal quantiles, see api.cu).
+const Nf4Table &nf4_table();
+
+// Address of the device status word on the current device (nullptr on error).
+int *device_status_ptr();
+
+// Current bound on pipeline waits, in clock cycles.
+uint64_t wait_limit();
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---- tensor maps ------------------------------------------------------------
+// 2D tiled map over a row-major [outer, inner] array.
+bool make_tmap_2d(CUtensorMap *tm, const void *base, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+// ---- kernels (launchers return the launch error) -------------------------------
+cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
+                            int *status, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
+                              int64_t numel, uint16_t *out, cudaStream_t st);
+
+// Fused dequant-GEMM on tensor cores.
+//   forward: out[M, wN] = act[M, wK] . W'^T + lora_act[M, r] . lora_w[wN, r]^T
+//   dgrad  : out[M, wK] = act[M, wN] . W'   + lora_act[M, r] . lora_w[r, wK]
+struct QGemmArgs {
+  bool dgrad;
+  int64_t M;
+  int64_t wN, wK;
+  const uint16_t *act;
+  const uint8_t *codes;
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  const uint16_t *lora_act;
+  const uint16_t *lora_w;
+  int r;
+  uint16_t *out;
+};
+qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
+
+// Few-token forward: Y[M, N] = X W'^T + (s X A^T) B^T for M <= 16.
+struct GemvArgs {
+  int64_t M, wN, wK;
+  const uint16_t *X;
+  const uint8_t *codes;
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  const uint16_t *A;   // [r, K]
+  const uint16_t *B;   // [N, r]
+  int r;
+  float s;
+  uint16_t *Y;
+  float *H_out;        // optional [M, r]
+  float *h_ws;         // [M, r] scratch when H_out is null
+};
+qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st);
+constexpr int kGemvMaxTokens = 16;
+bool gemv_enabled();
+
+// Tall-skinny products on tensor cores (mma.sync), split over the reduction
+// with fp32 partials part[z][I][J]:  C[i,j] = sum_k opA(i,k) opB(j,k),
+// opX(i,k) = X[i*ld + k] when K-major, X[k*ld + i] otherwise.
+struct SkinnyArgs {
+  const uint16_t *A;
+  int64_t lda;
+  bool a_kmajor;
+  const uint16_t *B;
+  int64_t ldb;
+  bool b_kmajor;
+  int64_t I, J, Kred;
+  int splits;
+  int64_t k_per_split;
+  float *part;
+};
+cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st);
+// Pick the split count for a skinny product (deterministic in the sizes).
+void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per_split);
+
+// Epilogues of the skinny products.
+//   H  = sum_z part            -> H (fp32 [M,r]); sH = bf16(s*H) [M,r]; Hs = [bf16 hi | bf16 lo] [M,2r] (optional)
+cudaError_t launch_finalize_h(const float *part, int splits, int64_t M, int r, float s, float *H, uint16_t *sH,
+                              uint16_t *Hs, cudaStream_t st);
+//   Hs from an existing fp32 H (backward with a saved H)
+cudaError_t launch_split_hilo(const float *H, int64_t M, int r, uint16_t *Hs, cudaStream_t st);
+//   G = s * sum_z part -> Gb = bf16(G) [M,r], Gs = [hi | lo] [M,2r]
+cudaError_t launch_finalize_g(const float *part, int splits, int64_t M, int r, float s, uint16_t *Gb, uint16_t *Gs,
+                              cudaStream_t st);
+//   out[i,j] = scale * sum_z (part[z][i][j] + part[z][i][j + half])  for j < half  (row-split layout, I rows)
+cudaError_t launch_finalize_cols(const float *part, int splits, int64_t I, int64_t half, float scale, float *out,
+                                 cudaStream_t st);
+//   out[i,j] = sum_z (part[z][i][j] + part[z][i + half][j])          for i < half  (J cols)
+cudaError_t launch_finalize_rows(const float *part, int splits, int64_t half, int64_t J, float *out,
+                                 cudaStream_t st);
+
+}  // namespace qlora

@@ -1,0 +1,164 @@
+/*
+ * qlora.h -- C ABI of libqlora.so: blockwise NF4 storage with double
+ * quantization and the LoRA linear on top of it, forward and backward, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages, cited by title and section):
+ *   - "QLoRA: efficient finetuning of quantized LLMs", Abstract: gradients are
+ *     backpropagated through a frozen 4-bit quantized model into low-rank
+ *     adapters; (a) the NF4 data type, (b) double quantization of the
+ *     quantization constants.
+ *   - "QLoRA: fine-tuning a 65B model on one GPU", section "Where the memory
+ *     goes": the base is stored in 4 bits, quantized once up front, and
+ *     dequantized on the fly to 16-bit for every forward and backward pass;
+ *     gradients flow through the dequantized weights into the adapters, which
+ *     stay 16-bit.  Section "NormalFloat, double quantization, paged
+ *     optimizers": 16 levels at normal quantiles; one scaling constant per
+ *     block; the constants themselves stored in 8 bits under a second,
+ *     coarser set of constants.
+ *   - "Qlora 4 Bit Quantization With Nf4 Fp4 Data Types And Lora Adapters",
+ *     entry "4-bit quantization with nf4 data type for llm weight
+ *     compression": block-wise absmax scaling plus double quantization.
+ *
+ * Conventions for every call
+ *   - Every pointer argument named as "device" is CUDA device memory owned by
+ *     the caller.  The library never allocates or frees device memory; the
+ *     linear calls take a caller-provided workspace whose size is returned by
+ *     qlora_workspace_bytes().
+ *   - bf16 tensors are passed as uint16_t bit patterns.  All tensors are dense
+ *     row-major and every device pointer must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; no call synchronizes the stream, except
+ *     qlora_device_status().
+ *   - Argument errors are detected on the host and returned before anything is
+ *     enqueued.  Errors only the device can see (a non-finite weight handed to
+ *     the quantizer, a pipeline wait that exceeded its bound) are latched in a
+ *     device status word; read and clear it with qlora_device_status().
+ *   - Outputs are overwritten, never accumulated into.
+ *
+ * Fixed format: block = 64 consecutive elements of the flat row-major weight,
+ * group = 256 consecutive blocks.  codes: element 2j in the low nibble of byte
+ * j, 2j+1 in the high nibble (an unused final high nibble is 0).
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad rank/scale   */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2, /* e.g. cols % 64 != 0 for the linear           */
+  QLORA_ERR_MISALIGNED = 3,        /* a device pointer not 16-byte aligned         */
+  QLORA_ERR_NONFINITE = 4,         /* device: non-finite weight seen by quantizer  */
+  QLORA_ERR_DEVICE_TIMEOUT = 5,    /* device: a pipeline wait exceeded its bound   */
+  QLORA_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed            */
+  QLORA_ERR_WORKSPACE = 7          /* workspace missing or smaller than required   */
+} qlora_status;
+
+/* The frozen base weight W [rows=N (out), cols=K (in)] in NF4 + double quant.
+ * All three arrays are device memory owned by the caller.
+ *   codes       : ceil(rows*cols/2) bytes
+ *   absmax_q    : ceil(rows*cols/64) bytes, one unsigned 8-bit constant per block
+ *   group_scale : ceil(rows*cols/16384) fp32, one per group of 256 blocks     */
+typedef struct {
+  int64_t rows;
+  int64_t cols;
+  uint8_t *codes;
+  uint8_t *absmax_q;
+  float *group_scale;
+} qlora_nf4_weight;
+
+/* Sizes in bytes of the three arrays for a rows x cols weight. */
+size_t qlora_codes_bytes(int64_t rows, int64_t cols);
+size_t qlora_absmax_bytes(int64_t rows, int64_t cols);
+size_t qlora_group_scale_bytes(int64_t rows, int64_t cols);
+
+/* qlora_quantize_nf4 -- quantize fp32 weights once, up front.
+ * ("Where the memory goes": the base never changes, so it is quantized once.)
+ *   W   : device fp32 [out->rows * out->cols], flat row-major.
+ *   out : rows/cols set by the caller; codes/absmax_q/group_scale receive the
+ *         result.  Any rows*cols >= 1 is accepted (last block/group partial).
+ * Per block b: a_b = max|w| (exact fp32); n = fl32(w / a_b) (n = 0 if a_b = 0);
+ * code = index of the nearest NF4 level, ties to the lower index.
+ * Per group g: c_g = max a_b; S_g = fl32(c_g / 255);
+ * q_b = min(255, round-half-even(fl32(a_b / S_g))) (0 if S_g = 0).
+ * A non-finite weight latches QLORA_ERR_NONFINITE (outputs then undefined). */
+qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream);
+
+/* qlora_dequantize -- W' = bf16(fl32(v_code * fl32(q_b * S_g))) into a device
+ * bf16 buffer of rows*cols elements, row-major.  ("Where the memory goes":
+ * dequantized on the fly to 16-bit.)  Bit-exact by construction. */
+qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream);
+
+/* Operation ids for qlora_workspace_bytes(). */
+#define QLORA_OP_FWD 0
+#define QLORA_OP_BWD 1
+
+/* Workspace bytes the linear calls need for the given sizes (0 never means
+ * "no workspace" for the linear; it is at least 256). */
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
+
+/* qlora_linear_fwd -- Y = X W'^T + s (X A^T) B^T   (W' = dequantized base).
+ * ("QLoRA" Abstract; "Where the memory goes".)
+ *   w      : the NF4 weight, rows = N, cols = K; K % 64 == 0.
+ *   X      : device bf16 [M, K];  A : device bf16 [r, K];  B : device bf16 [N, r]
+ *   r      : 16 <= r <= 256, r % 16 == 0;  s : the adapter scale alpha / r.
+ *   Y      : device bf16 [M, N] (output).
+ *   H_out  : optional device fp32 [M, r]; receives H = X A^T for the backward.
+ *   ws     : device workspace of ws_bytes >= qlora_workspace_bytes(FWD, ...).
+ * M >= 1.  M <= 16 runs the memory-bound dequant-GEMV path; larger M runs the
+ * tensor-core fused dequant-GEMM with the adapter term as an extra K segment of
+ * the same accumulation.  fp32 accumulation; Y rounded once to bf16. */
+qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M,
+                              const uint16_t *A, const uint16_t *B, int r, float s,
+                              uint16_t *Y, float *H_out, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/* qlora_linear_bwd -- gradients of the linear; the frozen W' gets none.
+ *   G  = s dY B                 (fp32, internal)
+ *   dX = dY W' + G A            device bf16 [M, K]
+ *   dA = G^T X                  device fp32 [r, K]
+ *   dB = s dY^T (X A^T)         device fp32 [N, r]
+ * ("QLoRA" Abstract: gradients flow through the frozen 4-bit model into the
+ * adapters; "Where the memory goes": through the dequantized weights.)
+ *   H_saved : optional device fp32 [M, r] from qlora_linear_fwd; NULL makes the
+ *             call recompute X A^T.
+ * Same shape rules as the forward; M >= 1. */
+qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY,
+                              int64_t M, const uint16_t *A, const uint16_t *B, int r, float s,
+                              const float *H_saved, uint16_t *dX, float *dA, float *dB,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/* The 16 NF4 levels (ascending, fp32) as the library computes them on the
+ * host: standard-normal quantiles at 8 positive and 7 negative equally spaced
+ * probabilities from d = 1 - (1/32 + 1/30)/2 to 1/2, plus an exact 0,
+ * normalised to [-1, 1].  ("NormalFloat, double quantization, paged
+ * optimizers": 16 levels at normal quantiles.)  out: host float[16]. */
+qlora_status qlora_nf4_codebook(float *out);
+
+/* Synchronize `stream`, return the latched device status and clear it. */
+qlora_status qlora_device_status(void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *qlora_status_string(qlora_status st);
+
+/* Upper bound, in GPU clock cycles, on every pipeline wait inside the
+ * library's kernels (default 2e9, about one second).  Returns the old value. */
+uint64_t qlora_set_wait_limit(uint64_t cycles);
+
+/* Self-test of the bounded wait: launches one block that waits on a barrier
+ * nothing ever signals, with a bound of `cycles`.  The wait must give up and
+ * latch QLORA_ERR_DEVICE_TIMEOUT (read it with qlora_device_status()). */
+qlora_status qlora_selftest_wait_timeout(uint64_t cycles, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

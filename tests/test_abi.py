@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports every declared symbol, and validates
+arguments on the host (no GPU needed: every call here returns before any CUDA
+work is enqueued)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_quantized_lora_nf4_b200 as q
+from oracle import nf4
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "qlora.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = q.load()
+    decl = _declared()
+    assert len(decl) >= 13
+    for name in decl:
+        assert hasattr(lib, name), name
+    assert sorted(q.EXPORTS) == decl
+
+
+def test_codebook_matches_oracle_bitwise():
+    lib_cb = np.array(q.codebook(), dtype=np.float32)
+    assert np.array_equal(lib_cb.view(np.uint32), nf4.nf4_codebook().view(np.uint32))
+
+
+def test_size_helpers():
+    lib = q.load()
+    for rows, cols in ((256, 256), (4096, 11008), (3, 5), (1, 1)):
+        n = rows * cols
+        assert lib.qlora_codes_bytes(rows, cols) == (n + 1) // 2
+        assert lib.qlora_absmax_bytes(rows, cols) == nf4.num_blocks(n)
+        assert lib.qlora_group_scale_bytes(rows, cols) == 4 * nf4.num_groups(n)
+        assert (lib.qlora_codes_bytes(rows, cols) + lib.qlora_absmax_bytes(rows, cols)
+                + lib.qlora_group_scale_bytes(rows, cols)) == nf4.footprint_bytes(n)
+
+
+def test_status_strings():
+    lib = q.load()
+    for code, name in q.STATUS_NAMES.items():
+        assert lib.qlora_status_string(code).decode() == name
+
+
+def test_workspace_sizes_positive_and_monotone():
+    for op in (q.QLORA_OP_FWD, q.QLORA_OP_BWD):
+        a = q.workspace_bytes(op, 4096, 4096, 4096, 64)
+        b = q.workspace_bytes(op, 8192, 4096, 4096, 64)
+        assert 256 <= a <= b
+    assert q.workspace_bytes(7, 1, 1, 1, 1) == 0
+
+
+# ---------------------------------------------------------------- host-side argument errors
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: validation fails first
+MIS = 0x10001           # misaligned
+
+
+def _w(rows=256, cols=256, codes=FAKE, absmax=FAKE, scale=FAKE):
+    return q.Nf4WeightC(rows, cols, codes, absmax, scale)
+
+
+def _fwd(w, X=FAKE, M=64, A=FAKE, B=FAKE, r=16, s=1.0, Y=FAKE, H=None, ws=FAKE, wsb=1 << 40):
+    lib = q.load()
+    return lib.qlora_linear_fwd(ctypes.byref(w), X, M, A, B, r, s, Y, H, ws, wsb, None)
+
+
+def _bwd(w, X=FAKE, dY=FAKE, M=64, A=FAKE, B=FAKE, r=16, s=1.0, dX=FAKE, dA=FAKE, dB=FAKE, ws=FAKE, wsb=1 << 40):
+    lib = q.load()
+    return lib.qlora_linear_bwd(ctypes.byref(w), X, dY, M, A, B, r, s, None, dX, dA, dB, ws, wsb, None)
+
+
+def test_linear_argument_errors():
+    assert _fwd(_w(codes=None)) == 1
+    assert _fwd(_w(), X=None) == 1
+    assert _fwd(_w(), M=0) == 1
+    assert _fwd(_w(), r=4) == 1
+    assert _fwd(_w(), r=512) == 1
+    assert _fwd(_w(), s=float("nan")) == 1
+    assert _fwd(_w(), r=20) == 2                     # r % 8
+    assert _fwd(_w(cols=200)) == 2                   # K % 64
+    assert _fwd(_w(rows=250)) == 2                   # N % 8
+    assert _fwd(_w(), X=MIS) == 3
+    assert _fwd(_w(absmax=MIS)) == 3
+    assert _fwd(_w(), wsb=16) == 7
+    assert _fwd(_w(), ws=None) == 7
+    assert _bwd(_w(), dY=None) == 1
+    assert _bwd(_w(), dA=MIS) == 3
+    assert _bwd(_w(), wsb=0) == 7
+
+
+def test_quantize_dequantize_argument_errors():
+    lib = q.load()
+    w = _w()
+    assert lib.qlora_quantize_nf4(None, ctypes.byref(w), None) == 1
+    assert lib.qlora_quantize_nf4(MIS, ctypes.byref(w), None) == 3
+    assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(_w(rows=0)), None) == 1
+    assert lib.qlora_dequantize(ctypes.byref(w), None, None) == 1
+    assert lib.qlora_dequantize(ctypes.byref(_w(scale=MIS)), FAKE, None) == 3
+    assert lib.qlora_nf4_codebook(None) == 1
+
+
+def test_wait_limit_roundtrip():
+    old = q.set_wait_limit(12345)
+    assert q.set_wait_limit(old) == 12345
