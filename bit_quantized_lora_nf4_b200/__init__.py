@@ -31,8 +31,12 @@ STATUS_NAMES = {
 EXPORTS = (
     "qlora_codes_bytes", "qlora_absmax_bytes", "qlora_group_scale_bytes", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
-    "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout",
+    "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
+    "qlora_profile_read",
 )
+
+# Kernel kinds of the timing hook (qlora_profile_read).
+PROF_ALL, PROF_GEMM_FWD, PROF_GEMM_DGRAD, PROF_LORA, PROF_QUANT, PROF_DEQUANT, PROF_GEMV = range(7)
 
 
 class QloraError(RuntimeError):
@@ -73,6 +77,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_status_string": (ctypes.c_char_p, [i32]),
         "qlora_set_wait_limit": (ctypes.c_uint64, [ctypes.c_uint64]),
         "qlora_selftest_wait_timeout": (i32, [ctypes.c_uint64, vp]),
+        "qlora_profile_enable": (None, [i32]),
+        "qlora_profile_read": (i32, [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +152,17 @@ def selftest_wait_timeout(cycles: int) -> int:
     return device_status()
 
 
+def profile_enable(on: bool) -> None:
+    load().qlora_profile_enable(1 if on else 0)
+
+
+def profile_read(kind: int):
+    """(summed kernel time in ms, launch count) of one kernel kind since profile_enable(True)."""
+    ms, n = ctypes.c_double(), ctypes.c_int64()
+    _check(load().qlora_profile_read(kind, ctypes.byref(ms), ctypes.byref(n)), "qlora_profile_read")
+    return ms.value, n.value
+
+
 def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None) -> NF4Weight:
     """Quantize a contiguous fp32 CUDA tensor [rows, cols] (flat row-major)."""
     lib = load()
@@ -167,12 +184,14 @@ def dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:
 
 
 def linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float, save_h: bool = True,
-               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+               h_out: torch.Tensor | None = None):
     """Y = X W'^T + s (X A^T) B^T.  Returns (Y bf16 [M,N], H fp32 [M,r] or None)."""
     lib = load()
     M, r = X.shape[0], A.shape[0]
     Y = out if out is not None else torch.empty((M, w.rows), dtype=torch.bfloat16, device=X.device)
-    H = torch.empty((M, r), dtype=torch.float32, device=X.device) if save_h else None
+    H = h_out if h_out is not None else (
+        torch.empty((M, r), dtype=torch.float32, device=X.device) if save_h else None)
     need = lib.qlora_workspace_bytes(QLORA_OP_FWD, M, w.rows, w.cols, r)
     ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=X.device)
     st = w.c_struct()

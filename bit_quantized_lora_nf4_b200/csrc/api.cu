@@ -4,6 +4,8 @@
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 
@@ -91,6 +93,47 @@ int *device_status_ptr() {
   return ptrs[dev];
 }
 
+// ----------------------------------------------------------------- kernel timing hook
+namespace {
+struct Prof {
+  bool on = false;
+  std::vector<cudaEvent_t> pool;                 // reused across enable() calls
+  size_t next = 0;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pairs[kProfKinds];
+  cudaEvent_t open[kProfKinds] = {};
+  int64_t launches[kProfKinds] = {};
+};
+Prof &prof() {
+  static Prof p;
+  return p;
+}
+cudaEvent_t prof_event() {
+  Prof &P = prof();
+  if (P.next == P.pool.size()) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    P.pool.push_back(e);
+  }
+  return P.pool[P.next++];
+}
+}  // namespace
+
+void prof_mark(int kind, bool begin, cudaStream_t st) {
+  Prof &P = prof();
+  if (!P.on || kind <= 0 || kind >= kProfKinds) return;
+  cudaEvent_t e = prof_event();
+  if (!e) return;
+  cudaEventRecord(e, st);
+  if (begin) {
+    P.open[kind] = e;
+  } else if (P.open[kind]) {
+    P.pairs[kind].emplace_back(P.open[kind], e);
+    P.open[kind] = nullptr;
+    ++P.launches[kind];
+    ++P.launches[kProfAll];
+  }
+}
+
 // ----------------------------------------------------------------- tensor maps
 namespace {
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -147,7 +190,8 @@ Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r) {
   if (op == QLORA_OP_FWD && M <= kGemvMaxTokens && gemv_enabled()) {
     p.gemv = true;
     p.H = take(Mr * 4);
-    p.total = off < kAlign ? kAlign : off;
+    p.part = take(gemv_partial_bytes(M, N, K));
+    p.total = off;
     return p;
   }
   skinny_plan(M, r, K, &p.spH, &p.kpsH);
@@ -264,6 +308,33 @@ qlora_status qlora_nf4_codebook(float *out) {
 
 uint64_t qlora_set_wait_limit(uint64_t cycles) { return g_wait_limit.exchange(cycles); }
 
+void qlora_profile_enable(int on) {
+  Prof &P = prof();
+  P.on = on != 0;
+  P.next = 0;
+  for (int k = 0; k < kProfKinds; ++k) {
+    P.pairs[k].clear();
+    P.open[k] = nullptr;
+    P.launches[k] = 0;
+  }
+}
+
+qlora_status qlora_profile_read(int kind, double *ms_total, int64_t *launches) {
+  if (kind < 0 || kind >= kProfKinds || !ms_total || !launches) return QLORA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QLORA_ERR_CUDA;
+  Prof &P = prof();
+  double tot = 0.0;
+  for (int k = (kind == kProfAll ? 1 : kind); k <= (kind == kProfAll ? kProfKinds - 1 : kind); ++k)
+    for (auto &pr : P.pairs[k]) {
+      float ms = 0.0f;
+      if (cudaEventElapsedTime(&ms, pr.first, pr.second) != cudaSuccess) return QLORA_ERR_CUDA;
+      tot += ms;
+    }
+  *ms_total = tot;
+  *launches = P.launches[kind];
+  return QLORA_OK;
+}
+
 qlora_status qlora_selftest_wait_timeout(uint64_t cycles, void *stream) {
   int *status = device_status_ptr();
   if (!status) return QLORA_ERR_CUDA;
@@ -322,7 +393,8 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int6
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *H = H_out ? H_out : at<float>(ws, p.H);
   if (p.gemv) {
-    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<float>(ws, p.H)};
+    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<float>(ws, p.H),
+               at<float>(ws, p.part)};
     return launch_gemv(g, st);
   }
   QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));

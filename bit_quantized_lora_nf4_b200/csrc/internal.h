@@ -23,6 +23,12 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// ---- kernel timing hook (see qlora_profile_enable) --------------------------
+enum ProfKind { kProfAll = 0, kProfGemmFwd = 1, kProfGemmDgrad = 2, kProfLora = 3, kProfQuant = 4, kProfDequant = 5,
+                kProfGemv = 6, kProfKinds = 7 };
+// Records an event before (begin=true) or after a launch of `kind` on `st` when profiling is on.
+void prof_mark(int kind, bool begin, cudaStream_t st);
+
 // ---- tensor maps ------------------------------------------------------------
 // 2D tiled map over a row-major [outer, inner] array.
 bool make_tmap_2d(CUtensorMap *tm, const void *base, CUtensorMapDataType dtype, uint64_t inner, uint64_t outer,
@@ -66,7 +72,9 @@ struct GemvArgs {
   uint16_t *Y;
   float *H_out;        // optional [M, r]
   float *h_ws;         // [M, r] scratch when H_out is null
+  float *part;         // gemv_partial_bytes() of fp32 partial sums
 };
+size_t gemv_partial_bytes(int64_t M, int64_t N, int64_t K);
 qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st);
 constexpr int kGemvMaxTokens = 16;
 bool gemv_enabled();

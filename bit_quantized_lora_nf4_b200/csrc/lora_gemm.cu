@@ -289,6 +289,7 @@ void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per
 cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>(ceil_div(a.I, TI)), static_cast<unsigned>(ceil_div(a.J, TJ)),
                   static_cast<unsigned>(a.splits));
+  prof_mark(kProfLora, true, st);
   if (a.a_kmajor && a.b_kmajor)
     skinny_kernel<true, true><<<grid, SK_THREADS, 0, st>>>(a.A, a.lda, a.B, a.ldb, a.I, a.J, a.Kred, a.k_per_split,
                                                            a.part);
@@ -301,35 +302,46 @@ cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st) {
   else
     skinny_kernel<false, false><<<grid, SK_THREADS, 0, st>>>(a.A, a.lda, a.B, a.ldb, a.I, a.J, a.Kred,
                                                              a.k_per_split, a.part);
+  prof_mark(kProfLora, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_finalize_h(const float *part, int splits, int64_t M, int r, float s, float *H, uint16_t *sH,
                               uint16_t *Hs, cudaStream_t st) {
+  prof_mark(kProfLora, true, st);
   finalize_h_kernel<<<ew_blocks(M * r), 256, 0, st>>>(part, splits, M, r, s, H, sH, Hs);
+  prof_mark(kProfLora, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_split_hilo(const float *H, int64_t M, int r, uint16_t *Hs, cudaStream_t st) {
+  prof_mark(kProfLora, true, st);
   split_hilo_kernel<<<ew_blocks(M * r), 256, 0, st>>>(H, M, r, Hs);
+  prof_mark(kProfLora, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_finalize_g(const float *part, int splits, int64_t M, int r, float s, uint16_t *Gb, uint16_t *Gs,
                               cudaStream_t st) {
+  prof_mark(kProfLora, true, st);
   finalize_g_kernel<<<ew_blocks(M * r), 256, 0, st>>>(part, splits, M, r, s, Gb, Gs);
+  prof_mark(kProfLora, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_finalize_cols(const float *part, int splits, int64_t I, int64_t half, float scale, float *out,
                                  cudaStream_t st) {
+  prof_mark(kProfLora, true, st);
   finalize_cols_kernel<<<ew_blocks(I * half), 256, 0, st>>>(part, splits, I, half, scale, out);
+  prof_mark(kProfLora, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_finalize_rows(const float *part, int splits, int64_t half, int64_t J, float *out,
                                  cudaStream_t st) {
+  prof_mark(kProfLora, true, st);
   finalize_rows_kernel<<<ew_blocks(half * J), 256, 0, st>>>(part, splits, half, J, out);
+  prof_mark(kProfLora, false, st);
   return cudaGetLastError();
 }
 

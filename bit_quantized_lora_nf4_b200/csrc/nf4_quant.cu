@@ -167,8 +167,10 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
                             int *status, cudaStream_t st) {
   const int64_t ngroups = (numel + kGroupElems - 1) / kGroupElems;
+  prof_mark(kProfQuant, true, st);
   nf4_quantize_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(W, numel, codes, absmax_q,
                                                                                  group_scale, nf4_table(), status);
+  prof_mark(kProfQuant, false, st);
   return cudaGetLastError();
 }
 
@@ -177,8 +179,10 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
   const int64_t nchunk = (numel + 7) / 8;
   int64_t blocks = (nchunk + kDeqThreads - 1) / kDeqThreads;
   if (blocks > 148 * 64) blocks = 148 * 64;
+  prof_mark(kProfDequant, true, st);
   nf4_dequantize_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(codes, absmax_q, group_scale, numel,
                                                                                out, nf4_table());
+  prof_mark(kProfDequant, false, st);
   return cudaGetLastError();
 }
 

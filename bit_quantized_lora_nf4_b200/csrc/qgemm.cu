@@ -388,13 +388,17 @@ qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st) {
 
   const dim3 grid(static_cast<unsigned>(ceil_div(n_out, BN)), static_cast<unsigned>(ceil_div(a.M, BM)));
   cudaError_t e;
+  const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
   if (a.dgrad) {
     e = cudaFuncSetAttribute(qgemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    prof_mark(kind, true, st);
     if (e == cudaSuccess) qgemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, nf4_table());
   } else {
     e = cudaFuncSetAttribute(qgemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    prof_mark(kind, true, st);
     if (e == cudaSuccess) qgemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, nf4_table());
   }
+  prof_mark(kind, false, st);
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

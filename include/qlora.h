@@ -108,11 +108,11 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
  * ("QLoRA" Abstract; "Where the memory goes".)
  *   w      : the NF4 weight, rows = N, cols = K; K % 64 == 0.
  *   X      : device bf16 [M, K];  A : device bf16 [r, K];  B : device bf16 [N, r]
- *   r      : 16 <= r <= 256, r % 16 == 0;  s : the adapter scale alpha / r.
+ *   r      : 8 <= r <= 256, r % 8 == 0;  s : the adapter scale alpha / r (finite).
  *   Y      : device bf16 [M, N] (output).
  *   H_out  : optional device fp32 [M, r]; receives H = X A^T for the backward.
  *   ws     : device workspace of ws_bytes >= qlora_workspace_bytes(FWD, ...).
- * M >= 1.  M <= 16 runs the memory-bound dequant-GEMV path; larger M runs the
+ * N % 8 == 0.  M >= 1.  M <= 16 runs the memory-bound dequant-GEMV path; larger M runs the
  * tensor-core fused dequant-GEMM with the adapter term as an extra K segment of
  * the same accumulation.  fp32 accumulation; Y rounded once to bf16. */
 qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M,
@@ -156,6 +156,18 @@ uint64_t qlora_set_wait_limit(uint64_t cycles);
  * nothing ever signals, with a bound of `cycles`.  The wait must give up and
  * latch QLORA_ERR_DEVICE_TIMEOUT (read it with qlora_device_status()). */
 qlora_status qlora_selftest_wait_timeout(uint64_t cycles, void *stream);
+
+/* Kernel timing for benchmarks.  While enabled, the library records a CUDA
+ * event pair on the launch stream around each of its own kernel launches and
+ * counts the launches, per kind:
+ *   0 all kernels, 1 fused dequant-GEMM forward, 2 fused dequant-GEMM dgrad,
+ *   3 adapter (low-rank) GEMMs and their reductions, 4 quantizer,
+ *   5 dequantizer, 6 dequant-GEMV.
+ * qlora_profile_enable(1) clears the records; qlora_profile_read()
+ * synchronizes the device and returns the summed event time (ms) and the
+ * launch count of one kind.  Not thread-safe; off by default. */
+void qlora_profile_enable(int on);
+qlora_status qlora_profile_read(int kind, double *ms_total, int64_t *launches);
 
 #ifdef __cplusplus
 }
