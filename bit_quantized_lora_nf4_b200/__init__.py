@@ -32,7 +32,7 @@ EXPORTS = (
     "qlora_codes_bytes", "qlora_absmax_bytes", "qlora_group_scale_bytes", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
     "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
-    "qlora_profile_read",
+    "qlora_profile_read", "qlora_linear_fwd_noalloc",
 )
 
 # Kernel kinds of the timing hook (qlora_profile_read).
@@ -79,6 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_selftest_wait_timeout": (i32, [ctypes.c_uint64, vp]),
         "qlora_profile_enable": (None, [i32]),
         "qlora_profile_read": (i32, [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
+        "qlora_linear_fwd_noalloc": (i32, [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

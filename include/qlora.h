@@ -135,6 +135,30 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
                               const float *H_saved, uint16_t *dX, float *dA, float *dB,
                               void *ws, size_t ws_bytes, void *stream);
 
+/* Size of the library-owned scratch array used by qlora_linear_fwd_noalloc(). */
+#define QLORA_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* qlora_linear_fwd_noalloc -- the same forward as qlora_linear_fwd, for
+ * callers that cannot allocate device memory (code running where cudaMalloc
+ * is unavailable or forbidden: inside host callbacks or allocator hooks,
+ * runtimes with a memory map fixed at start-up, plugin hosts that own every
+ * allocation).  The pages have no counterpart of this call; it is a
+ * deployment convenience.
+ *   Arguments as qlora_linear_fwd, minus the workspace.  The scratch is a
+ *   QLORA_STATIC_SCRATCH_BYTES array inside the library, held on every GPU that
+ *   loads the library until the process exits; the call allocates and frees
+ *   nothing.
+ *   Returns QLORA_ERR_WORKSPACE when qlora_workspace_bytes(QLORA_OP_FWD, M, N,
+ *   K, r) exceeds QLORA_STATIC_SCRATCH_BYTES (e.g. M = 4096, r = 64 fits;
+ *   M = 8192, r = 64 does not).
+ *   The first call on a device looks up the array's device address; make that
+ *   first call before any stream capture.  Every call shares the one array
+ *   (it keeps the previous call's contents; nothing needs clearing), so calls
+ *   that overlap on the GPU race: serialize them on one stream. */
+qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_weight *w, const uint16_t *X, int64_t M,
+                                      const uint16_t *A, const uint16_t *B, int r, float s,
+                                      uint16_t *Y, float *H_out, void *stream);
+
 /* The 16 NF4 levels (ascending, fp32) as the library computes them on the
  * host: standard-normal quantiles at 8 positive and 7 negative equally spaced
  * probabilities from d = 1 - (1/32 + 1/30)/2 to 1/2, plus an exact 0,
