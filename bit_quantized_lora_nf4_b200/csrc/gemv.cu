@@ -17,6 +17,7 @@
 //             (the same bijection is applied to the tokens).  fp32 partial
 //             sums per K chunk go to the workspace.
 //   kernel 3  Y = bf16(sum over chunks + (s H) B^T), chunks summed in order.
+#include "decode.cuh"
 #include "internal.h"
 
 namespace qlora {
@@ -36,33 +37,6 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Table of T[c] = bf16(fl32(level[c] * ap)) as low-byte / high-byte words.
-__device__ __forceinline__ void gv_table(float ap, const Nf4Table &tab, uint32_t (&LO)[4], uint32_t (&HI)[4]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t p0 = pack_bf16x2(__fmul_rn(tab.level[4 * j + 0], ap), __fmul_rn(tab.level[4 * j + 1], ap));
-    const uint32_t p1 = pack_bf16x2(__fmul_rn(tab.level[4 * j + 2], ap), __fmul_rn(tab.level[4 * j + 3], ap));
-    LO[j] = __byte_perm(p0, p1, 0x6420);
-    HI[j] = __byte_perm(p0, p1, 0x7531);
-  }
-}
-
-// 8 codes (nibble i = element i) -> 4 words of bf16 pairs (elements 2i, 2i+1).
-__device__ __forceinline__ void gv_lut8(uint32_t x, const uint32_t (&LO)[4], const uint32_t (&HI)[4],
-                                        uint32_t (&o)[4]) {
-  const uint32_t sel = x & 0x77777777u;
-  const uint32_t pick = ((x >> 1) & 0x44444444u) | 0x32103210u;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t s = sel >> (16 * h);
-    const uint32_t q = pick >> (16 * h);
-    const uint32_t lo = __byte_perm(__byte_perm(LO[0], LO[1], s), __byte_perm(LO[2], LO[3], s), q);
-    const uint32_t hi = __byte_perm(__byte_perm(HI[0], HI[1], s), __byte_perm(HI[2], HI[3], s), q);
-    o[2 * h + 0] = __byte_perm(lo, hi, 0x5140);
-    o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
-  }
 }
 
 // H[m][j] = sum_k X[m][k] A[j][k]; one warp per j, all M tokens at once.
@@ -155,8 +129,8 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
       }
     }
     uint32_t LO[2][4], HI[2][4];
-    gv_table(ap[0], tab, LO[0], HI[0]);
-    gv_table(ap[1], tab, LO[1], HI[1]);
+    nf4_block_table(ap[0], tab, LO[0], HI[0]);
+    nf4_block_table(ap[1], tab, LO[1], HI[1]);
     const uint32_t words[2][8] = {{cw[0][0].x, cw[0][0].y, cw[0][0].z, cw[0][0].w, cw[0][1].x, cw[0][1].y,
                                    cw[0][1].z, cw[0][1].w},
                                   {cw[1][0].x, cw[1][0].y, cw[1][0].z, cw[1][0].w, cw[1][1].x, cw[1][1].y,
@@ -164,8 +138,8 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       uint32_t o0[4], o1[4];
-      gv_lut8(words[0][w], LO[0], HI[0], o0);
-      gv_lut8(words[1][w], LO[1], HI[1], o1);
+      nf4_lut8(words[0][w], LO[0], HI[0], o0);
+      nf4_lut8(words[1][w], LO[1], HI[1], o1);
 #pragma unroll
       for (int hs = 0; hs < 2; ++hs) {
         const int s = 2 * w + hs;                      // k16 step: in-block offsets 4s .. 4s+3

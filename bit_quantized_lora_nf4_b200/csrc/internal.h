@@ -57,6 +57,8 @@ struct QGemmArgs {
   uint16_t *out;
 };
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
+// The same product on a CTA pair (256-row tiles); launch_qgemm dispatches to it for M > 128.
+qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st);
 
 // Few-token forward: Y[M, N] = X W'^T + (s X A^T) B^T for M <= 16.
 struct GemvArgs {

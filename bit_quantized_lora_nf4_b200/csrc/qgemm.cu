@@ -30,6 +30,7 @@
 // Every mbarrier wait is bounded; on expiry the CTA latches
 // QLORA_ERR_DEVICE_TIMEOUT, lets outstanding TMA loads and MMAs land, frees
 // TMEM and exits.
+#include "decode.cuh"
 #include "internal.h"
 
 namespace qlora {
@@ -88,51 +89,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, co
       latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
       return false;
     }
-  }
-}
-
-// Byte-permute lookup of 8 NF4 codes (one 32-bit word, element i in nibble i)
-// into 4 words of bf16 pairs.  LO/HI hold the low / high bytes of the 16 table
-// entries (entry e in byte e%4 of word e/4).
-__device__ __forceinline__ void lut8(uint32_t x, const uint32_t (&LO)[4], const uint32_t (&HI)[4], uint32_t (&o)[4]) {
-  const uint32_t sel = x & 0x77777777u;                             // entry index within a half table
-  const uint32_t pick = ((x >> 1) & 0x44444444u) | 0x32103210u;     // byte i from lower (i) or upper (i+4) half
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t s = sel >> (16 * h);
-    const uint32_t q = pick >> (16 * h);
-    const uint32_t lo = __byte_perm(__byte_perm(LO[0], LO[1], s), __byte_perm(LO[2], LO[3], s), q);
-    const uint32_t hi = __byte_perm(__byte_perm(HI[0], HI[1], s), __byte_perm(HI[2], HI[3], s), q);
-    o[2 * h + 0] = __byte_perm(lo, hi, 0x5140);
-    o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
-  }
-}
-
-// Build the low/high-byte tables of T[c] = bf16(fl32(level[c] * ap)).
-__device__ __forceinline__ void build_table(float ap, const Nf4Table &tab, uint32_t (&LO)[4], uint32_t (&HI)[4]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t p0 = pack_bf16x2(__fmul_rn(tab.level[4 * j + 0], ap), __fmul_rn(tab.level[4 * j + 1], ap));
-    const uint32_t p1 = pack_bf16x2(__fmul_rn(tab.level[4 * j + 2], ap), __fmul_rn(tab.level[4 * j + 3], ap));
-    LO[j] = __byte_perm(p0, p1, 0x6420);
-    HI[j] = __byte_perm(p0, p1, 0x7531);
-  }
-}
-
-// Decode 64 codes (two 16-byte smem chunks at c_lo / c_hi) into 8 swizzled
-// 16-byte chunks at row_addr (chunk w at row_addr + ((w ^ swz) << 4)).
-__device__ __forceinline__ void decode_row(uint32_t c_lo, uint32_t c_hi, uint32_t row_addr, uint32_t swz, float ap,
-                                           const Nf4Table &tab) {
-  uint32_t LO[4], HI[4];
-  build_table(ap, tab, LO, HI);
-  const uint4 a = ld_shared_v4(c_lo);
-  const uint4 b = ld_shared_v4(c_hi);
-  const uint32_t words[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    uint32_t o[4];
-    lut8(words[w], LO, HI, o);
-    st_shared_v4(row_addr + ((static_cast<uint32_t>(w) ^ swz) << 4), o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -275,12 +231,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (DGRAD) {
           const uint32_t j = dt >> 6, nl = dt & 63, sw = nl & 7;
           const uint32_t prow = pbase + nl * 128;
-          decode_row(prow + (((2 * j) ^ sw) << 4), prow + (((2 * j + 1) ^ sw) << 4), dbase + j * 8192 + nl * 128,
+          nf4_decode_row(prow + (((2 * j) ^ sw) << 4), prow + (((2 * j + 1) ^ sw) << 4), dbase + j * 8192 + nl * 128,
                      sw, ap, tab);
         } else {
           const uint32_t sw32 = (dt >> 2) & 1;
           const uint32_t prow = pbase + dt * 32;
-          decode_row(prow + ((0u ^ sw32) << 4), prow + ((1u ^ sw32) << 4), dbase + dt * 128, dt & 7, ap, tab);
+          nf4_decode_row(prow + ((0u ^ sw32) << 4), prow + ((1u ^ sw32) << 4), dbase + dt * 128, dt & 7, ap, tab);
         }
       } else {
         // adapter weight slice, copied into the same operand layout (zero past r / past the matrix)
@@ -353,6 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace
 
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st) {
+  if (a.M > BM) return launch_qgemm_pair(a, st);
   CUtensorMap tm_act, tm_codes, tm_lact;
   const int64_t kred = a.dgrad ? a.wN : a.wK;      // reduction length of the weight segment
   const int64_t n_out = a.dgrad ? a.wK : a.wN;

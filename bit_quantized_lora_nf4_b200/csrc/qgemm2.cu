@@ -1,0 +1,356 @@
+// Fused NF4 dequant-GEMM over a CTA pair (tcgen05 cta_group::2).
+//
+// Same computation as qgemm.cu ("Where the memory goes": the 4-bit base is
+// dequantized on the fly for each forward and backward pass; the adapter term
+// is the last K segment of the same accumulation), on a 256 x 256 output tile
+// per cluster of two CTAs.  The pair's MMA (M = 256, N = 256, K = 16) takes
+// its A rows from both CTAs (128 each) and its B columns from both CTAs (128
+// each), so every CTA decodes only half of the 256-row weight tile for the same
+// tensor-core work per SM as the one-CTA kernel: the decode (ALU) cost per MMA
+// flop halves.
+//
+// Per CTA (320 threads, K-step 128 = two NF4 blocks per weight row):
+//   warp 0      TMA: its 128 activation rows (two 128B-swizzled 64-column
+//               boxes) and its 128 rows x 64 B of packed codes (64B swizzle).
+//   warp 1      TMEM allocation for the pair; in the even CTA one lane issues
+//               the pair MMA and commits to both CTAs' barriers (multicast).
+//   warps 2-9   decode: thread (row = t % 128, j = t / 128) decodes block j of
+//               its row into the 128B-swizzled operand half (K-major for the
+//               forward, MN-major for dgrad; the byte address is the same
+//               formula in both), then signals the even CTA's "decoded"
+//               barrier.  After the last step they drain this CTA's TMEM.
+// Waits are bounded; on expiry a CTA latches QLORA_ERR_DEVICE_TIMEOUT, lets
+// its outstanding loads and the pair's MMAs land, frees TMEM and exits.
+#include "decode.cuh"
+#include "internal.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int BM = 128;            // rows per CTA
+constexpr int BN = 256;            // output columns per pair (128 B-operand columns per CTA)
+constexpr int BK = 128;            // K per stage (two 64-weight blocks)
+constexpr int STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;        // 32 KB: two 64-column atoms
+constexpr int P_BYTES = 128 * BK / 2;       //  8 KB: 128 rows x 64 B of codes
+constexpr int D_BYTES = 128 * BK * 2;       // 32 KB: this CTA's half of the operand
+constexpr int HALF = 16384;                 // byte stride between the two 64-wide halves
+constexpr int STAGE_BYTES = A_BYTES + P_BYTES + D_BYTES;
+constexpr int NUM_DEC_WARPS = 8;
+constexpr int THREADS = 32 * (2 + NUM_DEC_WARPS);
+constexpr int TMEM_COLS = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint64_t kDrainLimit = 4000000000ull;
+
+struct Params {
+  int64_t M;
+  int64_t n_out;
+  int64_t ldo;
+  int64_t wN, wK;
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  const uint16_t *lora_w;
+  int r;
+  int nkb;           // weight K-steps (of 128)
+  int nls;           // adapter K-steps (of 128)
+  uint16_t *out;
+  int *status;
+  uint64_t wait_limit;
+};
+
+struct Smem {
+  uint64_t full[STAGES];       // this CTA's TMA bytes landed
+  uint64_t empty[STAGES];      // the pair's MMAs of the stage completed (multicast commit)
+  uint64_t decoded[STAGES];    // even CTA only: all 16 decode warps of the pair are done
+  uint64_t acc_full;           // the pair's accumulation completed (multicast commit)
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <bool CLUSTER_SCOPE>
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const Params &p, Smem *sm) {
+  const uint32_t a = smem_addr(bar);
+  auto poll = [&]() { return CLUSTER_SCOPE ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity); };
+  if (poll()) return true;
+  const long long t0 = clock64();
+  volatile int *abort_flag = &sm->abort_flag;
+  while (true) {
+    if (poll()) return true;
+    if (*abort_flag) return false;
+    if (static_cast<uint64_t>(clock64() - t0) > p.wait_limit) {
+      *abort_flag = 1;
+      latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+template <bool DGRAD>
+__global__ void __launch_bounds__(THREADS, 1)
+    qgemm2_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+                  const __grid_constant__ CUtensorMap tm_lact, const Params p, const Nf4Table tab) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem *sm = reinterpret_cast<Smem *>(smem + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();                              // 0 = even (MMA-issuing) CTA
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x >> 1) * (2 * BM) + rank * BM;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * BN;            // pair's first output column
+  const int64_t nb0 = n0 + rank * 128;                                  // this CTA's operand columns
+  const int nsteps = p.nkb + p.nls;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm->full[s], 1);
+      mbar_init(&sm->empty[s], 1);
+      mbar_init(&sm->decoded[s], 2 * NUM_DEC_WARPS);
+    }
+    mbar_init(&sm->acc_full, 1);
+    sm->abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_act);
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_lact);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();        // peer barriers initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (each CTA)
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (i >= STAGES && !wait_or_abort<false>(&sm->empty[s], ph ^ 1, p, sm)) break;
+        uint8_t *st = smem + s * STAGE_BYTES;
+        if (i < p.nkb) {
+          mbar_arrive_expect_tx(&sm->full[s], A_BYTES + P_BYTES);
+          tma_load_2d(st, &tm_act, &sm->full[s], i * BK, static_cast<int>(m0));
+          tma_load_2d(st + HALF, &tm_act, &sm->full[s], i * BK + 64, static_cast<int>(m0));
+          if (DGRAD)
+            tma_load_2d(st + A_BYTES, &tm_codes, &sm->full[s], static_cast<int>(nb0 / 2), i * BK);
+          else
+            tma_load_2d(st + A_BYTES, &tm_codes, &sm->full[s], i * (BK / 2), static_cast<int>(nb0));
+        } else {
+          const int ls = i - p.nkb;
+          const bool two = p.r - ls * BK > 64;
+          mbar_arrive_expect_tx(&sm->full[s], two ? A_BYTES : A_BYTES / 2);
+          tma_load_2d(st, &tm_lact, &sm->full[s], ls * BK, static_cast<int>(m0));
+          if (two) tma_load_2d(st + HALF, &tm_lact, &sm->full[s], ls * BK + 64, static_cast<int>(m0));
+        }
+        issued = i + 1;
+      }
+      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+        mbar_wait(&sm->full[j % STAGES], (j / STAGES) & 1, kDrainLimit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, 0, DGRAD ? 1 : 0);
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!wait_or_abort<true>(&sm->decoded[s], ph, p, sm)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_addr(smem + s * STAGE_BYTES);
+        const uint32_t d_base = a_base + A_BYTES + P_BYTES;
+        int nk = BK / 16;
+        if (i >= p.nkb) {
+          const int rem = p.r - (i - p.nkb) * BK;
+          nk = rem >= BK ? BK / 16 : (rem + 15) / 16;
+        }
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
+          const uint64_t adesc = sdesc_sw128(a_base + koff, 16, 1024);
+          const uint64_t bdesc = DGRAD ? sdesc_sw128(d_base + kk * 2048, HALF, 1024)
+                                       : sdesc_sw128(d_base + koff, 16, 1024);
+          tc_mma_bf16_pair(tmem, adesc, bdesc, IDESC, (i | kk) != 0 ? 1u : 0u);
+        }
+        tc_commit_pair_mc(&sm->empty[s], 0x3);
+      }
+      tc_commit_pair_mc(&sm->acc_full, 0x3);
+    }
+  } else {
+    // ------------------------------------------------------------ decoders (each CTA)
+    const int dt = threadIdx.x - 64;          // 0..255
+    const int row = dt & 127;                 // operand row within this CTA's half
+    const int jb = dt >> 7;                   // which of the stage's two blocks
+    const int64_t kblocks = p.wK / kBlock;
+    auto block_index = [&](int i, int64_t *idx) -> bool {
+      int64_t n, kb;
+      if (DGRAD) {
+        n = static_cast<int64_t>(i) * BK + row;
+        kb = nb0 / kBlock + jb;
+      } else {
+        n = nb0 + row;
+        kb = 2 * static_cast<int64_t>(i) + jb;
+      }
+      *idx = n * kblocks + kb;
+      return n < p.wN && kb < kblocks;
+    };
+    uint32_t q_next = 0;
+    float s_next = 0.0f;
+    {
+      int64_t idx;
+      if (p.nkb > 0 && block_index(0, &idx)) {
+        q_next = __ldg(p.absmax_q + idx);
+        s_next = __ldg(p.group_scale + (idx >> 8));
+      }
+    }
+    const uint32_t swz64 = (row >> 1) & 3;    // 64B swizzle of the code tile
+    const uint32_t swz128 = row & 7;          // 128B swizzle of the operand
+    for (int i = 0; i < nsteps; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (i / STAGES) & 1;
+      const float ap = __fmul_rn(static_cast<float>(q_next), s_next);
+      q_next = 0;
+      s_next = 0.0f;
+      if (i + 1 < p.nkb) {
+        int64_t idx;
+        if (block_index(i + 1, &idx)) {
+          q_next = __ldg(p.absmax_q + idx);
+          s_next = __ldg(p.group_scale + (idx >> 8));
+        }
+      }
+      if (!__all_sync(0xffffffffu, wait_or_abort<false>(&sm->full[s], ph, p, sm))) break;
+      const uint32_t st = smem_addr(smem + s * STAGE_BYTES);
+      const uint32_t prow = st + A_BYTES + row * 64;
+      const uint32_t drow = st + A_BYTES + P_BYTES + jb * HALF + row * 128;
+      if (i < p.nkb) {
+        nf4_decode_row(prow + (((2 * jb) ^ swz64) << 4), prow + (((2 * jb + 1) ^ swz64) << 4), drow, swz128, ap,
+                       tab);
+      } else {
+        // adapter weight slice in the same operand layout; zero past r / past the matrix
+        const int64_t base_r = static_cast<int64_t>(i - p.nkb) * BK + 64 * jb;
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (DGRAD) {
+            const int64_t rr = static_cast<int64_t>(i - p.nkb) * BK + row;
+            const int64_t kk = nb0 + 64 * jb + 8 * c;
+            if (rr < p.r && kk < p.wK) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + rr * p.wK + kk));
+          } else {
+            const int64_t n = nb0 + row;
+            const int64_t rr = base_r + 8 * c;
+            if (n < p.wN && rr < p.r) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + n * p.r + rr));
+          }
+          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz128) << 4), v.x, v.y, v.z, v.w);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&sm->decoded[s]), 0));
+    }
+
+    // ------------------------------------------------------------ epilogue (each CTA, its 128 rows)
+    const bool acc_ok = mbar_wait(&sm->acc_full, 0, kDrainLimit);
+    tc_fence_after();
+    volatile int *abort_flag = &sm->abort_flag;
+    if (__all_sync(0xffffffffu, acc_ok && *abort_flag == 0)) {
+      const int quarter = warp & 3;
+      const int half = (warp - 2) >> 2;
+      const int64_t orow_i = m0 + quarter * 32 + lane;
+      uint16_t *orow = p.out + orow_i * p.ldo;
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col0 = half * 128 + cc * 32;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
+        tmem_ld_wait();
+        if (orow_i < p.M) {
+          const int64_t c0 = n0 + col0;
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          if (c0 + 32 <= p.n_out && (p.ldo & 7) == 0) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < p.n_out) orow[c0 + j] = static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1)));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();        // the peer is done with this CTA's shared memory and TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
+  CUtensorMap tm_act, tm_codes, tm_lact;
+  const int64_t kred = a.dgrad ? a.wN : a.wK;
+  const int64_t n_out = a.dgrad ? a.wK : a.wN;
+  const uint64_t codes_row = static_cast<uint64_t>(a.wK / 2);
+  bool ok = make_tmap_2d(&tm_act, a.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kred, a.M, kred * 2, 64, BM,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_tmap_2d(&tm_codes, a.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_row, a.wN, codes_row, 64, 128,
+                          CU_TENSOR_MAP_SWIZZLE_64B);
+  ok = ok && make_tmap_2d(&tm_lact, a.lora_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.r, a.M,
+                          static_cast<uint64_t>(a.r) * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return QLORA_ERR_CUDA;
+
+  Params p{};
+  p.M = a.M;
+  p.n_out = n_out;
+  p.ldo = n_out;
+  p.wN = a.wN;
+  p.wK = a.wK;
+  p.absmax_q = a.absmax_q;
+  p.group_scale = a.group_scale;
+  p.lora_w = a.lora_w;
+  p.r = a.r;
+  p.nkb = static_cast<int>(ceil_div(kred, BK));
+  p.nls = static_cast<int>(ceil_div(a.r, BK));
+  p.out = a.out;
+  p.status = device_status_ptr();
+  p.wait_limit = wait_limit();
+  if (!p.status) return QLORA_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * ceil_div(a.M, 2 * BM)), static_cast<unsigned>(ceil_div(n_out, BN)));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const Nf4Table tab = nf4_table();
+  const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
+  cudaError_t e;
+  if (a.dgrad) {
+    e = cudaFuncSetAttribute(qgemm2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    prof_mark(kind, true, st);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<true>, tm_act, tm_codes, tm_lact, p, tab);
+  } else {
+    e = cudaFuncSetAttribute(qgemm2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    prof_mark(kind, true, st);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<false>, tm_act, tm_codes, tm_lact, p, tab);
+  }
+  prof_mark(kind, false, st);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace qlora

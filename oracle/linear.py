@@ -41,15 +41,27 @@ def lora_linear_fwd(Wd, X, A, B, s):
     return Y, H
 
 
-def lora_linear_bwd(Wd, X, dY, A, B, s):
-    """Returns (dX, dA, dB) in fp64; W' receives no gradient."""
-    Wd, X, dY, A, B = _f64(Wd), _f64(X), _f64(dY), _f64(A), _f64(B)
+def lora_input_grad(Wd, dY, A, B, s):
+    """dX = dY W' + (s dY B) A.  Row m of dX depends only on row m of dY."""
+    Wd, dY, A, B = _f64(Wd), _f64(dY), _f64(A), _f64(B)
+    s = float(np.float32(s))
+    G = s * (dY @ B)
+    return dY @ Wd + G @ A
+
+
+def lora_adapter_grads(X, dY, A, B, s):
+    """(dA, dB) = ((s dY B)^T X, s dY^T (X A^T)): the gradients of the trainable adapters."""
+    X, dY, A, B = _f64(X), _f64(dY), _f64(A), _f64(B)
     s = float(np.float32(s))
     H = X @ A.T
     G = s * (dY @ B)
-    dX = dY @ Wd + G @ A
-    dA = G.T @ X
-    dB = s * (dY.T @ H)
+    return G.T @ X, s * (dY.T @ H)
+
+
+def lora_linear_bwd(Wd, X, dY, A, B, s):
+    """Returns (dX, dA, dB) in fp64; W' receives no gradient."""
+    dX = lora_input_grad(Wd, dY, A, B, s)
+    dA, dB = lora_adapter_grads(X, dY, A, B, s)
     return dX, dA, dB
 
 

@@ -44,6 +44,9 @@ def test_small_config(lib):
     (96, 512, 448, 128),
     (200, 128, 640, 256),
     (64, 8, 64, 8),           # minimal shapes
+    (129, 392, 640, 64),      # first size on the CTA-pair kernel (one pair, odd CTA mostly empty)
+    (256, 512, 1024, 32),     # exactly one pair tile
+    (520, 1800, 1344, 16),    # several pairs, ragged N and K (K % 128 != 0)
 ])
 def test_ragged_shapes(lib, M, N, K, r):
     _run_case(qi.LinearCase(f"ragged_{M}_{N}_{K}_{r}", M, N, K, r, 16.0, 100 + M + N + K + r))
@@ -74,3 +77,29 @@ def test_adapter_only_special_case(lib):
     assert rel(f64(Y), Yr) <= TOL
     assert torch.count_nonzero(dB).item() == 0
     assert rel(f64(dX), f64(d["dY"]) @ Wd) <= TOL
+
+
+@pytest.mark.parametrize("case", qi.LLAMA7B, ids=lambda c: c.name)
+def test_llama7b_projection_sampled(lib, case):
+    """Full-size projection (M = 4096, r = 64) in the launch configuration the
+    bench times; Y and dX checked on 48 sampled token rows against the oracle,
+    dA and dB in full."""
+    d = qi.make_linear(case)
+    oq, Wd = oracle_weight(d["W"])
+    w = gpu_weight(d["W"])
+    assert_weight_bits(w, oq)
+    X, A, B, dY = (d[k].cuda() for k in ("X", "A", "B", "dY"))
+    Y, H = q.linear_fwd(w, X, A, B, d["s"])
+    dX, dA, dB = q.linear_bwd(w, X, dY, A, B, d["s"], H=H)
+    torch.cuda.synchronize()
+    assert q.device_status() == 0
+    rows = np.random.default_rng(case.seed).choice(case.M, 48, replace=False)
+    rows.sort()
+    A64, B64 = f64(d["A"]), f64(d["B"])
+    Yr, _ = olin.lora_linear_fwd(Wd, f64(d["X"][rows]), A64, B64, d["s"])
+    dXr = olin.lora_input_grad(Wd, f64(d["dY"][rows]), A64, B64, d["s"])
+    dAr, dBr = olin.lora_adapter_grads(f64(d["X"]), f64(d["dY"]), A64, B64, d["s"])
+    errs = {"Y": rel(f64(Y[rows]), Yr), "dX": rel(f64(dX[rows]), dXr), "dA": rel(f64(dA), dAr),
+            "dB": rel(f64(dB), dBr)}
+    for k, e in errs.items():
+        assert e <= TOL, (k, errs)
