@@ -269,16 +269,25 @@ def measure_extras(q, rep, dev, pk, barrier):
             Y = torch.empty((M, case.N), dtype=torch.bfloat16, device=dev)
             ws = torch.empty(q.workspace_bytes(q.QLORA_OP_FWD, M, case.N, case.K, case.r), dtype=torch.uint8,
                              device=dev)
-            it = [0]
 
-            def gv():
-                w = copies[it[0] % ncopy]
-                it[0] += 1
-                q.linear_fwd(w, X, c["A"], c["B"], c["s"], save_h=False, out=Y, workspace=ws)
+            def calls():
+                for w in copies:
+                    q.linear_fwd(w, X, c["A"], c["B"], c["s"], save_h=False, out=Y, workspace=ws)
+            # one CUDA graph holds one call per weight copy, so the timing sees the GPU,
+            # not the Python/ctypes call overhead of these few-microsecond calls
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                calls()
+            torch.cuda.current_stream().wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                calls()
             for _ in range(3):
-                gv()
-            reps = 2 * ncopy
-            ms = timed(gv, reps, barrier) / reps
+                graph.replay()
+            reps = 4
+            ms = timed(graph.replay, reps, barrier) / (reps * ncopy)
+            del graph
             nbytes = c["w"].nbytes() + 2 * case.r * (case.N + case.K) + 2 * M * (case.N + case.K)
             tot_bytes += nbytes
             tot_ms += ms
@@ -286,7 +295,9 @@ def measure_extras(q, rep, dev, pk, barrier):
         gbs = tot_bytes / (tot_ms * 1e-3) / 1e9
         res[str(M)] = {"value": round(gbs, 1), "frac": round(gbs / pk["hbm"], 4), "us_per_call_avg": round(
             1e3 * tot_ms / len(rep.cases), 2)}
-    out["gemv"] = {"unit": "GB/s", "tokens": res, "note": "packed weight + adapters + X + Y bytes per call"}
+    out["gemv"] = {"unit": "GB/s", "tokens": res,
+                   "note": "packed weight + adapters + X + Y bytes per call; calls replayed from a CUDA graph, "
+                           "weights rotated over copies totalling > 400 MB (beyond L2)"}
     return out
 
 

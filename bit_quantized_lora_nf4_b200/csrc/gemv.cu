@@ -6,8 +6,7 @@
 // whole cost, so the weight is decoded straight into tensor-core register
 // fragments and never touches shared memory.
 //
-//   kernel 1  H = X A^T (fp32 [M, r]); one warp per adapter row.
-//   kernel 2  per CTA: 64 weight rows x one 1024-wide K chunk.  mma.sync
+//   kernel 1  per CTA: 64 weight rows x one 1024-wide K chunk.  mma.sync
 //             m16n8k16 with the weight as the 16-row A operand and the tokens
 //             as the 8-column B operand (two column tiles for M > 8).  Each
 //             thread owns one whole 64-weight block of two rows, builds that
@@ -15,8 +14,12 @@
 //             byte permutes.  Within a 256-wide macro-step the K index of the
 //             fragment slots is permuted so that thread (g, c) covers block c
 //             (the same bijection is applied to the tokens).  fp32 partial
-//             sums per K chunk go to the workspace.
-//   kernel 3  Y = bf16(sum over chunks + (s H) B^T), chunks summed in order.
+//             sums per K chunk go to the workspace.  The same CTAs also form
+//             the adapter prologue's partial sums H_z = X_z A^T over their K
+//             chunk (adapter rows spread over the CTAs of a chunk).
+//   kernel 2  per CTA of 64 output rows: s*H = s * sum_z H_z into shared
+//             memory, then Y = bf16(sum_z Y_z + (s H) B^T); all sums in a
+//             fixed order (deterministic).
 #include "decode.cuh"
 #include "internal.h"
 
@@ -39,66 +42,70 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// H[m][j] = sum_k X[m][k] A[j][k]; one warp per j, all M tokens at once.
-__global__ void __launch_bounds__(256) gemv_h_kernel(const uint16_t *__restrict__ X, const uint16_t *__restrict__ A,
-                                                     int M, int K, int r, float *__restrict__ H) {
-  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (j >= r) return;
-  float acc[GV_TOK];
-#pragma unroll
-  for (int m = 0; m < GV_TOK; ++m) acc[m] = 0.0f;
-  for (int k = lane * 8; k < K; k += 256) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(A + static_cast<int64_t>(j) * K + k));
-    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-    for (int m = 0; m < GV_TOK; ++m) {
-      if (m < M) {
-        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(m) * K + k));
-        const uint32_t xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc[m] = fmaf(__uint_as_float(xv[e] << 16), __uint_as_float(av[e] << 16), acc[m]);
-          acc[m] = fmaf(__uint_as_float(xv[e] & 0xFFFF0000u), __uint_as_float(av[e] & 0xFFFF0000u), acc[m]);
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < GV_TOK; ++m) {
-    float v = acc[m];
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if (lane == 0 && m < M) H[static_cast<int64_t>(m) * r + j] = v;
-  }
-}
-
 template <int NT>   // number of 8-token column tiles (1: M <= 8, 2: M <= 16)
 __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *__restrict__ X, int M, int64_t N,
                                                                int64_t K, const uint8_t *__restrict__ codes,
                                                                const uint8_t *__restrict__ absmax_q,
                                                                const float *__restrict__ group_scale,
-                                                               float *__restrict__ part, Nf4Table tab) {
-  // X chunk, permuted: word (8 B = 4 tokens-values of one token) at
-  // [macro][s][c][tok], so that the 32 lanes of a step read 32 distinct words.
-  __shared__ __align__(16) uint2 xs[GV_KC / GV_MACRO][16][4][NT * 8];
+                                                               const uint16_t *__restrict__ A, int r,
+                                                               float *__restrict__ part, float *__restrict__ hpart,
+                                                               Nf4Table tab) {
+  // X chunk, permuted: the 8-byte word holding X[tok][k .. k+3] for in-chunk
+  // k = 256 ms + 64 c + 4 s sits at xs[ms][s][tok][c], so the 32 lanes of one
+  // k16 step (token g, block c) read 32 consecutive words: no bank conflicts.
+  __shared__ __align__(16) uint2 xs[GV_KC / GV_MACRO][16][NT * 8][4];
   const int64_t n_base = static_cast<int64_t>(blockIdx.x) * GV_ROWS;
   const int64_t k_base = static_cast<int64_t>(blockIdx.y) * GV_KC;
   const int64_t kc = (K - k_base) < GV_KC ? (K - k_base) : GV_KC;   // multiple of 64
   const int nmacro = static_cast<int>((kc + GV_MACRO - 1) / GV_MACRO);
 
-  // Stage X[0:M, k_base : k_base+kc] (zero for tokens >= M or k past the chunk).
-  for (int w = threadIdx.x; w < (GV_KC / 4) * NT * 8; w += GV_THREADS) {
+  // Stage X[0:M, k_base : k_base+kc] with 16-byte loads (8 elements = two words);
+  // zero for tokens >= M or k past the chunk.
+  for (int w = threadIdx.x; w < (GV_KC / 8) * NT * 8; w += GV_THREADS) {
     const int tok = w % (NT * 8);
-    const int kq = w / (NT * 8);              // which 4-element group of the chunk
-    const int k = kq * 4;
+    const int k = (w / (NT * 8)) * 8;
     const int ms = k / GV_MACRO, in = k % GV_MACRO;
-    const int c = in / 64, s = (in % 64) / 4;
-    uint2 v = make_uint2(0, 0);
-    if (tok < M && k < kc) v = __ldg(reinterpret_cast<const uint2 *>(X + static_cast<int64_t>(tok) * K + k_base + k));
-    xs[ms][s][c][tok] = v;
+    const int c = in / 64, s = (in % 64) / 4;           // s is even
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (tok < M && k < kc) v = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(tok) * K + k_base + k));
+    xs[ms][s][tok][c] = make_uint2(v.x, v.y);
+    xs[ms][s + 1][tok][c] = make_uint2(v.z, v.w);
   }
   __syncthreads();
+
+  // Adapter prologue partials for this K chunk: hpart[z][m][j] = sum_k X[m][k] A[j][k],
+  // for the adapter rows j = blockIdx.x, blockIdx.x + gridDim.x, ...  Thread t
+  // takes token t % 16 and every 8th 4-element word of the chunk; the 8 word
+  // groups are summed in a fixed order through shared memory.
+  {
+    __shared__ float hred[8][GV_TOK];
+    const int tok = threadIdx.x & 15, grp = threadIdx.x >> 4;
+    const int nwords = static_cast<int>(kc / 4);
+    for (int j = blockIdx.x; j < r; j += gridDim.x) {
+      float acc_h = 0.0f;
+      if (tok < M && tok < NT * 8) {
+        for (int qw = grp; qw < nwords; qw += 8) {
+          const int k = qw * 4;
+          const int ms = k / GV_MACRO, in = k % GV_MACRO;
+          const uint2 xv = xs[ms][(in % 64) / 4][tok][in / 64];
+          const uint2 av = __ldg(reinterpret_cast<const uint2 *>(A + static_cast<int64_t>(j) * K + k_base + k));
+          acc_h = fmaf(__uint_as_float(xv.x << 16), __uint_as_float(av.x << 16), acc_h);
+          acc_h = fmaf(__uint_as_float(xv.x & 0xFFFF0000u), __uint_as_float(av.x & 0xFFFF0000u), acc_h);
+          acc_h = fmaf(__uint_as_float(xv.y << 16), __uint_as_float(av.y << 16), acc_h);
+          acc_h = fmaf(__uint_as_float(xv.y & 0xFFFF0000u), __uint_as_float(av.y & 0xFFFF0000u), acc_h);
+        }
+      }
+      hred[grp][tok] = acc_h;
+      __syncthreads();
+      if (threadIdx.x < M) {
+        float v = 0.0f;
+#pragma unroll
+        for (int gq = 0; gq < 8; ++gq) v += hred[gq][threadIdx.x];
+        hpart[(static_cast<int64_t>(blockIdx.y) * M + threadIdx.x) * r + j] = v;
+      }
+      __syncthreads();
+    }
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -110,11 +117,10 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
 
-  for (int ms = 0; ms < nmacro; ++ms) {
+  // codes / constants of one macro-step for rows row0 and row0 + 8 (zero when out of range)
+  auto fetch = [&](int ms, uint4 (&cw)[2][2], float (&ap)[2]) {
     const int64_t kb = (k_base + static_cast<int64_t>(ms) * GV_MACRO) / kBlock + c;
-    const bool kvalid = (static_cast<int64_t>(ms) * GV_MACRO + 64 * c) < kc;
-    uint4 cw[2][2];
-    float ap[2];
+    const bool kvalid = ms < nmacro && (static_cast<int64_t>(ms) * GV_MACRO + 64 * c) < kc;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int64_t n = row0 + 8 * h;
@@ -128,6 +134,12 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
         ap[h] = __fmul_rn(static_cast<float>(__ldg(absmax_q + bi)), __ldg(group_scale + (bi >> 8)));
       }
     }
+  };
+  uint4 cw[2][2], cn[2][2];
+  float ap[2], an[2];
+  fetch(0, cw, ap);
+  for (int ms = 0; ms < nmacro; ++ms) {
+    fetch(ms + 1, cn, an);                 // next macro-step's loads in flight while this one decodes
     uint32_t LO[2][4], HI[2][4];
     nf4_block_table(ap[0], tab, LO[0], HI[0]);
     nf4_block_table(ap[1], tab, LO[1], HI[1]);
@@ -145,10 +157,16 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
         const int s = 2 * w + hs;                      // k16 step: in-block offsets 4s .. 4s+3
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const uint2 xv = xs[ms][s][c][t * 8 + g];
+          const uint2 xv = xs[ms][s][t * 8 + g][c];
           mma16816(acc[t], o0[2 * hs], o1[2 * hs], o0[2 * hs + 1], o1[2 * hs + 1], xv.x, xv.y);
         }
       }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      cw[h][0] = cn[h][0];
+      cw[h][1] = cn[h][1];
+      ap[h] = an[h];
     }
   }
 
@@ -166,24 +184,36 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
   }
 }
 
-// Y[m][n] = bf16( sum_z part[z][n][m] + sum_j fl32(s*H[m][j]) B[n][j] ).
-__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restrict__ part, int nchunks, int M,
-                                                          int64_t N, const float *__restrict__ H,
-                                                          const uint16_t *__restrict__ B, int r, float s,
-                                                          uint16_t *__restrict__ Y) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= N * M) return;
-  const int64_t n = idx / M;
-  const int m = static_cast<int>(idx % M);
+constexpr int GV_RED_ROWS = 64;
+
+// Per CTA of 64 output rows: sH[m][j] = fl32(s * sum_z hpart[z][m][j]) into
+// shared memory (the CTA with blockIdx.x == 0 also writes the unscaled H when
+// asked), then Y[m][n] = bf16( sum_z part[z][n][m] + sum_j sH[m][j] B[n][j] ).
+__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restrict__ part,
+                                                          const float *__restrict__ hpart, int nchunks, int M,
+                                                          int64_t N, const uint16_t *__restrict__ B, int r, float s,
+                                                          float *__restrict__ H_out, uint16_t *__restrict__ Y) {
+  __shared__ float sh[GV_TOK * 256];
+  for (int e = threadIdx.x; e < M * r; e += blockDim.x) {
+    float h = 0.0f;
+    for (int z = 0; z < nchunks; ++z) h += hpart[static_cast<int64_t>(z) * M * r + e];
+    sh[e] = __fmul_rn(s, h);
+    if (H_out && blockIdx.x == 0) H_out[e] = h;
+  }
+  __syncthreads();
   const int ldp = (M + 1) & ~1;
-  float v = 0.0f;
-  for (int z = 0; z < nchunks; ++z) v += part[(static_cast<int64_t>(z) * N + n) * ldp + m];
-  float l = 0.0f;
-  for (int j = 0; j < r; ++j)
-    l = fmaf(__fmul_rn(s, H[static_cast<int64_t>(m) * r + j]),
-             __uint_as_float(static_cast<uint32_t>(B[n * r + j]) << 16), l);
-  const __nv_bfloat16 b = __float2bfloat16_rn(v + l);
-  Y[static_cast<int64_t>(m) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
+  const int64_t n_base = static_cast<int64_t>(blockIdx.x) * GV_RED_ROWS;
+  for (int idx = threadIdx.x; idx < GV_RED_ROWS * M; idx += blockDim.x) {
+    const int64_t n = n_base + idx % GV_RED_ROWS;
+    const int m = idx / GV_RED_ROWS;
+    if (n >= N) continue;
+    float v = 0.0f;
+    for (int z = 0; z < nchunks; ++z) v += part[(static_cast<int64_t>(z) * N + n) * ldp + m];
+    float l = 0.0f;
+    for (int j = 0; j < r; ++j) l = fmaf(sh[m * r + j], __uint_as_float(static_cast<uint32_t>(B[n * r + j]) << 16), l);
+    const __nv_bfloat16 b = __float2bfloat16_rn(v + l);
+    Y[static_cast<int64_t>(m) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
+  }
 }
 
 }  // namespace
@@ -194,26 +224,25 @@ size_t gemv_partial_bytes(int64_t M, int64_t N, int64_t K) {
   return static_cast<size_t>(ceil_div(K, GV_KC) * N * ((M + 1) & ~int64_t(1))) * 4;
 }
 
+size_t gemv_hpartial_bytes(int64_t M, int64_t K, int r) {
+  return static_cast<size_t>(ceil_div(K, GV_KC) * M * r) * 4;
+}
+
 qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st) {
   if (a.M < 1 || a.M > kGemvMaxTokens) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  float *H = a.H_out ? a.H_out : a.h_ws;
   const int64_t nchunks = ceil_div(a.wK, GV_KC);
-  prof_mark(kProfGemv, true, st);
-  gemv_h_kernel<<<static_cast<unsigned>(ceil_div(a.r, 8)), 256, 0, st>>>(a.X, a.A, static_cast<int>(a.M),
-                                                                         static_cast<int>(a.wK), a.r, H);
-  prof_mark(kProfGemv, false, st);
   const dim3 grid(static_cast<unsigned>(ceil_div(a.wN, GV_ROWS)), static_cast<unsigned>(nchunks));
   prof_mark(kProfGemv, true, st);
   if (a.M <= 8)
     gemv_main_kernel<1><<<grid, GV_THREADS, 0, st>>>(a.X, static_cast<int>(a.M), a.wN, a.wK, a.codes, a.absmax_q,
-                                                     a.group_scale, a.part, nf4_table());
+                                                     a.group_scale, a.A, a.r, a.part, a.hpart, nf4_table());
   else
     gemv_main_kernel<2><<<grid, GV_THREADS, 0, st>>>(a.X, static_cast<int>(a.M), a.wN, a.wK, a.codes, a.absmax_q,
-                                                     a.group_scale, a.part, nf4_table());
+                                                     a.group_scale, a.A, a.r, a.part, a.hpart, nf4_table());
   prof_mark(kProfGemv, false, st);
   prof_mark(kProfGemv, true, st);
-  gemv_reduce_kernel<<<static_cast<unsigned>(ceil_div(a.wN * a.M, 256)), 256, 0, st>>>(
-      a.part, static_cast<int>(nchunks), static_cast<int>(a.M), a.wN, H, a.B, a.r, a.s, a.Y);
+  gemv_reduce_kernel<<<static_cast<unsigned>(ceil_div(a.wN, GV_RED_ROWS)), 256, 0, st>>>(
+      a.part, a.hpart, static_cast<int>(nchunks), static_cast<int>(a.M), a.wN, a.B, a.r, a.s, a.H_out, a.Y);
   prof_mark(kProfGemv, false, st);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

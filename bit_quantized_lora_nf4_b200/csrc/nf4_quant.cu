@@ -15,6 +15,7 @@
 //   c_g = max a_b over 256 blocks;  S_g = fl32(c_g / 255)
 //   q_b = min(255, rint(fl32(a_b / S_g)))  (0 when S_g == 0)
 //   W'  = bf16(fl32(level[code] * fl32(q_b * S_g)))
+#include "decode.cuh"
 #include "internal.h"
 
 namespace qlora {
@@ -123,9 +124,9 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float
   if (bad) latch_status(status, QLORA_ERR_NONFINITE);
 }
 
-// Each thread turns one 32-bit word of codes (8 weights) into one 16-byte bf16
-// chunk.  Levels come from a 16-entry shared-memory copy (conflict-free: at
-// most 16 distinct words, one per bank).
+// Each thread turns 16 bytes of codes (32 weights, half of one block) into
+// 64 bytes of bf16 through the block's byte-permute table (decode.cuh), so a
+// warp streams 512 B in and 2 KB out per iteration.
 constexpr int kDeqThreads = 256;
 
 __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8_t *__restrict__ codes,
@@ -133,31 +134,109 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
                                                                      const float *__restrict__ group_scale,
                                                                      int64_t numel, uint16_t *__restrict__ out,
                                                                      Nf4Table tab) {
-  __shared__ float s_lv[16];
-  if (threadIdx.x < 16) s_lv[threadIdx.x] = tab.level[threadIdx.x];
-  __syncthreads();
-  const int64_t nchunk = (numel + 7) / 8;
+  const int64_t nchunk = (numel + 31) / 32;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nchunk; i += stride) {
-    const int64_t e0 = i * 8;
+    const int64_t e0 = i * 32;
     const int64_t blk = e0 >> 6;
     const float ap = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(group_scale + (blk >> 8)));
-    if (e0 + 8 <= numel) {
-      const uint32_t w = __ldcs(reinterpret_cast<const unsigned int *>(codes) + i);
-      uint32_t o[4];
+    uint32_t LO[4], HI[4];
+    nf4_block_table(ap, tab, LO, HI);
+    if (e0 + 32 <= numel) {
+      const uint4 c = __ldcs(reinterpret_cast<const uint4 *>(codes) + i);
+      const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+      uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float lo = __fmul_rn(s_lv[(w >> (8 * j)) & 15u], ap);
-        const float hi = __fmul_rn(s_lv[(w >> (8 * j + 4)) & 15u], ap);
-        o[j] = pack_bf16x2(lo, hi);
+      for (int w = 0; w < 4; ++w) {
+        uint32_t o[4];
+        nf4_lut8(words[w], LO, HI, o);
+        __stcs(dst + w, make_uint4(o[0], o[1], o[2], o[3]));
       }
-      __stcs(reinterpret_cast<uint4 *>(out + e0), make_uint4(o[0], o[1], o[2], o[3]));
     } else {
       for (int64_t e = e0; e < numel; ++e) {
-        const uint32_t c = (codes[e >> 1] >> (4 * (e & 1))) & 15u;
-        const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(s_lv[c], ap));
-        out[e] = *reinterpret_cast<const uint16_t *>(&b);
+        const uint32_t cd = (codes[e >> 1] >> (4 * (e & 1))) & 15u;
+        uint32_t o[4];
+        nf4_lut8(cd, LO, HI, o);                 // code in nibble 0 -> T[cd] in the low half of o[0]
+        out[e] = static_cast<uint16_t>(o[0] & 0xFFFFu);
       }
+    }
+  }
+}
+
+// Persistent dequantizer for whole chunks of 8192 weights (128 blocks): the
+// 4 KB of codes arrive by a 1-D bulk copy, 256 threads decode 32 weights each
+// into a 16 KB shared buffer, and one thread streams it out with a bulk store.
+// Two buffers of each kind overlap the next chunk's load and the previous
+// chunk's store with the current decode.
+constexpr int kDqChunk = 8192;
+constexpr int kDqCodeBytes = kDqChunk / 2;
+constexpr int kDqOutBytes = kDqChunk * 2;
+
+__global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const uint8_t *__restrict__ codes,
+                                                                          const uint8_t *__restrict__ absmax_q,
+                                                                          const float *__restrict__ group_scale,
+                                                                          int64_t nchunks, uint16_t *__restrict__ out,
+                                                                          Nf4Table tab, int *status,
+                                                                          uint64_t wait_limit) {
+  __shared__ __align__(128) uint8_t cbuf[2][kDqCodeBytes];
+  __shared__ __align__(128) uint8_t obuf[2][kDqOutBytes];
+  __shared__ uint64_t bar[2];
+  __shared__ int abort_flag;
+  const int t = threadIdx.x;
+  if (t == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int64_t first = blockIdx.x;
+  const int64_t step = gridDim.x;
+  if (t == 0 && first < nchunks) {
+    mbar_arrive_expect_tx(&bar[0], kDqCodeBytes);
+    bulk_load(cbuf[0], codes + first * kDqCodeBytes, kDqCodeBytes, &bar[0]);
+  }
+  int it = 0;
+  int last_issued = first < nchunks ? 0 : -1;       // iteration index of the newest load (thread 0)
+  for (int64_t ch = first; ch < nchunks; ch += step, ++it) {
+    const int b = it & 1;
+    // issue the next chunk's load into the other buffer (its previous contents were consumed last iteration)
+    if (t == 0 && ch + step < nchunks) {
+      mbar_arrive_expect_tx(&bar[b ^ 1], kDqCodeBytes);
+      bulk_load(cbuf[b ^ 1], codes + (ch + step) * kDqCodeBytes, kDqCodeBytes, &bar[b ^ 1]);
+      last_issued = it + 1;
+    }
+    const int64_t blk = (ch * kDqChunk + t * 32) >> 6;
+    const float ap = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(group_scale + (blk >> 8)));
+    uint32_t LO[4], HI[4];
+    nf4_block_table(ap, tab, LO, HI);
+    // obuf[b] was last used by the store issued two iterations ago
+    if (t == 0) bulk_wait_read<1>();
+    const bool ok = mbar_wait(&bar[b], (it >> 1) & 1, wait_limit);
+    if (!ok) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    const uint4 cw = ld_shared_v4(smem_addr(cbuf[b] + t * 16));
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t o[4];
+      nf4_lut8(words[w], LO, HI, o);
+      st_shared_v4(smem_addr(obuf[b] + t * 64 + w * 16), o[0], o[1], o[2], o[3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0) {
+      bulk_store(out + ch * kDqChunk, obuf[b], kDqOutBytes);
+      bulk_commit();
+    }
+  }
+  if (t == 0) {
+    bulk_wait_all<0>();
+    if (abort_flag) {
+      latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
+      // let the loads still in flight (iterations it .. last_issued) land before exiting
+      for (int j = it; j <= last_issued; ++j) mbar_wait(&bar[j & 1], (j >> 1) & 1, 4000000000ull);
     }
   }
 }
@@ -176,12 +255,26 @@ cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale, int64_t numel,
                               uint16_t *out, cudaStream_t st) {
-  const int64_t nchunk = (numel + 7) / 8;
-  int64_t blocks = (nchunk + kDeqThreads - 1) / kDeqThreads;
-  if (blocks > 148 * 64) blocks = 148 * 64;
+  // whole double-quantization groups (two chunks each) on the bulk path
+  const int64_t nfull = (numel / (kBlock * kGroup)) * (kBlock * kGroup / kDqChunk);
   prof_mark(kProfDequant, true, st);
-  nf4_dequantize_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(codes, absmax_q, group_scale, numel,
-                                                                               out, nf4_table());
+  if (nfull > 0) {
+    int *status = device_status_ptr();
+    int64_t blocks = nfull < 148 * 4 ? nfull : 148 * 4;
+    nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(
+        codes, absmax_q, group_scale, nfull, out, nf4_table(), status, wait_limit());
+  }
+  const int64_t done = nfull * kDqChunk;
+  if (done < numel) {
+    // ragged tail (less than one group of 16384 weights): the per-thread kernel on the
+    // remainder; the offset is a whole number of groups, so block and group indices line up.
+    const int64_t rest = numel - done;
+    const int64_t nchunk = (rest + 31) / 32;
+    int64_t blocks = (nchunk + kDeqThreads - 1) / kDeqThreads;
+    nf4_dequantize_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(
+        codes + done / 2, absmax_q + done / kBlock, group_scale + done / (kBlock * kGroup), rest, out + done,
+        nf4_table());
+  }
   prof_mark(kProfDequant, false, st);
   return cudaGetLastError();
 }

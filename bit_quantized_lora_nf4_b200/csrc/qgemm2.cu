@@ -9,16 +9,22 @@
 // tensor-core work per SM as the one-CTA kernel: the decode (ALU) cost per MMA
 // flop halves.
 //
-// Per CTA (320 threads, K-step 128 = two NF4 blocks per weight row):
-//   warp 0      TMA: its 128 activation rows (two 128B-swizzled 64-column
-//               boxes) and its 128 rows x 64 B of packed codes (64B swizzle).
+// Per CTA (320 threads, K-step 128 = two NF4 blocks per weight row), with
+// separate rings so that neither load latency nor decode sits on the MMA's
+// critical path:
+//   warp 0      TMA: activation tiles (128 rows x 128, two 128B-swizzled
+//               64-column boxes) into a 4-deep ring.
 //   warp 1      TMEM allocation for the pair; in the even CTA one lane issues
-//               the pair MMA and commits to both CTAs' barriers (multicast).
-//   warps 2-9   decode: thread (row = t % 128, j = t / 128) decodes block j of
-//               its row into the 128B-swizzled operand half (K-major for the
-//               forward, MN-major for dgrad; the byte address is the same
-//               formula in both), then signals the even CTA's "decoded"
-//               barrier.  After the last step they drain this CTA's TMEM.
+//               the pair MMA and commits to both CTAs' barriers (multicast);
+//               in the odd CTA one lane forwards "decoded" to the even CTA.
+//   warps 2-9   decode: thread (row = t % 128, j = t / 128) owns block j of its
+//               row.  Its 32 bytes of codes and its 8-bit constant are loaded
+//               from global memory into registers three K-steps ahead; it
+//               builds the block's 16-entry table, looks the codes up with byte
+//               permutes and writes 128 swizzled bytes into a 3-deep ring of
+//               operand halves (K-major for the forward, MN-major for dgrad;
+//               the byte address is the same formula in both).  After the last
+//               step the decode warps drain this CTA's TMEM.
 // Waits are bounded; on expiry a CTA latches QLORA_ERR_DEVICE_TIMEOUT, lets
 // its outstanding loads and the pair's MMAs land, frees TMEM and exits.
 #include "decode.cuh"
@@ -31,39 +37,43 @@ namespace {
 constexpr int BM = 128;            // rows per CTA
 constexpr int BN = 256;            // output columns per pair (128 B-operand columns per CTA)
 constexpr int BK = 128;            // K per stage (two 64-weight blocks)
-constexpr int STAGES = 3;
+constexpr int A_STAGES = 4;
+constexpr int D_STAGES = 3;
 constexpr int A_BYTES = BM * BK * 2;        // 32 KB: two 64-column atoms
-constexpr int P_BYTES = 128 * BK / 2;       //  8 KB: 128 rows x 64 B of codes
 constexpr int D_BYTES = 128 * BK * 2;       // 32 KB: this CTA's half of the operand
 constexpr int HALF = 16384;                 // byte stride between the two 64-wide halves
-constexpr int STAGE_BYTES = A_BYTES + P_BYTES + D_BYTES;
 constexpr int NUM_DEC_WARPS = 8;
 constexpr int THREADS = 32 * (2 + NUM_DEC_WARPS);
 constexpr int TMEM_COLS = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_STAGES * D_BYTES + 1024 + 256;
 constexpr uint64_t kDrainLimit = 4000000000ull;
+constexpr int kGroupM = 8;                  // M-pairs per raster group
 
 struct Params {
   int64_t M;
   int64_t n_out;
   int64_t ldo;
   int64_t wN, wK;
+  const uint8_t *codes;
   const uint8_t *absmax_q;
   const float *group_scale;
   const uint16_t *lora_w;
   int r;
   int nkb;           // weight K-steps (of 128)
   int nls;           // adapter K-steps (of 128)
+  int num_m, num_n;  // pair tiles along M and along the output columns
   uint16_t *out;
   int *status;
   uint64_t wait_limit;
 };
 
 struct Smem {
-  uint64_t full[STAGES];       // this CTA's TMA bytes landed
-  uint64_t empty[STAGES];      // the pair's MMAs of the stage completed (multicast commit)
-  uint64_t decoded[STAGES];    // even CTA only: all 16 decode warps of the pair are done
-  uint64_t acc_full;           // the pair's accumulation completed (multicast commit)
+  uint64_t afull[A_STAGES];        // activation tile landed (TMA)
+  uint64_t aempty[A_STAGES];       // the pair's MMAs reading it completed (multicast commit)
+  uint64_t dfree[D_STAGES];        // the pair's MMAs reading the operand half completed (multicast commit)
+  uint64_t decoded[D_STAGES];      // this CTA's 8 decode warps wrote the operand half
+  uint64_t peer_decoded[D_STAGES]; // even CTA only: the odd CTA's A tile and operand half are ready
+  uint64_t acc_full;               // the pair's accumulation completed (multicast commit)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -86,33 +96,57 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, co
   }
 }
 
+// Registers a decode thread needs for one K-step: its block's 32 code bytes
+// and the block constant q * S (zero for blocks outside the weight).
+struct BlockLoad {
+  uint4 lo, hi;
+  uint32_t q;
+  float S;
+};
+
 template <bool DGRAD>
 __global__ void __launch_bounds__(THREADS, 1)
-    qgemm2_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
-                  const __grid_constant__ CUtensorMap tm_lact, const Params p, const Nf4Table tab) {
+    qgemm2_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lact,
+                  const Params p, const Nf4Table tab) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Smem *sm = reinterpret_cast<Smem *>(smem + STAGES * STAGE_BYTES);
+  uint8_t *a_ring = smem;
+  uint8_t *d_ring = smem + A_STAGES * A_BYTES;
+  Smem *sm = reinterpret_cast<Smem *>(d_ring + D_STAGES * D_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();                              // 0 = even (MMA-issuing) CTA
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x >> 1) * (2 * BM) + rank * BM;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * BN;            // pair's first output column
+  // Grouped raster over pair tiles: consecutive clusters walk kGroupM M-pairs
+  // before moving to the next N tile, so a wave reuses both operands from L2.
+  int pm, pn;
+  {
+    const int cid = static_cast<int>(blockIdx.x >> 1);
+    const int in_group = kGroupM * p.num_n;
+    const int first_m = (cid / in_group) * kGroupM;
+    const int gsz = min(p.num_m - first_m, kGroupM);
+    pm = first_m + (cid % in_group) % gsz;
+    pn = (cid % in_group) / gsz;
+  }
+  const int64_t m0 = static_cast<int64_t>(pm) * (2 * BM) + rank * BM;
+  const int64_t n0 = static_cast<int64_t>(pn) * BN;                    // pair's first output column
   const int64_t nb0 = n0 + rank * 128;                                  // this CTA's operand columns
   const int nsteps = p.nkb + p.nls;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm->full[s], 1);
-      mbar_init(&sm->empty[s], 1);
-      mbar_init(&sm->decoded[s], 2 * NUM_DEC_WARPS);
+    for (int s = 0; s < A_STAGES; ++s) {
+      mbar_init(&sm->afull[s], 1);
+      mbar_init(&sm->aempty[s], 1);
+    }
+    for (int s = 0; s < D_STAGES; ++s) {
+      mbar_init(&sm->dfree[s], 1);
+      mbar_init(&sm->decoded[s], NUM_DEC_WARPS);
+      mbar_init(&sm->peer_decoded[s], 1);
     }
     mbar_init(&sm->acc_full, 1);
     sm->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_act);
-    tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_lact);
   }
   if (warp == 1) {
@@ -126,45 +160,42 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = sm->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (each CTA)
+    // ------------------------------------------------------------ activation TMA (each CTA)
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < nsteps; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (i >= STAGES && !wait_or_abort<false>(&sm->empty[s], ph ^ 1, p, sm)) break;
-        uint8_t *st = smem + s * STAGE_BYTES;
+        const int s = i % A_STAGES;
+        const uint32_t ph = (i / A_STAGES) & 1;
+        if (i >= A_STAGES && !wait_or_abort<false>(&sm->aempty[s], ph ^ 1, p, sm)) break;
+        uint8_t *st = a_ring + s * A_BYTES;
         if (i < p.nkb) {
-          mbar_arrive_expect_tx(&sm->full[s], A_BYTES + P_BYTES);
-          tma_load_2d(st, &tm_act, &sm->full[s], i * BK, static_cast<int>(m0));
-          tma_load_2d(st + HALF, &tm_act, &sm->full[s], i * BK + 64, static_cast<int>(m0));
-          if (DGRAD)
-            tma_load_2d(st + A_BYTES, &tm_codes, &sm->full[s], static_cast<int>(nb0 / 2), i * BK);
-          else
-            tma_load_2d(st + A_BYTES, &tm_codes, &sm->full[s], i * (BK / 2), static_cast<int>(nb0));
+          mbar_arrive_expect_tx(&sm->afull[s], A_BYTES);
+          tma_load_2d(st, &tm_act, &sm->afull[s], i * BK, static_cast<int>(m0));
+          tma_load_2d(st + HALF, &tm_act, &sm->afull[s], i * BK + 64, static_cast<int>(m0));
         } else {
           const int ls = i - p.nkb;
           const bool two = p.r - ls * BK > 64;
-          mbar_arrive_expect_tx(&sm->full[s], two ? A_BYTES : A_BYTES / 2);
-          tma_load_2d(st, &tm_lact, &sm->full[s], ls * BK, static_cast<int>(m0));
-          if (two) tma_load_2d(st + HALF, &tm_lact, &sm->full[s], ls * BK + 64, static_cast<int>(m0));
+          mbar_arrive_expect_tx(&sm->afull[s], two ? A_BYTES : A_BYTES / 2);
+          tma_load_2d(st, &tm_lact, &sm->afull[s], ls * BK, static_cast<int>(m0));
+          if (two) tma_load_2d(st + HALF, &tm_lact, &sm->afull[s], ls * BK + 64, static_cast<int>(m0));
         }
         issued = i + 1;
       }
-      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-        mbar_wait(&sm->full[j % STAGES], (j / STAGES) & 1, kDrainLimit);
+      for (int j = (issued > A_STAGES ? issued - A_STAGES : 0); j < issued; ++j)
+        mbar_wait(&sm->afull[j % A_STAGES], (j / A_STAGES) & 1, kDrainLimit);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ pair MMA issuer (even CTA)
     if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------- pair MMA issuer (even CTA)
       constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, 0, DGRAD ? 1 : 0);
       for (int i = 0; i < nsteps; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!wait_or_abort<true>(&sm->decoded[s], ph, p, sm)) break;
+        const int sa = i % A_STAGES, sd = i % D_STAGES;
+        if (!wait_or_abort<false>(&sm->afull[sa], (i / A_STAGES) & 1, p, sm)) break;
+        if (!wait_or_abort<false>(&sm->decoded[sd], (i / D_STAGES) & 1, p, sm)) break;
+        if (!wait_or_abort<true>(&sm->peer_decoded[sd], (i / D_STAGES) & 1, p, sm)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_addr(smem + s * STAGE_BYTES);
-        const uint32_t d_base = a_base + A_BYTES + P_BYTES;
+        const uint32_t a_base = smem_addr(a_ring + sa * A_BYTES);
+        const uint32_t d_base = smem_addr(d_ring + sd * D_BYTES);
         int nk = BK / 16;
         if (i >= p.nkb) {
           const int rem = p.r - (i - p.nkb) * BK;
@@ -177,9 +208,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                                        : sdesc_sw128(d_base + koff, 16, 1024);
           tc_mma_bf16_pair(tmem, adesc, bdesc, IDESC, (i | kk) != 0 ? 1u : 0u);
         }
-        tc_commit_pair_mc(&sm->empty[s], 0x3);
+        tc_commit_pair_mc(&sm->aempty[sa], 0x3);
+        tc_commit_pair_mc(&sm->dfree[sd], 0x3);
       }
       tc_commit_pair_mc(&sm->acc_full, 0x3);
+    } else if (lane == 0) {
+      // ---------------------------------------------------------- odd CTA: forward readiness
+      // The even CTA's MMA reads this CTA's activation tile and operand half:
+      // once both are in place, one cluster-scope release per stage (the
+      // decode warps only arrive locally).
+      for (int i = 0; i < nsteps; ++i) {
+        const int sd = i % D_STAGES;
+        if (!wait_or_abort<false>(&sm->afull[i % A_STAGES], (i / A_STAGES) & 1, p, sm)) break;
+        if (!wait_or_abort<false>(&sm->decoded[sd], (i / D_STAGES) & 1, p, sm)) break;
+        mbar_arrive_cluster(mapa_shared(smem_addr(&sm->peer_decoded[sd]), 0));
+      }
     }
   } else {
     // ------------------------------------------------------------ decoders (each CTA)
@@ -187,7 +230,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row = dt & 127;                 // operand row within this CTA's half
     const int jb = dt >> 7;                   // which of the stage's two blocks
     const int64_t kblocks = p.wK / kBlock;
-    auto block_index = [&](int i, int64_t *idx) -> bool {
+    auto fetch = [&](int i, BlockLoad &b) {
+      b.lo = b.hi = make_uint4(0, 0, 0, 0);
+      b.q = 0;
+      b.S = 0.0f;
+      if (i >= p.nkb) return;
       int64_t n, kb;
       if (DGRAD) {
         n = static_cast<int64_t>(i) * BK + row;
@@ -196,40 +243,41 @@ __global__ void __launch_bounds__(THREADS, 1)
         n = nb0 + row;
         kb = 2 * static_cast<int64_t>(i) + jb;
       }
-      *idx = n * kblocks + kb;
-      return n < p.wN && kb < kblocks;
+      if (n < p.wN && kb < kblocks) {
+        const int64_t idx = n * kblocks + kb;
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + idx * 32);
+        b.lo = __ldg(src);
+        b.hi = __ldg(src + 1);
+        b.q = __ldg(p.absmax_q + idx);
+        b.S = __ldg(p.group_scale + (idx >> 8));
+      }
     };
-    uint32_t q_next = 0;
-    float s_next = 0.0f;
-    {
-      int64_t idx;
-      if (p.nkb > 0 && block_index(0, &idx)) {
-        q_next = __ldg(p.absmax_q + idx);
-        s_next = __ldg(p.group_scale + (idx >> 8));
-      }
-    }
-    const uint32_t swz64 = (row >> 1) & 3;    // 64B swizzle of the code tile
-    const uint32_t swz128 = row & 7;          // 128B swizzle of the operand
+    BlockLoad b0, b1, b2;
+    fetch(0, b0);
+    fetch(1, b1);
+    fetch(2, b2);
+    const uint32_t swz = row & 7;             // 128B swizzle of the operand
     for (int i = 0; i < nsteps; ++i) {
-      const int s = i % STAGES;
-      const uint32_t ph = (i / STAGES) & 1;
-      const float ap = __fmul_rn(static_cast<float>(q_next), s_next);
-      q_next = 0;
-      s_next = 0.0f;
-      if (i + 1 < p.nkb) {
-        int64_t idx;
-        if (block_index(i + 1, &idx)) {
-          q_next = __ldg(p.absmax_q + idx);
-          s_next = __ldg(p.group_scale + (idx >> 8));
-        }
-      }
-      if (!__all_sync(0xffffffffu, wait_or_abort<false>(&sm->full[s], ph, p, sm))) break;
-      const uint32_t st = smem_addr(smem + s * STAGE_BYTES);
-      const uint32_t prow = st + A_BYTES + row * 64;
-      const uint32_t drow = st + A_BYTES + P_BYTES + jb * HALF + row * 128;
+      const int sd = i % D_STAGES;
+      BlockLoad cur = b0;
+      b0 = b1;
+      b1 = b2;
+      fetch(i + 3, b2);                       // three K-steps of latency hiding
+      if (i >= D_STAGES &&
+          !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
+        break;
+      const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * HALF + row * 128;
       if (i < p.nkb) {
-        nf4_decode_row(prow + (((2 * jb) ^ swz64) << 4), prow + (((2 * jb + 1) ^ swz64) << 4), drow, swz128, ap,
-                       tab);
+        const float ap = __fmul_rn(static_cast<float>(cur.q), cur.S);
+        uint32_t LO[4], HI[4];
+        nf4_block_table(ap, tab, LO, HI);
+        const uint32_t words[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          uint32_t o[4];
+          nf4_lut8(words[w], LO, HI, o);
+          st_shared_v4(drow + ((static_cast<uint32_t>(w) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+        }
       } else {
         // adapter weight slice in the same operand layout; zero past r / past the matrix
         const int64_t base_r = static_cast<int64_t>(i - p.nkb) * BK + 64 * jb;
@@ -244,12 +292,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int64_t rr = base_r + 8 * c;
             if (n < p.wN && rr < p.r) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + n * p.r + rr));
           }
-          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz128) << 4), v.x, v.y, v.z, v.w);
+          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), v.x, v.y, v.z, v.w);
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&sm->decoded[s]), 0));
+      if (lane == 0) mbar_arrive(&sm->decoded[sd]);
     }
 
     // ------------------------------------------------------------ epilogue (each CTA, its 128 rows)
@@ -296,14 +344,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace
 
 qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
-  CUtensorMap tm_act, tm_codes, tm_lact;
+  CUtensorMap tm_act, tm_lact;
   const int64_t kred = a.dgrad ? a.wN : a.wK;
   const int64_t n_out = a.dgrad ? a.wK : a.wN;
-  const uint64_t codes_row = static_cast<uint64_t>(a.wK / 2);
   bool ok = make_tmap_2d(&tm_act, a.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kred, a.M, kred * 2, 64, BM,
                          CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && make_tmap_2d(&tm_codes, a.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_row, a.wN, codes_row, 64, 128,
-                          CU_TENSOR_MAP_SWIZZLE_64B);
   ok = ok && make_tmap_2d(&tm_lact, a.lora_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.r, a.M,
                           static_cast<uint64_t>(a.r) * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return QLORA_ERR_CUDA;
@@ -314,6 +359,7 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   p.ldo = n_out;
   p.wN = a.wN;
   p.wK = a.wK;
+  p.codes = a.codes;
   p.absmax_q = a.absmax_q;
   p.group_scale = a.group_scale;
   p.lora_w = a.lora_w;
@@ -326,7 +372,9 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   if (!p.status) return QLORA_ERR_CUDA;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * ceil_div(a.M, 2 * BM)), static_cast<unsigned>(ceil_div(n_out, BN)));
+  p.num_m = static_cast<int>(ceil_div(a.M, 2 * BM));
+  p.num_n = static_cast<int>(ceil_div(n_out, BN));
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * p.num_m * p.num_n));
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
@@ -343,11 +391,11 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   if (a.dgrad) {
     e = cudaFuncSetAttribute(qgemm2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<true>, tm_act, tm_codes, tm_lact, p, tab);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<true>, tm_act, tm_lact, p, tab);
   } else {
     e = cudaFuncSetAttribute(qgemm2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<false>, tm_act, tm_codes, tm_lact, p, tab);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<false>, tm_act, tm_lact, p, tab);
   }
   prof_mark(kind, false, st);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
