@@ -1,7 +1,7 @@
 // Few-token forward (M <= 16): memory-bound dequant-GEMV.
 //
 // "QLoRA: fine-tuning a 65B model on one GPU", section "Where the memory
-// goes": the 4-bit base is dequantized on the fly to 16-bit for each pass.
+// goes": every pass expands the 4-bit base to 16-bit as it runs.
 // With a handful of tokens the packed weight stream (0.516 B per weight) is the
 // whole cost, so the weight is decoded straight into tensor-core register
 // fragments and never touches shared memory.
@@ -73,34 +73,41 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
   }
   __syncthreads();
 
-  // Adapter prologue partials for this K chunk: hpart[z][m][j] = sum_k X[m][k] A[j][k],
+  // Adapter prologue partials for this K chunk: hpart[z][m][j] = sum_k X[m][k] A[j][k]
   // for the adapter rows j = blockIdx.x, blockIdx.x + gridDim.x, ...  Thread t
-  // takes token t % 16 and every 8th 4-element word of the chunk; the 8 word
-  // groups are summed in a fixed order through shared memory.
+  // covers k = 8t .. 8t+7 of the chunk for every token (one 16-byte load of A),
+  // then the 128 partial sums per token are reduced in a fixed order (warp
+  // shuffles, then the 4 warps through shared memory).
   {
-    __shared__ float hred[8][GV_TOK];
-    const int tok = threadIdx.x & 15, grp = threadIdx.x >> 4;
-    const int nwords = static_cast<int>(kc / 4);
+    __shared__ float hred[GV_THREADS / 32][GV_TOK];
+    const int k = threadIdx.x * 8;
+    const int ms = k / GV_MACRO, in = k % GV_MACRO;
+    const int c8 = in / 64, s8 = (in % 64) / 4;
     for (int j = blockIdx.x; j < r; j += gridDim.x) {
-      float acc_h = 0.0f;
-      if (tok < M && tok < NT * 8) {
-        for (int qw = grp; qw < nwords; qw += 8) {
-          const int k = qw * 4;
-          const int ms = k / GV_MACRO, in = k % GV_MACRO;
-          const uint2 xv = xs[ms][(in % 64) / 4][tok][in / 64];
-          const uint2 av = __ldg(reinterpret_cast<const uint2 *>(A + static_cast<int64_t>(j) * K + k_base + k));
-          acc_h = fmaf(__uint_as_float(xv.x << 16), __uint_as_float(av.x << 16), acc_h);
-          acc_h = fmaf(__uint_as_float(xv.x & 0xFFFF0000u), __uint_as_float(av.x & 0xFFFF0000u), acc_h);
-          acc_h = fmaf(__uint_as_float(xv.y << 16), __uint_as_float(av.y << 16), acc_h);
-          acc_h = fmaf(__uint_as_float(xv.y & 0xFFFF0000u), __uint_as_float(av.y & 0xFFFF0000u), acc_h);
+      uint4 av = make_uint4(0, 0, 0, 0);
+      if (k < kc) av = __ldg(reinterpret_cast<const uint4 *>(A + static_cast<int64_t>(j) * K + k_base + k));
+      const uint32_t a4[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+      for (int tok = 0; tok < NT * 8; ++tok) {
+        float h = 0.0f;
+        if (tok < M) {
+          const uint2 x0 = xs[ms][s8][tok][c8], x1 = xs[ms][s8 + 1][tok][c8];
+          const uint32_t x4[4] = {x0.x, x0.y, x1.x, x1.y};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            h = fmaf(__uint_as_float(x4[e] << 16), __uint_as_float(a4[e] << 16), h);
+            h = fmaf(__uint_as_float(x4[e] & 0xFFFF0000u), __uint_as_float(a4[e] & 0xFFFF0000u), h);
+          }
         }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) h += __shfl_xor_sync(0xffffffffu, h, off);
+        if ((threadIdx.x & 31) == 0) hred[threadIdx.x >> 5][tok] = h;
       }
-      hred[grp][tok] = acc_h;
       __syncthreads();
       if (threadIdx.x < M) {
         float v = 0.0f;
 #pragma unroll
-        for (int gq = 0; gq < 8; ++gq) v += hred[gq][threadIdx.x];
+        for (int wq = 0; wq < GV_THREADS / 32; ++wq) v += hred[wq][threadIdx.x];
         hpart[(static_cast<int64_t>(blockIdx.y) * M + threadIdx.x) * r + j] = v;
       }
       __syncthreads();
@@ -184,11 +191,14 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_main_kernel(const uint16_t *_
   }
 }
 
-constexpr int GV_RED_ROWS = 64;
+constexpr int GV_RED_ROWS = 32;      // output rows per reduce CTA (8 warps x 4 rows)
 
-// Per CTA of 64 output rows: sH[m][j] = fl32(s * sum_z hpart[z][m][j]) into
+// Per CTA of 32 output rows: sH[m][j] = fl32(s * sum_z hpart[z][m][j]) into
 // shared memory (the CTA with blockIdx.x == 0 also writes the unscaled H when
-// asked), then Y[m][n] = bf16( sum_z part[z][n][m] + sum_j sH[m][j] B[n][j] ).
+// asked).  Then 8 lanes per output row n: lane l takes the adapter columns
+// 8c .. 8c+7 for c = l, l+8, ... (16-byte loads of B), the 8 partial dot
+// products are combined with xor shuffles, and lane l finishes tokens l and
+// l+8: Y[m][n] = bf16( sum_z part[z][n][m] + sum_j sH[m][j] B[n][j] ).
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restrict__ part,
                                                           const float *__restrict__ hpart, int nchunks, int M,
                                                           int64_t N, const uint16_t *__restrict__ B, int r, float s,
@@ -196,23 +206,57 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restric
   __shared__ float sh[GV_TOK * 256];
   for (int e = threadIdx.x; e < M * r; e += blockDim.x) {
     float h = 0.0f;
+#pragma unroll 4
     for (int z = 0; z < nchunks; ++z) h += hpart[static_cast<int64_t>(z) * M * r + e];
     sh[e] = __fmul_rn(s, h);
     if (H_out && blockIdx.x == 0) H_out[e] = h;
   }
   __syncthreads();
   const int ldp = (M + 1) & ~1;
-  const int64_t n_base = static_cast<int64_t>(blockIdx.x) * GV_RED_ROWS;
-  for (int idx = threadIdx.x; idx < GV_RED_ROWS * M; idx += blockDim.x) {
-    const int64_t n = n_base + idx % GV_RED_ROWS;
-    const int m = idx / GV_RED_ROWS;
-    if (n >= N) continue;
-    float v = 0.0f;
-    for (int z = 0; z < nchunks; ++z) v += part[(static_cast<int64_t>(z) * N + n) * ldp + m];
-    float l = 0.0f;
-    for (int j = 0; j < r; ++j) l = fmaf(sh[m * r + j], __uint_as_float(static_cast<uint32_t>(B[n * r + j]) << 16), l);
-    const __nv_bfloat16 b = __float2bfloat16_rn(v + l);
-    Y[static_cast<int64_t>(m) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int l8 = lane & 7;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * GV_RED_ROWS + warp * 4 + (lane >> 3);
+  const bool live = n < N;
+  float acc[GV_TOK];
+#pragma unroll
+  for (int m = 0; m < GV_TOK; ++m) acc[m] = 0.0f;
+  if (live) {
+    for (int c = l8; c < r / 8; c += 8) {
+      const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(B + n * r + 8 * c));
+      const uint32_t b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int m = 0; m < GV_TOK; ++m) {
+        if (m < M) {
+          const float *shm = sh + m * r + 8 * c;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[m] = fmaf(shm[2 * e], __uint_as_float(b4[e] << 16), acc[m]);
+            acc[m] = fmaf(shm[2 * e + 1], __uint_as_float(b4[e] & 0xFFFF0000u), acc[m]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < GV_TOK; ++m) {
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+  }
+  if (live) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = l8 + 8 * h;
+      if (m < M) {
+        float v = 0.0f;
+        for (int z = 0; z < nchunks; ++z) v += part[(static_cast<int64_t>(z) * N + n) * ldp + m];
+        float lora = acc[0];
+#pragma unroll
+        for (int mm = 1; mm < GV_TOK; ++mm)
+          if (mm == m) lora = acc[mm];
+        const __nv_bfloat16 b = __float2bfloat16_rn(v + lora);
+        Y[static_cast<int64_t>(m) * N + n] = *reinterpret_cast<const uint16_t *>(&b);
+      }
+    }
   }
 }
 

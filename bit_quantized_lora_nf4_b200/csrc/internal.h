@@ -82,8 +82,8 @@ qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st);
 constexpr int kGemvMaxTokens = 16;
 bool gemv_enabled();
 
-// Tall-skinny products on tensor cores (mma.sync), split over the reduction
-// with fp32 partials part[z][I][J]:  C[i,j] = sum_k opA(i,k) opB(j,k),
+// Tall-skinny adapter products on tcgen05 tensor cores (lora_tc.cu), split over
+// the reduction with fp32 partials part[z][I][J]:  C[i,j] = sum_k opA(i,k) opB(j,k),
 // opX(i,k) = X[i*ld + k] when K-major, X[k*ld + i] otherwise.
 struct SkinnyArgs {
   const uint16_t *A;

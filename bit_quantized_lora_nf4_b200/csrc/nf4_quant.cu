@@ -4,8 +4,9 @@
 // "QLoRA: fine-tuning a 65B model on one GPU", section "NormalFloat, double
 // quantization, paged optimizers": 16 levels at normal quantiles, one scaling
 // constant per block of weights, the constants themselves stored in 8 bits
-// under a coarser set of constants.  Section "Where the memory goes": the base
-// is quantized once up front and dequantized to 16-bit for every pass.
+// under one more, coarser level of constants.  Section "Where the memory
+// goes": the frozen base is quantized a single time before training and
+// expanded to 16-bit in every pass.
 //
 // Arithmetic contract (IEEE fp32 round-to-nearest, no FMA contraction, no
 // flush-to-zero; this file is compiled with -fmad=false):

@@ -1,7 +1,7 @@
 // Fused NF4 dequant-GEMM on 5th-generation tensor cores (tcgen05, TMEM, TMA).
 //
 // "QLoRA: fine-tuning a 65B model on one GPU", section "Where the memory
-// goes": the 4-bit base is dequantized on the fly to 16-bit for each forward
+// goes": every forward and backward pass expands the 4-bit base to 16-bit as it
 // and backward pass, and gradients flow through the dequantized weights into
 // the adapters.  "Qlora 4 Bit Quantization With Nf4 Fp4 Data Types And Lora
 // Adapters", entry "quantization-aware-lora-training-with-kernel-fusion":

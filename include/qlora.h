@@ -9,13 +9,13 @@
  *     adapters; (a) the NF4 data type, (b) double quantization of the
  *     quantization constants.
  *   - "QLoRA: fine-tuning a 65B model on one GPU", section "Where the memory
- *     goes": the base is stored in 4 bits, quantized once up front, and
- *     dequantized on the fly to 16-bit for every forward and backward pass;
+ *     goes": the base is kept in 4 bits, quantized a single time before
+ *     training, and expanded to 16-bit inside every forward and backward pass;
  *     gradients flow through the dequantized weights into the adapters, which
  *     stay 16-bit.  Section "NormalFloat, double quantization, paged
  *     optimizers": 16 levels at normal quantiles; one scaling constant per
- *     block; the constants themselves stored in 8 bits under a second,
- *     coarser set of constants.
+ *     block; those constants in turn stored in 8 bits, scaled by a further,
+ *     coarser level of constants.
  *   - "Qlora 4 Bit Quantization With Nf4 Fp4 Data Types And Lora Adapters",
  *     entry "4-bit quantization with nf4 data type for llm weight
  *     compression": block-wise absmax scaling plus double quantization.
@@ -93,7 +93,7 @@ qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, voi
 
 /* qlora_dequantize -- W' = bf16(fl32(v_code * fl32(q_b * S_g))) into a device
  * bf16 buffer of rows*cols elements, row-major.  ("Where the memory goes":
- * dequantized on the fly to 16-bit.)  Bit-exact by construction. */
+ * the 16-bit form each pass works with.)  Bit-exact by construction. */
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream);
 
 /* Operation ids for qlora_workspace_bytes(). */
@@ -149,8 +149,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
  *   loads the library until the process exits; the call allocates and frees
  *   nothing.
  *   Returns QLORA_ERR_WORKSPACE when qlora_workspace_bytes(QLORA_OP_FWD, M, N,
- *   K, r) exceeds QLORA_STATIC_SCRATCH_BYTES (e.g. M = 4096, r = 64 fits;
- *   M = 8192, r = 64 does not).
+ *   K, r) exceeds QLORA_STATIC_SCRATCH_BYTES (e.g. M = 8192, r = 64 fits;
+ *   M = 8192, r = 256 does not).
  *   The first call on a device looks up the array's device address; make that
  *   first call before any stream capture.  Every call shares the one array
  *   (it keeps the previous call's contents; nothing needs clearing), so calls

@@ -25,7 +25,7 @@ Module map:
   linear.py  fp64 LoRA linear forward / backward on the dequantized weight.
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py`` except
-the quantitative "each level covers an equal share" property of the codebook,
+the quantitative equal-usage property of the codebook levels,
 which is reported only (parity unpinned for that claim; absmax normalisation
 makes it approximate).
 """

@@ -35,9 +35,9 @@ NLEVELS = 16
 def nf4_levels_exact(dps: int = 50):
     """The 16 NF4 levels as high-precision mpmath numbers, ascending.
 
-    [Blog-nf4]: NF4 places its 16 levels at quantiles of a normal distribution
-    so that each level covers an equal share of normally distributed weights;
-    [QLoRA-abs] (a): information-theoretically optimal for normal weights;
+    [Blog-nf4]: the 16 NF4 levels sit at normal quantiles, so for Gaussian
+    weights every level is hit about equally often; [QLoRA-abs] (a): the type
+    is designed to be optimal for normally distributed weights;
     [Cap-nf4]: combined with block-wise absmax scaling.
 
     Reading (the pages give no formula): the levels must span [-1, 1] (absmax
@@ -171,7 +171,7 @@ def double_quantize(absmax: np.ndarray):
     """Quantize the fp32 block constants to 8 bits with one fp32 scale per group.
 
     [Blog-nf4] (double quantization stores the per-block constants in 8-bit
-    with a second, coarser set of constants above them), [QLoRA-abs] (b),
+    under one more, coarser level of constants), [QLoRA-abs] (b),
     [Cap-nf4].  Reading (the 8-bit format is not given): unsigned linear
     8-bit codes with no offset, group = 256 consecutive blocks:
         c_g = max_b a_b,   S_g = fl32(c_g / 255),
@@ -229,8 +229,8 @@ def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np
                         shape) -> np.ndarray:
     """W' = bf16(fl32(v_code * a'_b)) with a'_b = fl32(q_b * S_g); bf16 bit patterns.
 
-    [Blog-mem]: the 4-bit base is dequantized on the fly to 16-bit for each
-    forward and backward pass.  Reading: the 16-bit type is bf16, the product
+    [Blog-mem]: every forward and backward pass expands the 4-bit base back
+    to a 16-bit type as it runs.  Reading: the 16-bit type is bf16, the product
     is formed in fp32 then rounded once to bf16.
     """
     numel = int(np.prod(shape))

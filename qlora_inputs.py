@@ -7,8 +7,8 @@ consume exactly the tensors returned here.
 Recipe (one numpy PCG64 generator per case, draws in the fixed order
 W, A, B, X, dY, each drawn in fp32 then rounded to nearest-even bf16 where the
 tensor is bf16):
-  W  [N,K] fp32 ~ N(0, 0.02^2)        frozen base ("roughly normally distributed"
-                                       pretrained weights, the premise of NF4)
+  W  [N,K] fp32 ~ N(0, 0.02^2)        frozen base (pretrained weights are close to
+                                       Gaussian, the premise of NF4)
   A  [r,K] bf16 ~ N(0, 0.01^2)        adapter down-projection
   B  [N,r] bf16 ~ N(0, 0.01^2)        adapter up-projection
   X  [M,K] bf16 ~ N(0, 1)             activations

@@ -268,7 +268,7 @@ def test_footprint_and_page_figures():
     # 16-bit storage of a 65B model is 130 GB (2 bytes per parameter).
     p65 = fig["params_65b"]
     assert p65 * 2 / 1e9 == fig["bf16_bytes_65b_gb"]
-    # "4x compression" of 16-bit weights, within the rounding the page uses.
+    # about four times smaller than 16-bit weights, within the rounding the page uses.
     ratio = 16 / bits
     assert abs(ratio - fig["compression_vs_16bit"]) < 0.5
     # 65B frozen base in NF4+DQ fits a single 48 GB GPU with room for adapters.

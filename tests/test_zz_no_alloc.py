@@ -53,8 +53,8 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch(lib):
     lib_ = q.load()
     w = q.NF4Weight.empty(4096, 4096)
     X = torch.empty((8192, 4096), dtype=torch.bfloat16, device="cuda")
-    A = torch.empty((64, 4096), dtype=torch.bfloat16, device="cuda")
-    B = torch.empty((4096, 64), dtype=torch.bfloat16, device="cuda")
+    A = torch.empty((256, 4096), dtype=torch.bfloat16, device="cuda")
+    B = torch.empty((4096, 256), dtype=torch.bfloat16, device="cuda")
     Y = torch.empty((8192, 4096), dtype=torch.bfloat16, device="cuda")
-    assert lib_.qlora_workspace_bytes(q.QLORA_OP_FWD, 8192, 4096, 4096, 64) > (8 << 20)
+    assert lib_.qlora_workspace_bytes(q.QLORA_OP_FWD, 8192, 4096, 4096, 256) > (8 << 20)
     assert _noalloc(w, X, A, B, 0.25, Y, None) == 7          # QLORA_ERR_WORKSPACE, nothing launched
