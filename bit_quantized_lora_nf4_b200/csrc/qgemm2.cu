@@ -36,16 +36,29 @@ namespace {
 
 constexpr int BM = 128;            // rows per CTA
 constexpr int BN = 256;            // output columns per pair (128 B-operand columns per CTA)
-constexpr int BK = 128;            // K per stage (two 64-weight blocks)
 constexpr int A_STAGES = 4;
-constexpr int D_STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;        // 32 KB: two 64-column atoms
-constexpr int D_BYTES = 128 * BK * 2;       // 32 KB: this CTA's half of the operand
-constexpr int HALF = 16384;                 // byte stride between the two 64-wide halves
+constexpr int A_BYTES = 32768;              // one activation stage: NACC x 128 rows x BK bf16
+constexpr int HALF = 16384;                 // one 128-row x 64-column swizzled atom column
+constexpr int D_RING = 98304;               // 96 KB of decoded-operand stages
 constexpr int NUM_DEC_WARPS = 8;
 constexpr int THREADS = 32 * (2 + NUM_DEC_WARPS);
-constexpr int TMEM_COLS = 256;
-constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_STAGES * D_BYTES + 1024 + 256;
+constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + 256;
+
+// NACC = accumulators per CTA: the pair tile covers 256 * NACC rows.  With
+// NACC = 2 every decoded operand half feeds two MMAs (rows 0-255 and 256-511
+// of the pair tile), halving the decode work per tensor-core flop again; the
+// K-step shrinks to 64 so the activation stage stays 32 KB, and the decode
+// warps split into two groups that take alternate K-steps.
+template <int NACC>
+struct Cfg {
+  static constexpr int BK = 128 / NACC;                      // K per stage
+  static constexpr int KH = BK / 64;                         // 64-wide halves per stage
+  static constexpr int D_BYTES = 128 * BK * 2;               // this CTA's operand half per stage
+  static constexpr int D_STAGES = D_RING / D_BYTES;          // 3 or 6
+  static constexpr int TMEM_COLS = 256 * NACC;
+  static constexpr int GROUP_WARPS = NUM_DEC_WARPS / NACC;   // decode warps per group
+};
+constexpr int MAX_D_STAGES = 6;
 constexpr uint64_t kDrainLimit = 4000000000ull;
 constexpr int kGroupM = 8;                  // M-pairs per raster group
 
@@ -70,9 +83,9 @@ struct Params {
 struct Smem {
   uint64_t afull[A_STAGES];        // activation tile landed (TMA)
   uint64_t aempty[A_STAGES];       // the pair's MMAs reading it completed (multicast commit)
-  uint64_t dfree[D_STAGES];        // the pair's MMAs reading the operand half completed (multicast commit)
-  uint64_t decoded[D_STAGES];      // this CTA's 8 decode warps wrote the operand half
-  uint64_t peer_decoded[D_STAGES]; // even CTA only: the odd CTA's A tile and operand half are ready
+  uint64_t dfree[MAX_D_STAGES];        // the pair's MMAs reading the operand half completed (multicast commit)
+  uint64_t decoded[MAX_D_STAGES];      // this CTA's decode group wrote the operand half
+  uint64_t peer_decoded[MAX_D_STAGES]; // even CTA only: the odd CTA's A tile and operand half are ready
   uint64_t acc_full;               // the pair's accumulation completed (multicast commit)
   uint32_t tmem_base;
   int abort_flag;
@@ -104,15 +117,19 @@ struct BlockLoad {
   float S;
 };
 
-template <bool DGRAD>
+template <bool DGRAD, int NACC>
 __global__ void __launch_bounds__(THREADS, 1)
     qgemm2_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lact,
                   const Params p, const Nf4Table tab) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *a_ring = smem;
+  using C = Cfg<NACC>;
+  constexpr int BK = C::BK;
+  constexpr int D_STAGES = C::D_STAGES;
+  constexpr int D_BYTES = C::D_BYTES;
   uint8_t *d_ring = smem + A_STAGES * A_BYTES;
-  Smem *sm = reinterpret_cast<Smem *>(d_ring + D_STAGES * D_BYTES);
+  Smem *sm = reinterpret_cast<Smem *>(d_ring + D_RING);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -128,7 +145,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     pm = first_m + (cid % in_group) % gsz;
     pn = (cid % in_group) / gsz;
   }
-  const int64_t m0 = static_cast<int64_t>(pm) * (2 * BM) + rank * BM;
+  // this CTA's rows of accumulator t: mbase + 256 t .. + 127
+  const int64_t mbase = static_cast<int64_t>(pm) * (2 * BM * NACC) + rank * BM;
   const int64_t n0 = static_cast<int64_t>(pn) * BN;                    // pair's first output column
   const int64_t nb0 = n0 + rank * 128;                                  // this CTA's operand columns
   const int nsteps = p.nkb + p.nls;
@@ -140,7 +158,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int s = 0; s < D_STAGES; ++s) {
       mbar_init(&sm->dfree[s], 1);
-      mbar_init(&sm->decoded[s], NUM_DEC_WARPS);
+      mbar_init(&sm->decoded[s], C::GROUP_WARPS);
       mbar_init(&sm->peer_decoded[s], 1);
     }
     mbar_init(&sm->acc_full, 1);
@@ -150,7 +168,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tm_lact);
   }
   if (warp == 1) {
-    tmem_alloc_pair(&sm->tmem_base, TMEM_COLS);
+    tmem_alloc_pair(&sm->tmem_base, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
   tc_fence_before();
@@ -168,16 +186,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t ph = (i / A_STAGES) & 1;
         if (i >= A_STAGES && !wait_or_abort<false>(&sm->aempty[s], ph ^ 1, p, sm)) break;
         uint8_t *st = a_ring + s * A_BYTES;
+        // atom column (t, kh) of the stage at (t * KH + kh) * HALF
         if (i < p.nkb) {
           mbar_arrive_expect_tx(&sm->afull[s], A_BYTES);
-          tma_load_2d(st, &tm_act, &sm->afull[s], i * BK, static_cast<int>(m0));
-          tma_load_2d(st + HALF, &tm_act, &sm->afull[s], i * BK + 64, static_cast<int>(m0));
+          for (int t = 0; t < NACC; ++t)
+            for (int kh = 0; kh < C::KH; ++kh)
+              tma_load_2d(st + (t * C::KH + kh) * HALF, &tm_act, &sm->afull[s], i * BK + 64 * kh,
+                          static_cast<int>(mbase + 256 * t));
         } else {
           const int ls = i - p.nkb;
-          const bool two = p.r - ls * BK > 64;
-          mbar_arrive_expect_tx(&sm->afull[s], two ? A_BYTES : A_BYTES / 2);
-          tma_load_2d(st, &tm_lact, &sm->afull[s], ls * BK, static_cast<int>(m0));
-          if (two) tma_load_2d(st + HALF, &tm_lact, &sm->afull[s], ls * BK + 64, static_cast<int>(m0));
+          const int rem = p.r - ls * BK;
+          const int halves = rem > 64 ? C::KH : 1;
+          mbar_arrive_expect_tx(&sm->afull[s], NACC * halves * HALF);
+          for (int t = 0; t < NACC; ++t)
+            for (int kh = 0; kh < halves; ++kh)
+              tma_load_2d(st + (t * C::KH + kh) * HALF, &tm_lact, &sm->afull[s], ls * BK + 64 * kh,
+                          static_cast<int>(mbase + 256 * t));
         }
         issued = i + 1;
       }
@@ -203,10 +227,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int kk = 0; kk < nk; ++kk) {
           const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-          const uint64_t adesc = sdesc_sw128(a_base + koff, 16, 1024);
-          const uint64_t bdesc = DGRAD ? sdesc_sw128(d_base + kk * 2048, HALF, 1024)
+          const uint64_t bdesc = DGRAD ? sdesc_sw128(d_base + kk * 2048, BK * 128, 1024)
                                        : sdesc_sw128(d_base + koff, 16, 1024);
-          tc_mma_bf16_pair(tmem, adesc, bdesc, IDESC, (i | kk) != 0 ? 1u : 0u);
+          for (int t = 0; t < NACC; ++t) {
+            const uint64_t adesc = sdesc_sw128(a_base + t * C::KH * HALF + koff, 16, 1024);
+            tc_mma_bf16_pair(tmem + 256 * t, adesc, bdesc, IDESC, (i | kk) != 0 ? 1u : 0u);
+          }
         }
         tc_commit_pair_mc(&sm->aempty[sa], 0x3);
         tc_commit_pair_mc(&sm->dfree[sd], 0x3);
@@ -226,9 +252,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ decoders (each CTA)
-    const int dt = threadIdx.x - 64;          // 0..255
-    const int row = dt & 127;                 // operand row within this CTA's half
-    const int jb = dt >> 7;                   // which of the stage's two blocks
+    // NACC groups of decode warps take alternate K-steps; within a group,
+    // thread u owns block jb of operand row `row` (forward: weight row,
+    // 128 per stage; dgrad: reduction row, BK per stage).
+    const int dwarp = warp - 2;
+    const int grp = dwarp / C::GROUP_WARPS;
+    const int u = (threadIdx.x - 64) % (C::GROUP_WARPS * 32);
+    constexpr int DROWS = DGRAD ? BK : 128;
+    const int row = u % DROWS;
+    const int jb = u / DROWS;
     const int64_t kblocks = p.wK / kBlock;
     auto fetch = [&](int i, BlockLoad &b) {
       b.lo = b.hi = make_uint4(0, 0, 0, 0);
@@ -241,7 +273,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         kb = nb0 / kBlock + jb;
       } else {
         n = nb0 + row;
-        kb = 2 * static_cast<int64_t>(i) + jb;
+        kb = static_cast<int64_t>(i) * C::KH + jb;
       }
       if (n < p.wN && kb < kblocks) {
         const int64_t idx = n * kblocks + kb;
@@ -253,20 +285,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     };
     BlockLoad b0, b1, b2;
-    fetch(0, b0);
-    fetch(1, b1);
-    fetch(2, b2);
+    fetch(grp, b0);
+    fetch(grp + NACC, b1);
+    fetch(grp + 2 * NACC, b2);
     const uint32_t swz = row & 7;             // 128B swizzle of the operand
-    for (int i = 0; i < nsteps; ++i) {
+    for (int i = grp; i < nsteps; i += NACC) {
       const int sd = i % D_STAGES;
       BlockLoad cur = b0;
       b0 = b1;
       b1 = b2;
-      fetch(i + 3, b2);                       // three K-steps of latency hiding
+      fetch(i + 3 * NACC, b2);                // three of this group's K-steps of latency hiding
       if (i >= D_STAGES &&
           !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
         break;
-      const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * HALF + row * 128;
+      const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
       if (i < p.nkb) {
         const float ap = __fmul_rn(static_cast<float>(cur.q), cur.S);
         uint32_t LO[4], HI[4];
@@ -300,19 +332,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&sm->decoded[sd]);
     }
 
-    // ------------------------------------------------------------ epilogue (each CTA, its 128 rows)
+    // ------------------------------------------------------------ epilogue (each CTA, its rows)
     const bool acc_ok = mbar_wait(&sm->acc_full, 0, kDrainLimit);
     tc_fence_after();
     volatile int *abort_flag = &sm->abort_flag;
     if (__all_sync(0xffffffffu, acc_ok && *abort_flag == 0)) {
+      // NACC 1: the two warps of a lane quarter split the 256 columns;
+      // NACC 2: decode group g drains accumulator g (256 columns).
       const int quarter = warp & 3;
-      const int half = (warp - 2) >> 2;
-      const int64_t orow_i = m0 + quarter * 32 + lane;
+      const int acc = NACC == 1 ? 0 : (dwarp >> 2);
+      const int col_begin = NACC == 1 ? (dwarp >> 2) * 128 : 0;
+      const int nchunk = NACC == 1 ? 4 : 8;
+      const int64_t orow_i = mbase + 256 * acc + quarter * 32 + lane;
       uint16_t *orow = p.out + orow_i * p.ldo;
-      for (int cc = 0; cc < 4; ++cc) {
-        const int col0 = half * 128 + cc * 32;
+      for (int cc = 0; cc < nchunk; ++cc) {
+        const int col0 = col_begin + cc * 32;
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
+        tmem_ld_32x32b_x32(tmem + 256 * acc + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
         tmem_ld_wait();
         if (orow_i < p.M) {
           const int64_t c0 = n0 + col0;
@@ -337,7 +373,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync_all();        // the peer is done with this CTA's shared memory and TMEM
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
 }
 
@@ -364,16 +400,20 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   p.group_scale = a.group_scale;
   p.lora_w = a.lora_w;
   p.r = a.r;
-  p.nkb = static_cast<int>(ceil_div(kred, BK));
-  p.nls = static_cast<int>(ceil_div(a.r, BK));
   p.out = a.out;
   p.status = device_status_ptr();
   p.wait_limit = wait_limit();
   if (!p.status) return QLORA_ERR_CUDA;
 
-  cudaLaunchConfig_t cfg = {};
-  p.num_m = static_cast<int>(ceil_div(a.M, 2 * BM));
+  // two accumulators per CTA (512-row pair tile) once M fills them
+  const int nacc = a.M > 2 * BM ? 2 : 1;
+  const int bk = nacc == 2 ? Cfg<2>::BK : Cfg<1>::BK;
+  p.nkb = static_cast<int>(ceil_div(kred, bk));
+  p.nls = static_cast<int>(ceil_div(a.r, bk));
+  p.num_m = static_cast<int>(ceil_div(a.M, 2 * BM * nacc));
   p.num_n = static_cast<int>(ceil_div(n_out, BN));
+
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * p.num_m * p.num_n));
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
@@ -387,17 +427,18 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   cfg.numAttrs = 1;
   const Nf4Table tab = nf4_table();
   const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
+  auto go = [&](auto kern) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    prof_mark(kind, true, st);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, kern, tm_act, tm_lact, p, tab);
+    prof_mark(kind, false, st);
+    return e;
+  };
   cudaError_t e;
-  if (a.dgrad) {
-    e = cudaFuncSetAttribute(qgemm2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    prof_mark(kind, true, st);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<true>, tm_act, tm_lact, p, tab);
-  } else {
-    e = cudaFuncSetAttribute(qgemm2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    prof_mark(kind, true, st);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, qgemm2_kernel<false>, tm_act, tm_lact, p, tab);
-  }
-  prof_mark(kind, false, st);
+  if (a.dgrad)
+    e = nacc == 2 ? go(qgemm2_kernel<true, 2>) : go(qgemm2_kernel<true, 1>);
+  else
+    e = nacc == 2 ? go(qgemm2_kernel<false, 2>) : go(qgemm2_kernel<false, 1>);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
