@@ -36,10 +36,23 @@ namespace {
 
 constexpr int BM = 128;            // rows per CTA
 constexpr int BN = 256;            // output columns per pair (128 B-operand columns per CTA)
-constexpr int A_STAGES = 4;
+// Pipeline depths (compile-time tunables): activation stages, KB of decoded
+// operand stages, and how many of its own K-steps ahead a decode thread loads
+// its codes.
+#ifndef QLORA_PAIR_A_STAGES
+#define QLORA_PAIR_A_STAGES 4
+#endif
+#ifndef QLORA_PAIR_D_RING_KB
+#define QLORA_PAIR_D_RING_KB 96
+#endif
+#ifndef QLORA_PAIR_PREFETCH
+#define QLORA_PAIR_PREFETCH 3
+#endif
+constexpr int A_STAGES = QLORA_PAIR_A_STAGES;
 constexpr int A_BYTES = 32768;              // one activation stage: NACC x 128 rows x BK bf16
 constexpr int HALF = 16384;                 // one 128-row x 64-column swizzled atom column
-constexpr int D_RING = 98304;               // 96 KB of decoded-operand stages
+constexpr int D_RING = QLORA_PAIR_D_RING_KB * 1024;   // decoded-operand stages
+constexpr int PREFETCH = QLORA_PAIR_PREFETCH;
 constexpr int NUM_DEC_WARPS = 8;
 constexpr int THREADS = 32 * (2 + NUM_DEC_WARPS);
 constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + 256;
@@ -58,7 +71,9 @@ struct Cfg {
   static constexpr int TMEM_COLS = 256 * NACC;
   static constexpr int GROUP_WARPS = NUM_DEC_WARPS / NACC;   // decode warps per group
 };
-constexpr int MAX_D_STAGES = 6;
+constexpr int MAX_D_STAGES = 8;
+static_assert(Cfg<1>::D_STAGES >= 2 && Cfg<2>::D_STAGES <= MAX_D_STAGES, "operand ring depth");
+static_assert(A_STAGES * A_BYTES + D_RING + 1280 <= 232448, "shared memory budget");
 constexpr uint64_t kDrainLimit = 4000000000ull;
 constexpr int kGroupM = 8;                  // M-pairs per raster group
 
@@ -284,17 +299,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         b.S = __ldg(p.group_scale + (idx >> 8));
       }
     };
-    BlockLoad b0, b1, b2;
-    fetch(grp, b0);
-    fetch(grp + NACC, b1);
-    fetch(grp + 2 * NACC, b2);
+    BlockLoad bq[PREFETCH];                   // this group's next PREFETCH K-steps
+#pragma unroll
+    for (int j = 0; j < PREFETCH; ++j) fetch(grp + j * NACC, bq[j]);
     const uint32_t swz = row & 7;             // 128B swizzle of the operand
     for (int i = grp; i < nsteps; i += NACC) {
       const int sd = i % D_STAGES;
-      BlockLoad cur = b0;
-      b0 = b1;
-      b1 = b2;
-      fetch(i + 3 * NACC, b2);                // three of this group's K-steps of latency hiding
+      const BlockLoad cur = bq[0];
+#pragma unroll
+      for (int j = 0; j + 1 < PREFETCH; ++j) bq[j] = bq[j + 1];
+      fetch(i + PREFETCH * NACC, bq[PREFETCH - 1]);
       if (i >= D_STAGES &&
           !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
         break;
