@@ -189,8 +189,7 @@ Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r) {
   const size_t Mr = static_cast<size_t>(M) * r;
   if (op == QLORA_OP_FWD && M <= kGemvMaxTokens && gemv_enabled()) {
     p.gemv = true;
-    p.H = take(gemv_hpartial_bytes(M, K, r));
-    p.part = take(gemv_partial_bytes(M, N, K));
+    p.part = take(gemv_workspace_bytes(M, N, K, r));
     p.total = off;
     return p;
   }
@@ -393,8 +392,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int6
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *H = H_out ? H_out : at<float>(ws, p.H);
   if (p.gemv) {
-    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<float>(ws, p.part),
-               at<float>(ws, p.H)};
+    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<void>(ws, p.part)};
     return launch_gemv(g, st);
   }
   QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));

@@ -73,11 +73,9 @@ struct GemvArgs {
   float s;
   uint16_t *Y;
   float *H_out;        // optional [M, r]
-  float *part;         // gemv_partial_bytes() of fp32 partial sums of Y
-  float *hpart;        // gemv_hpartial_bytes() of fp32 partial sums of H
+  void *workspace;     // gemv_workspace_bytes(M, N, K, r) bytes, 256-byte aligned
 };
-size_t gemv_partial_bytes(int64_t M, int64_t N, int64_t K);
-size_t gemv_hpartial_bytes(int64_t M, int64_t K, int r);
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st);
 constexpr int kGemvMaxTokens = 16;
 bool gemv_enabled();
