@@ -194,13 +194,13 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     launches_per_gemm = (g_fwd_n + g_dg_n) / kp
     achieved = rep.gemm_flops() / (gemm_ms * 1e-3) / 1e12
     per_launch_flops = rep.gemm_flops() / launches_per_gemm
-    roofline = {"bound": "tensor", "kernel": "qgemm_kernel (fused NF4 dequant-GEMM, forward + dgrad)",
+    roofline = {"bound": "tensor", "kernel": "qgemm2_kernel (fused NF4 dequant-GEMM, forward + dgrad)",
                 "achieved": round(achieved, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_sus"], 4),
                 "peak_kind": f"bf16 dense, sustained ({pk['src']})",
                 "frac_of_burst_peak": round(achieved / pk["bf16"], 4),
                 "flops_per_launch": per_launch_flops,
-                "traffic": traffic_record("qgemm_kernel"),
+                "traffic": traffic_record("qgemm2_kernel"),
                 "share_of_step": round(gemm_ms / (all_ms / kp), 3),
                 "adapter_gemms_ms_per_step": round(lora_ms / kp, 4)}
     gpu_launches = int(round(all_n / kp * args.steps))
@@ -409,6 +409,13 @@ def run_ncu_case(args):
     q.load()
     dev = torch.device("cuda", 0)
     name = args.ncu_case
+    if name == "step":   # the timed step: the three projections, forward and backward
+        rep = Replica(q, dev)
+        for _ in range(args.warmup + args.steps):
+            rep.step()
+        torch.cuda.synchronize()
+        assert q.device_status() == 0
+        return
     case = {"q": qi.LLAMA7B[0], "up": qi.LLAMA7B[1], "down": qi.LLAMA7B[2]}.get(name, qi.LLAMA7B[1])
     M = {"gemv1": 1, "gemv16": 16}.get(name, case.M)
     d = qi.make_linear(case, M=M)
@@ -434,7 +441,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--ncu-case", choices=["q", "up", "down", "gemv1", "gemv16", "dequant"], default=None,
+    ap.add_argument("--ncu-case", choices=["step", "q", "up", "down", "gemv1", "gemv16", "dequant"], default=None,
                     help="profiling entry: run only one projection's calls (--warmup + --steps times), no JSON")
     args = ap.parse_args()
     if args.ncu_case:
