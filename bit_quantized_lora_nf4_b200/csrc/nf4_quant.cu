@@ -165,13 +165,17 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
 }
 
 // Persistent dequantizer for whole chunks of 8192 weights (128 blocks): the
-// 4 KB of codes arrive by a 1-D bulk copy, 256 threads decode 32 weights each
-// into a 16 KB shared buffer, and one thread streams it out with a bulk store.
-// Two buffers of each kind overlap the next chunk's load and the previous
-// chunk's store with the current decode.
+// 4 KB of codes and the chunk's 128 block constants arrive by 1-D bulk copies
+// into a ring of kDqStages stages issued kDqStages - 1 chunks ahead, 256
+// threads decode 32 weights each into a 16 KB shared buffer, and one thread
+// streams it out with a bulk store (two output buffers).
 constexpr int kDqChunk = 8192;
 constexpr int kDqCodeBytes = kDqChunk / 2;
+constexpr int kDqConstBytes = kDqChunk / kBlock;                 // 128 u8 block constants
+constexpr int kDqStageBytes = kDqCodeBytes + kDqConstBytes;
 constexpr int kDqOutBytes = kDqChunk * 2;
+constexpr int kDqStages = 4;
+constexpr int kDqSmem = kDqStages * kDqStageBytes + 2 * kDqOutBytes + kDqStages * 8 + 16;
 
 __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const uint8_t *__restrict__ codes,
                                                                           const uint8_t *__restrict__ absmax_q,
@@ -179,65 +183,67 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
                                                                           int64_t nchunks, uint16_t *__restrict__ out,
                                                                           Nf4Table tab, int *status,
                                                                           uint64_t wait_limit) {
-  __shared__ __align__(128) uint8_t cbuf[2][kDqCodeBytes];
-  __shared__ __align__(128) uint8_t obuf[2][kDqOutBytes];
-  __shared__ uint64_t bar[2];
-  __shared__ int abort_flag;
+  extern __shared__ __align__(128) uint8_t dq_smem[];
+  uint8_t *cbuf = dq_smem;                                         // [kDqStages][kDqStageBytes]
+  uint8_t *obuf = dq_smem + kDqStages * kDqStageBytes;             // [2][kDqOutBytes]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(obuf + 2 * kDqOutBytes);
+  int *abort_flag = reinterpret_cast<int *>(bar + kDqStages);
   const int t = threadIdx.x;
-  if (t == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
   const int64_t first = blockIdx.x;
   const int64_t step = gridDim.x;
-  if (t == 0 && first < nchunks) {
-    mbar_arrive_expect_tx(&bar[0], kDqCodeBytes);
-    bulk_load(cbuf[0], codes + first * kDqCodeBytes, kDqCodeBytes, &bar[0]);
+  int issued = 0;   // chunks whose load thread 0 has issued
+  auto issue = [&](int j) {   // the load of this CTA's chunk number j into stage j % kDqStages
+    const int64_t ch = first + j * step;
+    uint8_t *dst = cbuf + (j % kDqStages) * kDqStageBytes;
+    mbar_arrive_expect_tx(&bar[j % kDqStages], kDqStageBytes);
+    bulk_load(dst, codes + ch * kDqCodeBytes, kDqCodeBytes, &bar[j % kDqStages]);
+    bulk_load(dst + kDqCodeBytes, absmax_q + ch * kDqConstBytes, kDqConstBytes, &bar[j % kDqStages]);
+  };
+  if (t == 0) {
+    for (int i = 0; i < kDqStages; ++i) mbar_init(&bar[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    for (; issued < kDqStages && first + issued * step < nchunks; ++issued) issue(issued);
   }
+  __syncthreads();
   int it = 0;
-  int last_issued = first < nchunks ? 0 : -1;       // iteration index of the newest load (thread 0)
+  float S = first < nchunks ? __ldg(group_scale + (first >> 1)) : 0.0f;   // one group per two chunks
   for (int64_t ch = first; ch < nchunks; ch += step, ++it) {
-    const int b = it & 1;
-    // issue the next chunk's load into the other buffer (its previous contents were consumed last iteration)
-    if (t == 0 && ch + step < nchunks) {
-      mbar_arrive_expect_tx(&bar[b ^ 1], kDqCodeBytes);
-      bulk_load(cbuf[b ^ 1], codes + (ch + step) * kDqCodeBytes, kDqCodeBytes, &bar[b ^ 1]);
-      last_issued = it + 1;
-    }
-    const int64_t blk = (ch * kDqChunk + t * 32) >> 6;
-    const float ap = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(group_scale + (blk >> 8)));
+    const int ls = it % kDqStages, ob = it & 1;
+    const float S_next = ch + step < nchunks ? __ldg(group_scale + ((ch + step) >> 1)) : 0.0f;
+    // obuf[ob] was last used by the store issued two iterations ago
+    if (t == 0) bulk_wait_read<1>();
+    const bool ok = mbar_wait(&bar[ls], (it / kDqStages) & 1, wait_limit);
+    if (!ok) *abort_flag = 1;
+    __syncthreads();
+    if (*abort_flag) break;
+    const uint8_t *stage = cbuf + ls * kDqStageBytes;
+    const float ap = __fmul_rn(static_cast<float>(stage[kDqCodeBytes + (t >> 1)]), S);
     uint32_t LO[4], HI[4];
     nf4_block_table(ap, tab, LO, HI);
-    // obuf[b] was last used by the store issued two iterations ago
-    if (t == 0) bulk_wait_read<1>();
-    const bool ok = mbar_wait(&bar[b], (it >> 1) & 1, wait_limit);
-    if (!ok) abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) break;
-    const uint4 cw = ld_shared_v4(smem_addr(cbuf[b] + t * 16));
+    const uint4 cw = ld_shared_v4(smem_addr(stage + t * 16));
     const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       uint32_t o[4];
       nf4_lut8(words[w], LO, HI, o);
-      st_shared_v4(smem_addr(obuf[b] + t * 64 + w * 16), o[0], o[1], o[2], o[3]);
+      st_shared_v4(smem_addr(obuf + ob * kDqOutBytes + t * 64 + w * 16), o[0], o[1], o[2], o[3]);
     }
     fence_proxy_async_smem();
-    __syncthreads();
+    __syncthreads();   // stage ls is consumed and obuf[ob] is written
     if (t == 0) {
-      bulk_store(out + ch * kDqChunk, obuf[b], kDqOutBytes);
+      bulk_store(out + ch * kDqChunk, obuf + ob * kDqOutBytes, kDqOutBytes);
       bulk_commit();
+      if (first + issued * step < nchunks) issue(issued++);   // refill stage ls, kDqStages chunks ahead
     }
+    S = S_next;
   }
   if (t == 0) {
     bulk_wait_all<0>();
-    if (abort_flag) {
+    if (*abort_flag) {
       latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
-      // let the loads still in flight (iterations it .. last_issued) land before exiting
-      for (int j = it; j <= last_issued; ++j) mbar_wait(&bar[j & 1], (j >> 1) & 1, 4000000000ull);
+      // let the loads still in flight (chunks it .. issued - 1) land before exiting
+      for (int j = it; j < issued; ++j) mbar_wait(&bar[j % kDqStages], (j / kDqStages) & 1, 4000000000ull);
     }
   }
 }
@@ -262,7 +268,10 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
   if (nfull > 0) {
     int *status = device_status_ptr();
     int64_t blocks = nfull < 148 * 4 ? nfull : 148 * 4;
-    nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(
+    cudaError_t e = cudaFuncSetAttribute(nf4_dequantize_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDqSmem);
+    if (e != cudaSuccess) return e;
+    nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, kDqSmem, st>>>(
         codes, absmax_q, group_scale, nfull, out, nf4_table(), status, wait_limit());
   }
   const int64_t done = nfull * kDqChunk;
