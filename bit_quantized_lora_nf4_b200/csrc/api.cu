@@ -262,6 +262,16 @@ qlora_status check_ws(const void *ws, size_t ws_bytes, size_t need) {
 qlora_status run_h(const Plan &p, void *ws, const uint16_t *X, const uint16_t *A, int64_t M, int64_t K, int r,
                    float s, float *H, uint16_t *sH, uint16_t *Hs, cudaStream_t st) {
   SkinnyArgs a{X, K, true, A, K, true, M, r, K, p.spH, p.kpsH, at<float>(ws, p.part)};
+  a.ep.kind = kSkinnyH;
+  a.ep.s = s;
+  a.ep.out_f = H;
+  a.ep.out_b = sH;
+  a.ep.out_hl = Hs;
+  if (skinny_fused_ok(a)) {
+    QL_CUDA(launch_skinny(a, st));
+    return QLORA_OK;
+  }
+  a.ep = SkinnyEpilogue{};
   QL_CUDA(launch_skinny(a, st));
   QL_CUDA(launch_finalize_h(at<float>(ws, p.part), p.spH, M, r, s, H, sH, Hs, st));
   return QLORA_OK;
@@ -416,34 +426,64 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
   uint16_t *Gb = at<uint16_t>(ws, p.Gb);
   uint16_t *Gs = at<uint16_t>(ws, p.Gs);
 
-  // H (recomputed when not saved) as a hi/lo bf16 pair for dB.
+  // H (recomputed when not saved) as a hi/lo bf16 pair for dB.  With a saved H
+  // the split is done by the G product's epilogue (fused path) or a small kernel.
+  bool hs_pending = false;
   if (H_saved) {
-    QL_CUDA(launch_split_hilo(H_saved, M, r, Hs, st));
+    hs_pending = true;
   } else {
-    float *H = at<float>(ws, p.H);
-    SkinnyArgs a{X, K, true, A, K, true, M, r, K, p.spH, p.kpsH, part};
-    QL_CUDA(launch_skinny(a, st));
-    QL_CUDA(launch_finalize_h(part, p.spH, M, r, s, H, Gb /* scratch for s*H, overwritten below */, Hs, st));
+    QL_TRY(run_h(p, ws, X, A, M, K, r, s, at<float>(ws, p.H), Gb /* scratch for s*H, overwritten below */, Hs,
+                 st));
   }
   // G = s dY B  -> Gb (dgrad operand) and Gs (hi/lo, for dA)
   {
     SkinnyArgs a{dY, N, true, B, r, false, M, r, N, p.spG, p.kpsG, part};
-    QL_CUDA(launch_skinny(a, st));
-    QL_CUDA(launch_finalize_g(part, p.spG, M, r, s, Gb, Gs, st));
+    a.ep.kind = kSkinnyG;
+    a.ep.s = s;
+    a.ep.out_b = Gb;
+    a.ep.out_hl = Gs;
+    if (hs_pending) {
+      a.ep.aux = H_saved;
+      a.ep.aux_hl = Hs;
+    }
+    if (skinny_fused_ok(a)) {
+      QL_CUDA(launch_skinny(a, st));
+      hs_pending = false;
+    } else {
+      a.ep = SkinnyEpilogue{};
+      QL_CUDA(launch_skinny(a, st));
+      QL_CUDA(launch_finalize_g(part, p.spG, M, r, s, Gb, Gs, st));
+    }
   }
+  if (hs_pending) QL_CUDA(launch_split_hilo(H_saved, M, r, Hs, st));
   // dB = s dY^T H
   {
     SkinnyArgs a{dY, N, false, Hs, 2 * static_cast<int64_t>(r), false, N, 2 * static_cast<int64_t>(r), M, p.spB,
                  p.kpsB, part};
-    QL_CUDA(launch_skinny(a, st));
-    QL_CUDA(launch_finalize_cols(part, p.spB, N, r, s, dB, st));
+    a.ep.kind = kSkinnyCols;
+    a.ep.s = s;
+    a.ep.out_f = dB;
+    if (skinny_fused_ok(a)) {
+      QL_CUDA(launch_skinny(a, st));
+    } else {
+      a.ep = SkinnyEpilogue{};
+      QL_CUDA(launch_skinny(a, st));
+      QL_CUDA(launch_finalize_cols(part, p.spB, N, r, s, dB, st));
+    }
   }
   // dA = G^T X
   {
     SkinnyArgs a{Gs, 2 * static_cast<int64_t>(r), false, X, K, false, 2 * static_cast<int64_t>(r), K, M, p.spA,
                  p.kpsA, part};
-    QL_CUDA(launch_skinny(a, st));
-    QL_CUDA(launch_finalize_rows(part, p.spA, r, K, dA, st));
+    a.ep.kind = kSkinnyRows;
+    a.ep.out_f = dA;
+    if (skinny_fused_ok(a)) {
+      QL_CUDA(launch_skinny(a, st));
+    } else {
+      a.ep = SkinnyEpilogue{};
+      QL_CUDA(launch_skinny(a, st));
+      QL_CUDA(launch_finalize_rows(part, p.spA, r, K, dA, st));
+    }
   }
   // dX = dY W' + Gb A
   QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX};

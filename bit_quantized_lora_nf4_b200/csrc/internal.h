@@ -83,6 +83,24 @@ bool gemv_enabled();
 // Tall-skinny adapter products on tcgen05 tensor cores (lora_tc.cu), split over
 // the reduction with fp32 partials part[z][I][J]:  C[i,j] = sum_k opA(i,k) opB(j,k),
 // opX(i,k) = X[i*ld + k] when K-major, X[k*ld + i] otherwise.
+// What the product's epilogue writes.  With kind != kSkinnyPartial the splits
+// of one output tile run as a thread-block cluster and are added in split
+// order inside the kernel (no partial buffer, no second kernel):
+//   kSkinnyH     H = sum; out_f = H, out_b = bf16(s H), out_hl = [hi | lo] of H (optional)
+//   kSkinnyG     G = s sum; out_b = bf16(G), out_hl = [hi | lo] of G; and, when aux is set,
+//                aux_hl = [hi | lo] of the fp32 matrix aux (same [I, J] shape) for the tile's rows
+//   kSkinnyCols  out_f[i][j] = s * sum (C[i][j] + C[i][half + j]),  j < half = J / 2
+//   kSkinnyRows  out_f[i][j] = sum (C[i][j] + C[half + i][j]),      i < half = I / 2
+enum SkinnyKind { kSkinnyPartial = 0, kSkinnyH = 1, kSkinnyG = 2, kSkinnyCols = 3, kSkinnyRows = 4 };
+struct SkinnyEpilogue {
+  int kind = kSkinnyPartial;
+  float s = 1.0f;
+  float *out_f = nullptr;
+  uint16_t *out_b = nullptr;
+  uint16_t *out_hl = nullptr;
+  const float *aux = nullptr;
+  uint16_t *aux_hl = nullptr;
+};
 struct SkinnyArgs {
   const uint16_t *A;
   int64_t lda;
@@ -93,8 +111,11 @@ struct SkinnyArgs {
   int64_t I, J, Kred;
   int splits;
   int64_t k_per_split;
-  float *part;
+  float *part;                 // [splits][I][J] fp32, written only by kSkinnyPartial
+  SkinnyEpilogue ep;
 };
+// Whether the product can finish inside the kernel (cluster of its splits).
+bool skinny_fused_ok(const SkinnyArgs &a);
 cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st);
 // Pick the split count for a skinny product (deterministic in the sizes).
 void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per_split);

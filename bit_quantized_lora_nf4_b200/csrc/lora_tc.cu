@@ -10,8 +10,15 @@
 // One CTA computes a 128 x BN tile (BN = 64 .. 256) over one slice of the
 // reduction, staged by TMA in 64-deep steps into a 4-deep ring (128B swizzle,
 // K-major or MN-major as the operand is stored), issued by one thread as
-// tcgen05.mma (M = 128) into TMEM, and written as fp32 partial sums
-// part[z][i][j]; a second kernel adds the slices in a fixed order.
+// tcgen05.mma (M = 128) into TMEM.  The slices of one tile run as a thread-
+// block cluster: each CTA stages its fp32 tile in shared memory, and after a
+// cluster barrier CTA z adds rows z*128/Z .. of all Z tiles in slice order
+// through distributed shared memory and applies the epilogue (scale, bf16,
+// hi/lo split, the halves of a stacked operand).  When a tile cannot finish in
+// its cluster the kernel writes fp32 partial sums part[z][i][j] instead and a
+// second kernel adds them in the same fixed order.
+#include <cooperative_groups.h>
+
 #include "internal.h"
 
 namespace qlora {
@@ -38,9 +45,11 @@ struct TParams {
   int64_t I, J, Kred, kps;
   int bn;              // N of the MMA (multiple of 64, <= 256)
   float *part;
+  SkinnyEpilogue ep;
   int *status;
   uint64_t wait_limit;
 };
+constexpr int TPITCH_PAD = 4;   // staged tile row pitch = bn + 4 floats (spreads rows over banks)
 
 struct TSmem {
   uint64_t full[TMAX_STAGES];
@@ -64,6 +73,78 @@ __device__ __forceinline__ bool t_wait(uint64_t *bar, uint32_t parity, const TPa
       return false;
     }
   }
+}
+
+__device__ __forceinline__ uint16_t t_bf16(float x) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<const uint16_t *>(&b);
+}
+__device__ __forceinline__ float t_bf16_val(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
+
+// After every slice of the tile is staged: CTA z of the Z in the cluster adds
+// its share of the rows over all Z staged tiles in slice order (distributed
+// shared memory) and writes the epilogue's outputs; a second cluster barrier
+// keeps every staged tile alive until all its readers are done.
+__device__ __forceinline__ void cluster_finish(const TParams &p, float *stage, int64_t i0, int64_t j0) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int Z = static_cast<int>(cl.num_blocks());
+  const int z = static_cast<int>(cl.block_rank());
+  cluster_sync_all();
+  const int pitch = p.bn + TPITCH_PAD;
+  const SkinnyEpilogue &ep = p.ep;
+  const int kind = ep.kind;
+  const int64_t J = p.J;
+  const int half_j = static_cast<int>(J / 2), half_i = static_cast<int>(p.I / 2);
+  // rows of the tile this kind produces, and columns
+  const int trows = kind == kSkinnyRows ? half_i : TBM;
+  const int tcols = kind == kSkinnyCols ? half_j : static_cast<int>(J - j0 < p.bn ? J - j0 : p.bn);
+  const int per = (trows + Z - 1) / Z;
+  const int rbeg = z * per, rend = rbeg + per < trows ? rbeg + per : trows;
+  const int n = rend > rbeg ? (rend - rbeg) * tcols : 0;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int row = rbeg + e / tcols, col = e - (e / tcols) * tcols;
+    const int64_t gi = i0 + row, gj = j0 + col;
+    if (kind != kSkinnyRows && gi >= p.I) continue;
+    float v = 0.0f;
+    for (int q = 0; q < Z; ++q) {   // slice order: fixed, so the result is deterministic
+      const float *t = cl.map_shared_rank(stage, q);
+      if (kind == kSkinnyCols)
+        v = __fadd_rn(v, __fadd_rn(t[row * pitch + col], t[row * pitch + col + half_j]));
+      else if (kind == kSkinnyRows)
+        v = __fadd_rn(v, __fadd_rn(t[row * pitch + col], t[(row + half_i) * pitch + col]));
+      else
+        v = __fadd_rn(v, t[row * pitch + col]);
+    }
+    if (kind == kSkinnyH) {
+      const int64_t idx = gi * J + gj;
+      ep.out_f[idx] = v;
+      ep.out_b[idx] = t_bf16(__fmul_rn(ep.s, v));
+      if (ep.out_hl) {
+        const uint16_t hi = t_bf16(v);
+        ep.out_hl[gi * 2 * J + gj] = hi;
+        ep.out_hl[gi * 2 * J + J + gj] = t_bf16(__fsub_rn(v, t_bf16_val(hi)));
+      }
+    } else if (kind == kSkinnyG) {
+      const int64_t idx = gi * J + gj;
+      const float g = __fmul_rn(ep.s, v);
+      const uint16_t hi = t_bf16(g);
+      ep.out_b[idx] = hi;
+      ep.out_hl[gi * 2 * J + gj] = hi;
+      ep.out_hl[gi * 2 * J + J + gj] = t_bf16(__fsub_rn(g, t_bf16_val(hi)));
+      if (ep.aux) {
+        const float h = ep.aux[idx];
+        const uint16_t hh = t_bf16(h);
+        ep.aux_hl[gi * 2 * J + gj] = hh;
+        ep.aux_hl[gi * 2 * J + J + gj] = t_bf16(__fsub_rn(h, t_bf16_val(hh)));
+      }
+    } else if (kind == kSkinnyCols) {
+      ep.out_f[gi * half_j + gj] = __fmul_rn(ep.s, v);
+    } else {   // kSkinnyRows
+      ep.out_f[static_cast<int64_t>(row) * J + gj] = v;
+    }
+  }
+  cluster_sync_all();
 }
 
 template <bool A_MN, bool B_MN>
@@ -154,7 +235,28 @@ __global__ void __launch_bounds__(TTHREADS, 1)
     const bool ok = mbar_wait(&sm->acc_full, 0, kTDrain);
     tc_fence_after();
     volatile int *abort_flag = &sm->abort_flag;
-    if (__all_sync(0xffffffffu, ok && *abort_flag == 0 && nsteps > 0)) {
+    if (p.ep.kind != kSkinnyPartial) {
+      // stage this slice's tile (rows of this warp's TMEM lanes) for the cluster reduction;
+      // the ring is free: every MMA that read it has completed
+      const int quarter = warp & 3;
+      float *st = reinterpret_cast<float *>(smem) + (quarter * 32 + lane) * (p.bn + TPITCH_PAD);
+      const bool live = __all_sync(0xffffffffu, ok && *abort_flag == 0 && nsteps > 0);
+      for (int cc = 0; cc < p.bn / 32; ++cc) {
+        uint32_t v[32];
+        if (live) {
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + cc * 32, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;   // empty slice (or aborted): zero
+        }
+        float4 *dst = reinterpret_cast<float4 *>(st + cc * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+      }
+    } else if (__all_sync(0xffffffffu, ok && *abort_flag == 0 && nsteps > 0)) {
       const int quarter = warp & 3;
       const int64_t row = i0 + quarter * 32 + lane;
       float *out = p.part + static_cast<int64_t>(blockIdx.z) * p.I * p.J + row * p.J;
@@ -189,6 +291,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (p.ep.kind != kSkinnyPartial) cluster_finish(p, reinterpret_cast<float *>(smem), i0, j0);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TBN_MAX);
@@ -198,6 +301,7 @@ __global__ void __launch_bounds__(TTHREADS, 1)
 }  // namespace
 
 namespace {
+constexpr int kMaxSkinnyCluster = 8;   // portable cluster size
 int64_t tc_bn(int64_t J) {
   const int64_t b = ceil_div(J, 64) * 64;
   return b > TBN_MAX ? TBN_MAX : b;
@@ -212,11 +316,26 @@ void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per
   int64_t sp = 148 / tiles;
   const int64_t max_sp = Kred / (4 * TBK) > 0 ? Kred / (4 * TBK) : 1;
   if (sp > max_sp) sp = max_sp;
-  if (sp > 64) sp = 64;
+  if (sp > kMaxSkinnyCluster) sp = kMaxSkinnyCluster;   // the splits of a tile form one cluster
   if (sp < 1) sp = 1;
   const int64_t kps = ceil_div(ceil_div(Kred, sp), TBK) * TBK;
   *splits = static_cast<int>(ceil_div(Kred, kps));
   *k_per_split = kps;
+}
+
+bool skinny_fused_ok(const SkinnyArgs &a) {
+  const int64_t bn = tc_bn(a.J);
+  if (a.ep.kind == kSkinnyPartial || a.splits < 1 || a.splits > kMaxSkinnyCluster) return false;
+  switch (a.ep.kind) {
+    case kSkinnyH:
+    case kSkinnyG:
+    case kSkinnyCols:
+      return a.J <= bn && a.J % 2 == 0;           // one tile covers every column (and both halves)
+    case kSkinnyRows:
+      return a.I <= TBM && a.I % 2 == 0 && a.J % 4 == 0;   // one tile covers both row halves
+    default:
+      return false;
+  }
 }
 
 cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st) {
@@ -243,6 +362,9 @@ cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st) {
   p.kps = a.k_per_split;
   p.bn = static_cast<int>(bn);
   p.part = a.part;
+  const bool fused = skinny_fused_ok(a);
+  if (a.ep.kind != kSkinnyPartial && !fused) return cudaErrorInvalidValue;   // callers check first
+  p.ep = a.ep;
   p.status = device_status_ptr();
   p.wait_limit = wait_limit();
   if (!p.status) return cudaErrorInvalidValue;
@@ -251,8 +373,19 @@ cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st) {
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TSMEM);
     if (e != cudaSuccess) return e;
-    kern<<<grid, TTHREADS, TSMEM, st>>>(tmA, tmB, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(TTHREADS);
+    cfg.dynamicSmemBytes = TSMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;   // the splits of one tile: one cluster
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = fused ? static_cast<unsigned>(a.splits) : 1u;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p);
   };
   prof_mark(kProfLora, true, st);
   cudaError_t e;

@@ -174,7 +174,13 @@ constexpr int kDqCodeBytes = kDqChunk / 2;
 constexpr int kDqConstBytes = kDqChunk / kBlock;                 // 128 u8 block constants
 constexpr int kDqStageBytes = kDqCodeBytes + kDqConstBytes;
 constexpr int kDqOutBytes = kDqChunk * 2;
-constexpr int kDqStages = 4;
+#ifndef QLORA_DQ_STAGES
+#define QLORA_DQ_STAGES 4
+#endif
+#ifndef QLORA_DQ_CTAS_PER_SM
+#define QLORA_DQ_CTAS_PER_SM 4
+#endif
+constexpr int kDqStages = QLORA_DQ_STAGES;
 constexpr int kDqSmem = kDqStages * kDqStageBytes + 2 * kDqOutBytes + kDqStages * 8 + 16;
 
 __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const uint8_t *__restrict__ codes,
@@ -267,7 +273,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
   prof_mark(kProfDequant, true, st);
   if (nfull > 0) {
     int *status = device_status_ptr();
-    int64_t blocks = nfull < 148 * 4 ? nfull : 148 * 4;
+    int64_t blocks = nfull < 148 * QLORA_DQ_CTAS_PER_SM ? nfull : 148 * QLORA_DQ_CTAS_PER_SM;
     cudaError_t e = cudaFuncSetAttribute(nf4_dequantize_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kDqSmem);
     if (e != cudaSuccess) return e;
