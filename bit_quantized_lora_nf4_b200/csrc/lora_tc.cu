@@ -30,7 +30,11 @@ constexpr int TBN_MAX = 256;
 constexpr int TBK = 64;
 constexpr int TMAX_STAGES = 8;
 constexpr int TA_BYTES = TBM * TBK * 2;         // 16 KB
-constexpr int TRING_BYTES = 196608;             // 192 KB of stages: one CTA per SM
+#ifndef QLORA_TC_RING_KB
+#define QLORA_TC_RING_KB 104
+#endif
+constexpr int TRING_BYTES = QLORA_TC_RING_KB * 1024;   // stages (104 KB: two CTAs per SM)
+constexpr int TCTAS_PER_SM = TRING_BYTES > 110 * 1024 ? 1 : 2;
 constexpr int TTHREADS = 192;                   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int TSMEM = TRING_BYTES + 1024 + 256;
 
@@ -312,8 +316,8 @@ void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per
   int64_t tiles = ceil_div(I, TBM) * ceil_div(J, tc_bn(J));
   if (tiles < 1) tiles = 1;
   if (Kred < 1) Kred = 1;
-  // one CTA per SM (192 KB of stages): keep every split of every tile in one wave
-  int64_t sp = 148 / tiles;
+  // keep every split of every tile in one wave
+  int64_t sp = 148 * TCTAS_PER_SM / tiles;
   const int64_t max_sp = Kred / (4 * TBK) > 0 ? Kred / (4 * TBK) : 1;
   if (sp > max_sp) sp = max_sp;
   if (sp > kMaxSkinnyCluster) sp = kMaxSkinnyCluster;   // the splits of a tile form one cluster
@@ -326,6 +330,7 @@ void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per
 bool skinny_fused_ok(const SkinnyArgs &a) {
   const int64_t bn = tc_bn(a.J);
   if (a.ep.kind == kSkinnyPartial || a.splits < 1 || a.splits > kMaxSkinnyCluster) return false;
+  if (static_cast<int64_t>(TBM) * (bn + TPITCH_PAD) * 4 > TRING_BYTES) return false;   // staged tile fits the ring
   switch (a.ep.kind) {
     case kSkinnyH:
     case kSkinnyG:
