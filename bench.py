@@ -295,6 +295,17 @@ def measure_extras(q, rep, dev, pk, barrier):
         gbs = tot_bytes / (tot_ms * 1e-3) / 1e9
         res[str(M)] = {"value": round(gbs, 1), "frac": round(gbs / pk["hbm"], 4), "us_per_call_avg": round(
             1e3 * tot_ms / len(rep.cases), 2)}
+    # the 4-bit tables the pages compare NF4 against: reconstruction error through the library
+    Wq = qi.make_weight(4096, 4096, qi.LLAMA7B[0].seed).to(dev)
+    errs = {}
+    for name, fid in (("nf4", q.FORMAT_NF4), ("fp4", q.FORMAT_FP4), ("int4", q.FORMAT_INT4)):
+        wq = q.quantize_nf4(Wq, format=fid)
+        d = q.dequantize(wq).double() - Wq.double()
+        errs[name] = round(float(d.norm() / Wq.double().norm()), 5)
+        del wq, d
+    del Wq
+    out["formats"] = {"rel_frobenius_error": errs, "note": "||dequant(quant(W)) - W|| / ||W|| on the 4096x4096 "
+                      "Gaussian q-projection weight, blocks of 64, double-quantized constants"}
     out["gemv"] = {"unit": "GB/s", "tokens": res,
                    "note": "packed weight + adapters + X + Y bytes per call; calls replayed from a CUDA graph, "
                            "weights rotated over copies totalling > 400 MB (beyond L2)"}

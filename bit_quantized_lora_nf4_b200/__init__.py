@@ -32,8 +32,12 @@ EXPORTS = (
     "qlora_codes_bytes", "qlora_absmax_bytes", "qlora_group_scale_bytes", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
     "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
-    "qlora_profile_read", "qlora_linear_fwd_noalloc",
+    "qlora_profile_read", "qlora_linear_fwd_noalloc", "qlora_format_codebook",
 )
+
+# 4-bit code tables (QLORA_FORMAT_*): NF4 is the method's type; FP4 (e2m1) and
+# INT4 are the plain float and integer types it is compared against.
+FORMAT_NF4, FORMAT_FP4, FORMAT_INT4 = 0, 1, 2
 
 # Kernel kinds of the timing hook (qlora_profile_read).
 PROF_ALL, PROF_GEMM_FWD, PROF_GEMM_DGRAD, PROF_LORA, PROF_QUANT, PROF_DEQUANT, PROF_GEMV = range(7)
@@ -47,7 +51,8 @@ class QloraError(RuntimeError):
 
 class Nf4WeightC(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p),
-                ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p)]
+                ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p), ("format", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 _lib = None
@@ -73,6 +78,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_linear_fwd": (i32, [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "qlora_linear_bwd": (i32, [wp, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "qlora_nf4_codebook": (i32, [ctypes.POINTER(ctypes.c_float)]),
+        "qlora_format_codebook": (i32, [i32, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
         "qlora_device_status": (i32, [vp]),
         "qlora_status_string": (ctypes.c_char_p, [i32]),
         "qlora_set_wait_limit": (ctypes.c_uint64, [ctypes.c_uint64]),
@@ -110,29 +116,32 @@ class NF4Weight:
     codes: torch.Tensor        # uint8 [ceil(rows*cols/2)]
     absmax_q: torch.Tensor     # uint8 [ceil(rows*cols/64)]
     group_scale: torch.Tensor  # float32 [ceil(rows*cols/16384)]
+    format: int = FORMAT_NF4   # code table (FORMAT_*)
 
     def c_struct(self) -> Nf4WeightC:
         return Nf4WeightC(self.rows, self.cols, self.codes.data_ptr(), self.absmax_q.data_ptr(),
-                          self.group_scale.data_ptr())
+                          self.group_scale.data_ptr(), self.format, 0)
 
     @staticmethod
-    def empty(rows: int, cols: int, device="cuda") -> "NF4Weight":
+    def empty(rows: int, cols: int, device="cuda", format: int = FORMAT_NF4) -> "NF4Weight":
         lib = load()
         return NF4Weight(rows, cols,
                          torch.empty(lib.qlora_codes_bytes(rows, cols), dtype=torch.uint8, device=device),
                          torch.empty(lib.qlora_absmax_bytes(rows, cols), dtype=torch.uint8, device=device),
                          torch.empty(lib.qlora_group_scale_bytes(rows, cols) // 4, dtype=torch.float32,
-                                     device=device))
+                                     device=device), format)
 
     def nbytes(self) -> int:
         return self.codes.numel() + self.absmax_q.numel() + 4 * self.group_scale.numel()
 
 
-def codebook() -> list:
+def codebook(format: int = FORMAT_NF4, thresholds: bool = False):
+    """The 16 levels of a code table (and its 15 decision thresholds when asked)."""
     lib = load()
-    out = (ctypes.c_float * 16)()
-    _check(lib.qlora_nf4_codebook(out), "qlora_nf4_codebook")
-    return list(out)
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    _check(lib.qlora_format_codebook(format, lv, th), "qlora_format_codebook")
+    return (list(lv), list(th)) if thresholds else list(lv)
 
 
 def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
@@ -164,12 +173,13 @@ def profile_read(kind: int):
     return ms.value, n.value
 
 
-def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None) -> NF4Weight:
-    """Quantize a contiguous fp32 CUDA tensor [rows, cols] (flat row-major)."""
+def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, format: int = FORMAT_NF4) -> NF4Weight:
+    """Quantize a contiguous fp32 CUDA tensor [rows, cols] (flat row-major) to a
+    4-bit table (NF4 unless `format` says otherwise, or `out.format` when given)."""
     lib = load()
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
     rows, cols = (W.shape[0], W[0].numel()) if W.dim() >= 2 else (1, W.numel())
-    w = out if out is not None else NF4Weight.empty(rows, cols, W.device)
+    w = out if out is not None else NF4Weight.empty(rows, cols, W.device, format)
     s = w.c_struct()
     _check(lib.qlora_quantize_nf4(_ptr(W), ctypes.byref(s), _stream()), "qlora_quantize_nf4")
     return w

@@ -44,13 +44,43 @@ Nf4Table build_nf4_table() {
   for (int i = 0; i < 16; ++i) top = fmaxl(top, fabsl(v[i]));
   Nf4Table t{};
   for (int i = 0; i < 16; ++i) t.level[i] = static_cast<float>(v[i] / top);
-  // thresholds: exact midpoint (representable in double) rounded toward -inf to fp32
-  for (int i = 0; i < 15; ++i) {
+  return t;
+}
+
+// Decision thresholds of an ascending table: code = #{ i : n > thresh[i] } is the
+// nearest level with ties to the lower index.  thresh[i] = exact midpoint of
+// level[i] and level[i+1] (representable in double) rounded toward -inf to fp32;
+// between two equal levels the upper one is never nearer, so the threshold is
+// the next one (code i+1 is skipped).
+void set_thresholds(Nf4Table &t) {
+  for (int i = 14; i >= 0; --i) {
+    if (t.level[i] == t.level[i + 1] && i < 14) {
+      t.thresh[i] = t.thresh[i + 1];
+      continue;
+    }
     const double mid = (static_cast<double>(t.level[i]) + static_cast<double>(t.level[i + 1])) * 0.5;
     float f = static_cast<float>(mid);
     if (static_cast<double>(f) > mid) f = nextafterf(f, -INFINITY);
     t.thresh[i] = f;
   }
+}
+
+Nf4Table build_table(int format) {
+  Nf4Table t{};
+  if (format == QLORA_FORMAT_NF4) {
+    t = build_nf4_table();
+  } else if (format == QLORA_FORMAT_FP4) {
+    // e2m1: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (scaled by 1/6 so the largest is 1);
+    // codes 0..7 carry the negative values from -1 up to -0, codes 8..15 +0 up to +1
+    const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    for (int i = 0; i < 8; ++i) {
+      t.level[7 - i] = -mag[i] / 6.0f;
+      t.level[8 + i] = mag[i] / 6.0f;
+    }
+  } else {   // QLORA_FORMAT_INT4
+    for (int c = 0; c < 16; ++c) t.level[c] = static_cast<float>(c - 8) / 7.0f;
+  }
+  set_thresholds(t);
   return t;
 }
 
@@ -69,10 +99,13 @@ __global__ void selftest_wait_kernel(uint64_t limit, int *status) {
 
 }  // namespace
 
-const Nf4Table &nf4_table() {
-  static const Nf4Table t = build_nf4_table();
-  return t;
+const Nf4Table &format_table(int format) {
+  static const Nf4Table t[3] = {build_table(QLORA_FORMAT_NF4), build_table(QLORA_FORMAT_FP4),
+                                build_table(QLORA_FORMAT_INT4)};
+  return t[format == QLORA_FORMAT_FP4 ? 1 : (format == QLORA_FORMAT_INT4 ? 2 : 0)];
 }
+
+const Nf4Table &nf4_table() { return format_table(QLORA_FORMAT_NF4); }
 
 uint64_t wait_limit() { return g_wait_limit.load(); }
 
@@ -224,6 +257,7 @@ T *at(void *ws, size_t off) {
 qlora_status check_weight(const qlora_nf4_weight *w) {
   if (!w || !w->codes || !w->absmax_q || !w->group_scale) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < 1) return QLORA_ERR_INVALID_ARG;
+  if (w->format < QLORA_FORMAT_NF4 || w->format > QLORA_FORMAT_INT4 || w->reserved != 0) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale)) return QLORA_ERR_MISALIGNED;
   return QLORA_OK;
 }
@@ -315,6 +349,14 @@ qlora_status qlora_nf4_codebook(float *out) {
   return QLORA_OK;
 }
 
+qlora_status qlora_format_codebook(int format, float *levels, float *thresh) {
+  if (!levels || format < QLORA_FORMAT_NF4 || format > QLORA_FORMAT_INT4) return QLORA_ERR_INVALID_ARG;
+  const Nf4Table &t = format_table(format);
+  std::memcpy(levels, t.level, sizeof(float) * 16);
+  if (thresh) std::memcpy(thresh, t.thresh, sizeof(float) * 15);
+  return QLORA_OK;
+}
+
 uint64_t qlora_set_wait_limit(uint64_t cycles) { return g_wait_limit.exchange(cycles); }
 
 void qlora_profile_enable(int on) {
@@ -376,8 +418,8 @@ qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, voi
   if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
   int *status = device_status_ptr();
   if (!status) return QLORA_ERR_CUDA;
-  QL_CUDA(launch_quantize(W, out->rows * out->cols, out->codes, out->absmax_q, out->group_scale, status,
-                          static_cast<cudaStream_t>(stream)));
+  QL_CUDA(launch_quantize(W, out->rows * out->cols, out->codes, out->absmax_q, out->group_scale, out->format,
+                          status, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
 }
 
@@ -385,8 +427,8 @@ qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *
   if (!W_out) return QLORA_ERR_INVALID_ARG;
   QL_TRY(check_weight(w));
   if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
-  QL_CUDA(launch_dequantize(w->codes, w->absmax_q, w->group_scale, w->rows * w->cols, W_out,
-                            static_cast<cudaStream_t>(stream)));
+  QL_CUDA(launch_dequantize(w->codes, w->absmax_q, w->group_scale, w->rows * w->cols, w->format,
+                            W_out, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
 }
 
@@ -402,11 +444,12 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int6
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *H = H_out ? H_out : at<float>(ws, p.H);
   if (p.gemv) {
-    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<void>(ws, p.part)};
+    GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<void>(ws, p.part),
+               w->format};
     return launch_gemv(g, st);
   }
   QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
-  QGemmArgs g{false, M, N, K, X, w->codes, w->absmax_q, w->group_scale, at<uint16_t>(ws, p.sH), B, r, Y};
+  QGemmArgs g{false, M, N, K, X, w->codes, w->absmax_q, w->group_scale, at<uint16_t>(ws, p.sH), B, r, Y, w->format};
   return launch_qgemm(g, st);
 }
 
@@ -486,7 +529,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
     }
   }
   // dX = dY W' + Gb A
-  QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX};
+  QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX, w->format};
   return launch_qgemm(g, st);
 }
 

@@ -680,7 +680,7 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
                reinterpret_cast<float *>(ws + L.off_pieces), reinterpret_cast<float *>(ws + L.off_hpart),
                static_cast<int>(a.M), a.r, L.r16, L.JT, L.HS, static_cast<int>(G), static_cast<int>(L.S),
                static_cast<int>(L.U), static_cast<int>(L.T), L.P, xs ? xs_row_bytes(KB) : 0, a.wN, a.wK, status,
-               wait_limit(), nf4_table()};
+               wait_limit(), format_table(a.format)};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(GV_THREADS);

@@ -12,6 +12,8 @@ namespace qlora {
 
 // NF4 table computed once on the host (normal quantiles, see api.cu).
 const Nf4Table &nf4_table();
+// The table of a QLORA_FORMAT_* (the NF4 one for QLORA_FORMAT_NF4); format must be valid.
+const Nf4Table &format_table(int format);
 
 // Address of the device status word on the current device (nullptr on error).
 int *device_status_ptr();
@@ -36,9 +38,9 @@ bool make_tmap_2d(CUtensorMap *tm, const void *base, CUtensorMapDataType dtype, 
 
 // ---- kernels (launchers return the launch error) -------------------------------
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
-                            int *status, cudaStream_t st);
+                            int format, int *status, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
-                              int64_t numel, uint16_t *out, cudaStream_t st);
+                              int64_t numel, int format, uint16_t *out, cudaStream_t st);
 
 // Fused dequant-GEMM on tensor cores.
 //   forward: out[M, wN] = act[M, wK] . W'^T + lora_act[M, r] . lora_w[wN, r]^T
@@ -55,6 +57,7 @@ struct QGemmArgs {
   const uint16_t *lora_w;
   int r;
   uint16_t *out;
+  int format;          // QLORA_FORMAT_* of the weight
 };
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
 // The same product on a CTA pair (256-row tiles); launch_qgemm dispatches to it for M > 128.
@@ -74,6 +77,7 @@ struct GemvArgs {
   uint16_t *Y;
   float *H_out;        // optional [M, r]
   void *workspace;     // gemv_workspace_bytes(M, N, K, r) bytes, 256-byte aligned
+  int format;          // QLORA_FORMAT_* of the weight
 };
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st);

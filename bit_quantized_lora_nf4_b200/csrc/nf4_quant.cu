@@ -257,16 +257,17 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
 }  // namespace
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
-                            int *status, cudaStream_t st) {
+                            int format, int *status, cudaStream_t st) {
   const int64_t ngroups = (numel + kGroupElems - 1) / kGroupElems;
   prof_mark(kProfQuant, true, st);
   nf4_quantize_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(W, numel, codes, absmax_q,
-                                                                                 group_scale, nf4_table(), status);
+                                                                                 group_scale, format_table(format), status);
   prof_mark(kProfQuant, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale, int64_t numel,
+                              int format,
                               uint16_t *out, cudaStream_t st) {
   // whole double-quantization groups (two chunks each) on the bulk path
   const int64_t nfull = (numel / (kBlock * kGroup)) * (kBlock * kGroup / kDqChunk);
@@ -278,7 +279,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
                                          kDqSmem);
     if (e != cudaSuccess) return e;
     nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, kDqSmem, st>>>(
-        codes, absmax_q, group_scale, nfull, out, nf4_table(), status, wait_limit());
+        codes, absmax_q, group_scale, nfull, out, format_table(format), status, wait_limit());
   }
   const int64_t done = nfull * kDqChunk;
   if (done < numel) {
@@ -289,7 +290,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
     int64_t blocks = (nchunk + kDeqThreads - 1) / kDeqThreads;
     nf4_dequantize_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(
         codes + done / 2, absmax_q + done / kBlock, group_scale + done / (kBlock * kGroup), rest, out + done,
-        nf4_table());
+        format_table(format));
   }
   prof_mark(kProfDequant, false, st);
   return cudaGetLastError();

@@ -349,11 +349,11 @@ qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st) {
   if (a.dgrad) {
     e = cudaFuncSetAttribute(qgemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) qgemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, nf4_table());
+    if (e == cudaSuccess) qgemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, format_table(a.format));
   } else {
     e = cudaFuncSetAttribute(qgemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) qgemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, nf4_table());
+    if (e == cudaSuccess) qgemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, format_table(a.format));
   }
   prof_mark(kind, false, st);
   if (e == cudaSuccess) e = cudaGetLastError();

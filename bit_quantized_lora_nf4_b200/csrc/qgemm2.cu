@@ -439,7 +439,7 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const Nf4Table tab = nf4_table();
+  const Nf4Table tab = format_table(a.format);
   const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);

@@ -66,12 +66,27 @@ typedef enum {
  *   codes       : ceil(rows*cols/2) bytes
  *   absmax_q    : ceil(rows*cols/64) bytes, one unsigned 8-bit constant per block
  *   group_scale : ceil(rows*cols/16384) fp32, one per group of 256 blocks     */
+/* 4-bit code tables.  NF4 is the method's type; the other two are the plain
+ * 4-bit float and integer types the pages compare it against (the same
+ * storage, block constants and kernels, another 16-entry table):
+ *   QLORA_FORMAT_NF4   levels at normal quantiles (qlora_nf4_codebook)
+ *   QLORA_FORMAT_FP4   e2m1 float: +-{0, 0.5, 1, 1.5, 2, 3, 4, 6} / 6, codes
+ *                      0..7 negative (code 7 = -0), 8..15 positive (code 8 = +0;
+ *                      nearest-level encoding with ties to the lower index never
+ *                      emits code 8)
+ *   QLORA_FORMAT_INT4  symmetric integer grid: level[c] = fl32((c - 8) / 7) */
+#define QLORA_FORMAT_NF4 0
+#define QLORA_FORMAT_FP4 1
+#define QLORA_FORMAT_INT4 2
+
 typedef struct {
   int64_t rows;
   int64_t cols;
   uint8_t *codes;
   uint8_t *absmax_q;
   float *group_scale;
+  int32_t format;     /* QLORA_FORMAT_*; 0 (NF4) for a zero-initialised struct */
+  int32_t reserved;   /* must be 0 */
 } qlora_nf4_weight;
 
 /* Sizes in bytes of the three arrays for a rows x cols weight. */
@@ -79,13 +94,14 @@ size_t qlora_codes_bytes(int64_t rows, int64_t cols);
 size_t qlora_absmax_bytes(int64_t rows, int64_t cols);
 size_t qlora_group_scale_bytes(int64_t rows, int64_t cols);
 
-/* qlora_quantize_nf4 -- quantize fp32 weights once, up front.
+/* qlora_quantize_nf4 -- quantize fp32 weights once, up front (in out->format;
+ * NF4 unless the caller chose another table).
  * ("Where the memory goes": the base never changes, so it is quantized once.)
  *   W   : device fp32 [out->rows * out->cols], flat row-major.
  *   out : rows/cols set by the caller; codes/absmax_q/group_scale receive the
  *         result.  Any rows*cols >= 1 is accepted (last block/group partial).
  * Per block b: a_b = max|w| (exact fp32); n = fl32(w / a_b) (n = 0 if a_b = 0);
- * code = index of the nearest NF4 level, ties to the lower index.
+ * code = index of the nearest level of the table, ties to the lower index.
  * Per group g: c_g = max a_b; S_g = fl32(c_g / 255);
  * q_b = min(255, round-half-even(fl32(a_b / S_g))) (0 if S_g = 0).
  * A non-finite weight latches QLORA_ERR_NONFINITE (outputs then undefined). */
@@ -165,6 +181,14 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_weight *w, const uint16_t 
  * normalised to [-1, 1].  ("NormalFloat, double quantization, paged
  * optimizers": 16 levels at normal quantiles.)  out: host float[16]. */
 qlora_status qlora_nf4_codebook(float *out);
+
+/* The 16 fp32 levels of any QLORA_FORMAT_* table (ascending), and the 15 fp32
+ * decision thresholds the quantizer compares against: code = #{ i : n >
+ * thresh[i] }, thresh[i] = the midpoint of level[i] and level[i+1] rounded
+ * toward -inf (for two equal levels, the next threshold).  levels: host
+ * float[16]; thresh: host float[15] or NULL.  QLORA_ERR_INVALID_ARG for an
+ * unknown format or a NULL levels pointer. */
+qlora_status qlora_format_codebook(int format, float *levels, float *thresh);
 
 /* Synchronize `stream`, return the latched device status and clear it. */
 qlora_status qlora_device_status(void *stream);

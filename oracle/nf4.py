@@ -64,6 +64,42 @@ def nf4_levels_exact(dps: int = 50):
     return [v / top for v in vals]
 
 
+FORMATS = ("nf4", "fp4", "int4")
+
+
+def fp4_codebook() -> np.ndarray:
+    """Plain 4-bit float ([Blog-nf4] / [Cap-qlora] name it only as the weaker
+    alternative; reading: the e2m1 layout, 1 sign, 2 exponent, 1 mantissa bit,
+    magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) scaled by 1/6 so the largest level is
+    1.  Codes 0..7 hold -1 .. -0 ascending, codes 8..15 hold +0 .. +1.  The two
+    zeros are equal, so nearest-level encoding with ties to the lower index
+    never emits code 8."""
+    mag = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float32)
+    pos = (mag / np.float32(6.0)).astype(np.float32)
+    neg = (-mag[::-1] / np.float32(6.0)).astype(np.float32)   # -1 .. -0 (the last one is -0.0)
+    return np.concatenate([neg, pos]).astype(np.float32)
+
+
+def int4_codebook() -> np.ndarray:
+    """Plain 4-bit integer grid ([Blog-nf4]: NF4 beats plain integer types;
+    reading: symmetric absmax scaling, the block maximum maps to 7):
+    level[c] = fl32((c - 8) / 7), c = 0..15 (level[0] = -8/7 is never the
+    nearest level of a normalised value in [-1, 1])."""
+    c = np.arange(16, dtype=np.float32)
+    return ((c - np.float32(8.0)) / np.float32(7.0)).astype(np.float32)
+
+
+def codebook(fmt: str = "nf4") -> np.ndarray:
+    """The 16 ascending fp32 levels of a 4-bit table."""
+    if fmt == "nf4":
+        return nf4_codebook()
+    if fmt == "fp4":
+        return fp4_codebook()
+    if fmt == "int4":
+        return int4_codebook()
+    raise ValueError(fmt)
+
+
 def nf4_codebook() -> np.ndarray:
     """The 16 levels rounded to fp32 (round-to-nearest), ascending."""
     return np.array([float(v) for v in nf4_levels_exact()], dtype=np.float64).astype(np.float32)
@@ -201,7 +237,7 @@ def dequantize_absmax(q: np.ndarray, S: np.ndarray) -> np.ndarray:
     return (q.astype(np.float32) * Sb).astype(np.float32)
 
 
-def quantize_nf4(W: np.ndarray):
+def quantize_nf4(W: np.ndarray, fmt: str = "nf4"):
     """Quantize fp32 weights once, up front ([Blog-mem]: the base never changes,
     so it is quantized once).
 
@@ -219,14 +255,14 @@ def quantize_nf4(W: np.ndarray):
     flat = W.ravel()
     a = block_absmax(flat)
     n = normalize(flat, a)
-    codes = nearest_code(n, nf4_codebook())
+    codes = nearest_code(n, codebook(fmt))
     q, S = double_quantize(a)
     return {"codes": pack_nibbles(codes), "absmax_q": q, "group_scale": S,
-            "shape": tuple(W.shape)}
+            "shape": tuple(W.shape), "format": fmt}
 
 
 def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np.ndarray,
-                        shape) -> np.ndarray:
+                        shape, fmt: str = "nf4") -> np.ndarray:
     """W' = bf16(fl32(v_code * a'_b)) with a'_b = fl32(q_b * S_g); bf16 bit patterns.
 
     [Blog-mem]: every forward and backward pass expands the 4-bit base back
@@ -235,7 +271,7 @@ def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np
     """
     numel = int(np.prod(shape))
     c = unpack_nibbles(codes, numel)
-    v = nf4_codebook()[c]
+    v = codebook(fmt)[c]
     ap = np.repeat(dequantize_absmax(absmax_q, group_scale), BLOCK)[:numel]
     w32 = (v * ap).astype(np.float32)
     return bf16_rne_bits(w32).reshape(shape)
@@ -243,4 +279,14 @@ def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np
 
 def dequantize_nf4(q: dict) -> np.ndarray:
     """Convenience: dequantize a quantize_nf4() result to bf16 bit patterns."""
-    return dequantize_nf4_bits(q["codes"], q["absmax_q"], q["group_scale"], q["shape"])
+    return dequantize_nf4_bits(q["codes"], q["absmax_q"], q["group_scale"], q["shape"], q.get("format", "nf4"))
+
+
+def reconstruction_error(W: np.ndarray, fmt: str = "nf4") -> float:
+    """Relative Frobenius error ||bf16 dequant(quant(W)) - W|| / ||W|| of a 4-bit
+    table on the given weights: the proxy, on Gaussian weights, for the pages'
+    statement that NF4 beats plain 4-bit float and integer types ([Blog-nf4])."""
+    W = np.asarray(W, dtype=np.float32)
+    Wd = bf16_bits_to_f32(dequantize_nf4(quantize_nf4(W, fmt))).astype(np.float64)
+    W64 = W.astype(np.float64)
+    return float(np.linalg.norm(Wd - W64) / np.linalg.norm(W64))
