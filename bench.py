@@ -111,10 +111,10 @@ class ClockSampler:
 class Replica:
     """Device-resident inputs, outputs and workspaces of the three projections."""
 
-    def __init__(self, q, dev):
+    def __init__(self, q, dev, cases=qi.LLAMA7B):
         self.q = q
         self.cases = []
-        for case in qi.LLAMA7B:
+        for case in cases:
             d = qi.make_linear(case)
             w = q.quantize_nf4(d["W"].to(dev))
             M, N, K, r = case.M, case.N, case.K, case.r
@@ -206,6 +206,7 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     gpu_launches = int(round(all_n / kp * args.steps))
 
     extras = measure_extras(q, rep, dev, pk, barrier)
+    extras["llama65b"] = measure_65b(q, dev, pk, barrier)
     e2e = measure_e2e(q, rep, dev, min(args.steps, 20), barrier, allmax, world)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -221,6 +222,25 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(world)
         print(json.dumps(line), flush=True)
+
+
+def measure_65b(q, dev, pk, barrier):
+    """The LLaMA-65B-shaped projections (8192 x 8192, 22016 x 8192, 8192 x 22016; 8192 tokens, r = 64),
+    one fwd + bwd of each per step, device-timed like the main line (a parity-test configuration,
+    reported beside the main line)."""
+    rep = Replica(q, dev, qi.LLAMA65B)
+    for _ in range(3):
+        rep.step()
+    torch.cuda.synchronize()
+    steps = 10
+    ms = timed(rep.step, steps, barrier) / steps
+    tf = rep.flops() / (ms * 1e-3) / 1e12
+    out = {"value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+           "frac_of_bf16_peak": round(tf / pk["bf16_sus"], 4), "flops_per_step": rep.flops(),
+           "workload": "llama65b_projections_q8192x8192_up22016x8192_down8192x22016_m8192_r64_fwd_bwd"}
+    del rep
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_extras(q, rep, dev, pk, barrier):

@@ -187,6 +187,30 @@ def nearest_code(n: np.ndarray, levels: np.ndarray, chunk: int = 1 << 20) -> np.
     return out
 
 
+def nearest_code_fast(n: np.ndarray, levels: np.ndarray) -> np.ndarray:
+    """The same code as nearest_code (nearest level, ties to the lower index),
+    for large inputs: with ascending levels, the nearest level of n is the
+    number of midpoints strictly below n, each midpoint of two fp32 levels
+    being exact in fp64; between two equal levels the upper one is never
+    strictly nearer, so that midpoint is skipped.  Equality with the argmin
+    definition is checked by the tests on dense probes around every midpoint."""
+    v = np.asarray(levels, dtype=np.float32).astype(np.float64)
+    mids = [(v[i] + v[i + 1]) / 2 for i in range(len(v) - 1) if v[i] != v[i + 1]]
+    skip = [i for i in range(len(v) - 1) if v[i] == v[i + 1]]
+    x = np.asarray(n, dtype=np.float32).ravel().astype(np.float64)
+    k = np.searchsorted(np.array(mids), x, side="left")     # midpoints strictly below x
+    # map the count over distinct-level midpoints back to a code index
+    code_of = []
+    c = 0
+    for i in range(len(v) - 1):
+        if i in skip:
+            continue
+        code_of.append(c)
+        c = i + 1
+    code_of.append(c)
+    return np.asarray(code_of, dtype=np.uint8)[k]
+
+
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:
     """Two 4-bit codes per byte: element 2j -> low nibble, 2j+1 -> high nibble."""
     c = np.asarray(codes, dtype=np.uint8).ravel()
@@ -255,7 +279,7 @@ def quantize_nf4(W: np.ndarray, fmt: str = "nf4"):
     flat = W.ravel()
     a = block_absmax(flat)
     n = normalize(flat, a)
-    codes = nearest_code(n, codebook(fmt))
+    codes = nearest_code(n, codebook(fmt)) if n.size <= (1 << 24) else nearest_code_fast(n, codebook(fmt))
     q, S = double_quantize(a)
     return {"codes": pack_nibbles(codes), "absmax_q": q, "group_scale": S,
             "shape": tuple(W.shape), "format": fmt}

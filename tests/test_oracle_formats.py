@@ -100,3 +100,23 @@ def test_library_rejects_unknown_formats(lib):
     lv = (ctypes.c_float * 16)()
     assert lib.load().qlora_format_codebook(3, lv, None) == 1
     assert lib.load().qlora_format_codebook(-1, lv, None) == 1
+
+
+@pytest.mark.parametrize("fmt", nf4.FORMATS)
+def test_fast_encoder_equals_the_argmin_definition(fmt):
+    """The midpoint-count encoder used for large weights returns the same code
+    as the nearest-level argmin (ties low) on dense probes around every
+    midpoint and on random values."""
+    lv = nf4.codebook(fmt)
+    probes = []
+    for i in range(15):
+        v = np.float32((np.float64(lv[i]) + np.float64(lv[i + 1])) / 2)
+        for _ in range(4):
+            v = np.nextafter(v, np.float32(-np.inf))
+        for _ in range(9):
+            probes.append(v)
+            v = np.nextafter(v, np.float32(np.inf))
+    rng = np.random.default_rng(5)
+    n = np.concatenate([np.array(probes, np.float32), rng.uniform(-1, 1, 100000).astype(np.float32),
+                        np.array([0.0, -0.0, 1.0, -1.0], np.float32)])
+    assert np.array_equal(nf4.nearest_code(n, lv), nf4.nearest_code_fast(n, lv))
