@@ -207,6 +207,7 @@ def run_ours(args, rank, world, dev, barrier, allmax):
 
     extras = measure_extras(q, rep, dev, pk, barrier)
     extras["llama65b"] = measure_65b(q, dev, pk, barrier)
+    extras["decoder_layer"] = measure_layer(q, dev, pk, barrier)
     e2e = measure_e2e(q, rep, dev, min(args.steps, 20), barrier, allmax, world)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -222,6 +223,50 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(world)
         print(json.dumps(line), flush=True)
+
+
+def measure_layer(q, dev, pk, barrier):
+    """One fwd + bwd step of a LLaMA-7B-shaped decoder layer (batch 4 x seq 2048, d 4096, 32 heads,
+    SwiGLU 11008, RMSNorm) whose seven projections are the library's NF4 + LoRA (r = 64) linears and
+    whose glue (norms, rotary embedding, attention, SwiGLU) is torch.  The linears' share is measured
+    by the library's own per-launch events in a second pass."""
+    import qlora_layer as ql
+    cfg = ql.LayerConfig()
+    params = ql.make_params(cfg, seed=21)
+    layer = ql.QLoRADecoderLayer(cfg, params, dev)
+    del params
+    g = torch.Generator(device=dev).manual_seed(3)
+    x = torch.randn(4, 2048, cfg.d, generator=g, device=dev).to(torch.bfloat16)
+    gout = torch.randn(4, 2048, cfg.d, generator=g, device=dev).to(torch.bfloat16)
+
+    def step():
+        for _, A, B in layer.adapters():
+            A.grad = None
+            B.grad = None
+        xd = x.detach().requires_grad_(True)
+        out = layer(xd)
+        (out.float() * gout.float()).sum().backward()
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    steps = 10
+    ms = timed(step, steps, barrier) / steps
+    q.profile_enable(True)
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    lib_ms, _ = q.profile_read(q.PROF_ALL)
+    q.profile_enable(False)
+    lib_ms /= 5
+    flops = cfg.linear_flops_fwd_bwd(4 * 2048)
+    tf = flops / (lib_ms * 1e-3) / 1e12
+    out = {"ms_per_step": round(ms, 3), "linear_ms_per_step": round(lib_ms, 3),
+           "linear_tflops": round(tf, 1), "linear_frac_of_bf16_peak": round(tf / pk["bf16_sus"], 4),
+           "linear_flops_per_step": flops, "step_tflops_counting_linears": round(flops / (ms * 1e-3) / 1e12, 1),
+           "workload": "llama7b_decoder_layer_b4_s2048_d4096_h32_ffn11008_r64_fwd_bwd_7_nf4_lora_linears"}
+    del layer, x, gout
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_65b(q, dev, pk, barrier):

@@ -23,6 +23,8 @@ Module map:
   nf4.py     codebook, blockwise absmax, nearest-code encode, double
              quantization, packing, dequantization (fp32 step semantics).
   linear.py  fp64 LoRA linear forward / backward on the dequantized weight.
+  layer.py   fp64 LLaMA-shaped decoder layer around seven such linears
+             (torch CPU fp64 with autograd), for the decoder-layer tests.
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py`` except
 the quantitative equal-usage property of the codebook levels,
@@ -31,3 +33,4 @@ makes it approximate).
 """
 
 from . import nf4, linear  # noqa: F401
+# layer.py imports torch; it is imported where used (from oracle import layer).
