@@ -10,8 +10,10 @@ Data layout (the same contract the CUDA library implements independently):
   * group  = 256 consecutive blocks (last group may be partial);
   * codes  = ceil(numel/2) bytes, flat element 2j in the LOW nibble of byte j,
              element 2j+1 in the HIGH nibble; an unused final high nibble is 0;
-  * absmax_q    = one uint8 per block;
-  * group_scale = one fp32 per group.
+  * absmax_q    = one uint8 per block (the int8 bit pattern in the signed
+                  double-quantization variant);
+  * group_scale = one fp32 per group;
+  * offset      = the signed variant's tensor-wide mean block constant (fp32).
 
 Precision: all scalar steps are IEEE fp32 round-to-nearest-even (numpy float32
 arithmetic, no fused multiply-add), written ``fl32(.)`` below; bf16(.) is
@@ -19,6 +21,8 @@ fp32 -> bf16 round-to-nearest-even.
 """
 
 from __future__ import annotations
+
+import math
 
 import numpy as np
 import mpmath
@@ -261,18 +265,106 @@ def dequantize_absmax(q: np.ndarray, S: np.ndarray) -> np.ndarray:
     return (q.astype(np.float32) * Sb).astype(np.float32)
 
 
-def quantize_nf4(W: np.ndarray, fmt: str = "nf4"):
+# ---------------------------------------------------------------------------
+# Double quantization, variant with a tensor-wide offset and signed codes
+# ---------------------------------------------------------------------------
+#
+# The pages say only that the block constants are stored in 8 bits under a
+# coarser set of constants ([Blog-nf4], [QLoRA-abs] (b), [Cap-nf4] "nested
+# quantization").  The variant below is a second reading of that sentence:
+# the block constants of a tensor are all positive and cluster around their
+# mean, so the mean is taken out first and the 8-bit code only carries the
+# signed deviation from it.  Every step is fixed so that the result does not
+# depend on any summation order:
+#
+#   mu   = fl32( fl64( fl64(sum_b a_b) / n_blocks ) )   sum_b a_b exact
+#   c_b  = fl32(a_b - mu)
+#   S_g  = fl32( max_{b in g} |c_b| / 127 )
+#   q_b  = clamp(round_half_even(fl32(c_b / S_g)), -127, 127)   (0 if S_g == 0)
+#   a'_b = fl32( fl32(q_b * S_g) + mu )
+#
+# fl64(.) is round-to-nearest-even to binary64.  The codes are stored as the
+# int8 bit patterns of q_b; -128 is never produced.
+
+F32_MIN_EXP = -149          # exponent of the smallest fp32 subnormal
+
+
+def exact_sum_units(a: np.ndarray) -> int:
+    """sum_b a_b exactly, as an integer count of 2^-149 units.
+
+    Every finite fp32 value is an integer multiple of 2^-149, so the sum of
+    non-negative fp32 values is an integer in those units; Python integers hold
+    it without rounding.  a * 2^149 is exact in fp64 (a power-of-two scaling
+    inside fp64's range) and int() of an integral fp64 value is exact."""
+    a64 = np.asarray(a, dtype=np.float32).astype(np.float64).ravel()
+    if np.any(a64 < 0):
+        raise ValueError("block constants are non-negative")
+    scaled = np.ldexp(a64, -F32_MIN_EXP)
+    return sum(int(x) for x in scaled.tolist())
+
+
+def block_constant_mean(a: np.ndarray) -> np.float32:
+    """mu = fl32(fl64(fl64(exact sum) / n)): the tensor-wide mean block constant.
+
+    float() of a Python int rounds to nearest-even; ldexp by -149 is exact
+    (the sum of fp32 values is far inside fp64's normal range); the fp64
+    division is IEEE round-to-nearest-even; np.float32() rounds once more."""
+    n = int(np.asarray(a).size)
+    if n == 0:
+        return np.float32(0.0)
+    s64 = math.ldexp(float(exact_sum_units(a)), F32_MIN_EXP)
+    return np.float32(s64 / float(n))
+
+
+def double_quantize_signed(absmax: np.ndarray):
+    """Signed 8-bit block constants around the tensor-wide mean (see above).
+
+    Returns (q uint8 [nblocks] holding int8 bit patterns, S float32 [ngroups],
+    mu float32)."""
+    a = np.asarray(absmax, dtype=np.float32).ravel()
+    nb = a.size
+    ng = -(-nb // GROUP)
+    mu = block_constant_mean(a)
+    c = (a - mu).astype(np.float32)                         # fl32(a_b - mu)
+    pad = ng * GROUP - nb
+    cp = np.concatenate([c, np.zeros(pad, np.float32)]) if pad else c
+    m = np.abs(cp).reshape(ng, GROUP).max(axis=1).astype(np.float32)
+    S = (m / np.float32(127.0)).astype(np.float32)
+    Sb = np.repeat(S, GROUP)[:nb]
+    q = np.zeros(nb, dtype=np.int8)
+    nz = Sb != 0
+    ratio = (c[nz] / Sb[nz]).astype(np.float32)            # fl32(c_b / S_g)
+    q[nz] = np.clip(np.rint(ratio), -127.0, 127.0).astype(np.int8)
+    return q.view(np.uint8), S, mu
+
+
+def dequantize_absmax_signed(q: np.ndarray, S: np.ndarray, mu) -> np.ndarray:
+    """a'_b = fl32(fl32(q_b * S_g) + mu), q_b the int8 value of the stored byte."""
+    qi = np.asarray(q, dtype=np.uint8).ravel().view(np.int8)
+    Sb = np.repeat(np.asarray(S, np.float32), GROUP)[: qi.size]
+    return ((qi.astype(np.float32) * Sb).astype(np.float32) + np.float32(mu)).astype(np.float32)
+
+
+DQ_VARIANTS = ("plain", "signed")
+
+
+def quantize_nf4(W: np.ndarray, fmt: str = "nf4", dq: str = "plain"):
     """Quantize fp32 weights once, up front ([Blog-mem]: the base never changes,
     so it is quantized once).
 
     Steps in the pages' order: block absmax -> normalise -> nearest NF4 level
     -> pack 4-bit codes -> double-quantize the block constants.  The codes use
     the exact fp32 block absmax (the constants are quantized afterwards, as a
-    separate second level).  Raises ValueError on non-finite input.
+    separate second level).  dq picks the reading of the second level:
+    "plain" (double_quantize) or "signed" (double_quantize_signed).  Raises
+    ValueError on non-finite input.
 
     Returns dict(codes=uint8[ceil(numel/2)], absmax_q=uint8[nblocks],
-    group_scale=float32[ngroups], shape=W.shape).
+    group_scale=float32[ngroups], offset=float32 (mu; 0 for "plain"),
+    shape=W.shape, format=fmt, dq=dq).
     """
+    if dq not in DQ_VARIANTS:
+        raise ValueError(f"unknown double-quantization variant {dq!r}")
     W = np.asarray(W, dtype=np.float32)
     if not np.all(np.isfinite(W)):
         raise ValueError("non-finite weight")
@@ -280,14 +372,19 @@ def quantize_nf4(W: np.ndarray, fmt: str = "nf4"):
     a = block_absmax(flat)
     n = normalize(flat, a)
     codes = nearest_code(n, codebook(fmt)) if n.size <= (1 << 24) else nearest_code_fast(n, codebook(fmt))
-    q, S = double_quantize(a)
-    return {"codes": pack_nibbles(codes), "absmax_q": q, "group_scale": S,
-            "shape": tuple(W.shape), "format": fmt}
+    if dq == "plain":
+        q, S = double_quantize(a)
+        mu = np.float32(0.0)
+    else:
+        q, S, mu = double_quantize_signed(a)
+    return {"codes": pack_nibbles(codes), "absmax_q": q, "group_scale": S, "offset": mu,
+            "shape": tuple(W.shape), "format": fmt, "dq": dq}
 
 
 def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np.ndarray,
-                        shape, fmt: str = "nf4") -> np.ndarray:
-    """W' = bf16(fl32(v_code * a'_b)) with a'_b = fl32(q_b * S_g); bf16 bit patterns.
+                        shape, fmt: str = "nf4", dq: str = "plain", offset=0.0) -> np.ndarray:
+    """W' = bf16(fl32(v_code * a'_b)); bf16 bit patterns.  a'_b = fl32(q_b * S_g)
+    for the plain constants, fl32(fl32(q_b * S_g) + mu) for the signed ones.
 
     [Blog-mem]: every forward and backward pass expands the 4-bit base back
     to a 16-bit type as it runs.  Reading: the 16-bit type is bf16, the product
@@ -296,21 +393,26 @@ def dequantize_nf4_bits(codes: np.ndarray, absmax_q: np.ndarray, group_scale: np
     numel = int(np.prod(shape))
     c = unpack_nibbles(codes, numel)
     v = codebook(fmt)[c]
-    ap = np.repeat(dequantize_absmax(absmax_q, group_scale), BLOCK)[:numel]
+    if dq == "plain":
+        a_deq = dequantize_absmax(absmax_q, group_scale)
+    else:
+        a_deq = dequantize_absmax_signed(absmax_q, group_scale, offset)
+    ap = np.repeat(a_deq, BLOCK)[:numel]
     w32 = (v * ap).astype(np.float32)
     return bf16_rne_bits(w32).reshape(shape)
 
 
 def dequantize_nf4(q: dict) -> np.ndarray:
     """Convenience: dequantize a quantize_nf4() result to bf16 bit patterns."""
-    return dequantize_nf4_bits(q["codes"], q["absmax_q"], q["group_scale"], q["shape"], q.get("format", "nf4"))
+    return dequantize_nf4_bits(q["codes"], q["absmax_q"], q["group_scale"], q["shape"], q.get("format", "nf4"),
+                               q.get("dq", "plain"), q.get("offset", 0.0))
 
 
-def reconstruction_error(W: np.ndarray, fmt: str = "nf4") -> float:
+def reconstruction_error(W: np.ndarray, fmt: str = "nf4", dq: str = "plain") -> float:
     """Relative Frobenius error ||bf16 dequant(quant(W)) - W|| / ||W|| of a 4-bit
     table on the given weights: the proxy, on Gaussian weights, for the pages'
     statement that NF4 beats plain 4-bit float and integer types ([Blog-nf4])."""
     W = np.asarray(W, dtype=np.float32)
-    Wd = bf16_bits_to_f32(dequantize_nf4(quantize_nf4(W, fmt))).astype(np.float64)
+    Wd = bf16_bits_to_f32(dequantize_nf4(quantize_nf4(W, fmt, dq))).astype(np.float64)
     W64 = W.astype(np.float64)
     return float(np.linalg.norm(Wd - W64) / np.linalg.norm(W64))
