@@ -68,8 +68,17 @@ def traffic_record(kernel: str):
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons sampled every 5 ms from a background thread
+    through NVML (read-only queries), so a timed region of a few tens of ms still
+    gets samples; start() returns once the first sample is in.  Falls back to
+    nvidia-smi polling when NVML is unavailable."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
     def __init__(self, dev: int):
         self.proc = None
+        self.thread = None
         self.samples = []
         try:
             uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -77,7 +86,32 @@ class ClockSampler:
         except Exception:
             self.sel = None
 
+    def _nvml_loop(self, nv, h, first):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM), int(get_reasons(h))))
+            except Exception:
+                pass
+            first.set()
+            self.stop_flag.wait(0.005)
+
     def start(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self.sel) if self.sel else nv.nvmlDeviceGetHandleByIndex(0)
+            self.stop_flag = threading.Event()
+            first = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, first), daemon=True)
+            self.thread.start()
+            first.wait(2.0)
+            return
+        except Exception:
+            self.thread = None
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -90,6 +124,15 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(2.0)
+            rows = self.samples
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+            reasons = sorted({name for _, _, bits in rows for name, bit in self.REASONS if bits & bit})
+            return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                    "reasons": reasons, "samples": len(rows), "source": "nvml, 5 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         self.proc.terminate()
@@ -104,19 +147,19 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi, 100 ms"}
 
 
 # --------------------------------------------------------------------------- our arm
 class Replica:
     """Device-resident inputs, outputs and workspaces of the three projections."""
 
-    def __init__(self, q, dev, cases=qi.LLAMA7B):
+    def __init__(self, q, dev, cases=qi.LLAMA7B, dq=0):
         self.q = q
         self.cases = []
         for case in cases:
             d = qi.make_linear(case)
-            w = q.quantize_nf4(d["W"].to(dev))
+            w = q.quantize_nf4(d["W"].to(dev), dq=dq)
             M, N, K, r = case.M, case.N, case.K, case.r
             c = {"case": case, "w": w, "s": case.s,
                  "X": d["X"].to(dev), "A": d["A"].to(dev), "B": d["B"].to(dev), "dY": d["dY"].to(dev),
@@ -208,6 +251,7 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     extras = measure_extras(q, rep, dev, pk, barrier)
     extras["llama65b"] = measure_65b(q, dev, pk, barrier)
     extras["decoder_layer"] = measure_layer(q, dev, pk, barrier)
+    extras["dq_signed"] = measure_dq_signed(q, dev, pk, barrier)
     e2e = measure_e2e(q, rep, dev, min(args.steps, 20), barrier, allmax, world)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -288,39 +332,85 @@ def measure_65b(q, dev, pk, barrier):
     return out
 
 
-def measure_extras(q, rep, dev, pk, barrier):
-    """Standalone dequantizer, quantizer and few-token forward, each in GB/s."""
-    out = {}
-    # dequantizer: 0.5 + 1/64 + 4/16384 B in, 2 B out per weight
-    bufs = [torch.empty((c["case"].N, c["case"].K), dtype=torch.bfloat16, device=dev) for c in rep.cases]
-    nw = sum(c["case"].N * c["case"].K for c in rep.cases)
-    dq_bytes = sum(c["w"].nbytes() for c in rep.cases) + 2 * nw
+def dequant_gbs(q, cases, dev, pk, barrier):
+    """Standalone dequantizer over the cases' weights: 0.5 + 1/64 + 4/16384 B in, 2 B out per weight."""
+    bufs = [torch.empty((c["case"].N, c["case"].K), dtype=torch.bfloat16, device=dev) for c in cases]
+    nw = sum(c["case"].N * c["case"].K for c in cases)
+    dq_bytes = sum(c["w"].nbytes() for c in cases) + 2 * nw
 
     def dq():
-        for c, b in zip(rep.cases, bufs):
+        for c, b in zip(cases, bufs):
             q.dequantize(c["w"], out=b)
     for _ in range(3):
         dq()
     reps = 20
     ms = timed(dq, reps, barrier) / reps
     gbs = dq_bytes / (ms * 1e-3) / 1e9
-    out["dequant"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4),
-                      "peak": pk["hbm"], "bytes_per_weight": round(dq_bytes / nw, 4)}
-    del bufs
-    # quantizer: 4 B in, 0.516 B out per weight (re-quantizes fresh fp32 copies)
-    Ws = [torch.randn((c["case"].N, c["case"].K), device=dev, dtype=torch.float32) * 0.02 for c in rep.cases]
-    tmp = [q.NF4Weight.empty(c["case"].N, c["case"].K, dev) for c in rep.cases]
+    return {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4),
+            "peak": pk["hbm"], "bytes_per_weight": round(dq_bytes / nw, 4)}
+
+
+def quantize_gbs(q, cases, dev, pk, barrier, dq=0):
+    """Quantizer over fresh fp32 copies of the cases' shapes: 4 B in, 0.516 B out per weight
+    (the signed reading's workspace round trip of 4 B per block is not counted)."""
+    nw = sum(c["case"].N * c["case"].K for c in cases)
+    Ws = [torch.randn((c["case"].N, c["case"].K), device=dev, dtype=torch.float32) * 0.02 for c in cases]
+    tmp = [q.NF4Weight.empty(c["case"].N, c["case"].K, dev, dq=dq) for c in cases]
+    wss = [torch.empty(max(16, q.load().qlora_quantize_workspace_bytes(c["case"].N, c["case"].K, dq)),
+                       dtype=torch.uint8, device=dev) for c in cases]
 
     def qz():
-        for W, t in zip(Ws, tmp):
-            q.quantize_nf4(W, out=t)
+        for W, t, ws in zip(Ws, tmp, wss):
+            q.quantize_nf4(W, out=t, workspace=ws)
     for _ in range(3):
         qz()
     ms = timed(qz, 10, barrier) / 10
     qb = 4 * nw + sum(t.nbytes() for t in tmp)
     gbs = qb / (ms * 1e-3) / 1e9
-    out["quantize"] = {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4)}
-    del Ws, tmp
+    del Ws, tmp, wss
+    return {"value": round(gbs, 1), "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4)}
+
+
+def measure_dq_signed(q, dev, pk, barrier):
+    """The signed reading of the block constants (int8 codes around the tensor-wide mean mu): one
+    fwd + bwd step of the LLaMA-7B projections, the dequantizer and the quantizer with such weights,
+    and the error of the constants and of the weight against the plain reading."""
+    rep = Replica(q, dev, qi.LLAMA7B, dq=q.DQ_SIGNED)
+    for _ in range(3):
+        rep.step()
+    torch.cuda.synchronize()
+    steps = 10
+    ms = timed(rep.step, steps, barrier) / steps
+    tf = rep.flops() / (ms * 1e-3) / 1e12
+    out = {"step": {"value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+                    "frac_of_bf16_peak": round(tf / pk["bf16_sus"], 4)},
+           "dequant": dequant_gbs(q, rep.cases, dev, pk, barrier),
+           "quantize": quantize_gbs(q, rep.cases, dev, pk, barrier, dq=q.DQ_SIGNED)}
+    Wq = qi.make_weight(4096, 4096, qi.LLAMA7B[0].seed).to(dev)
+    a = Wq.reshape(-1, 64).abs().amax(dim=1).double()
+    for name, dq in (("plain", q.DQ_PLAIN), ("signed", q.DQ_SIGNED)):
+        wq = q.quantize_nf4(Wq, dq=dq)
+        d = q.dequantize(wq).double() - Wq.double()
+        # a' of every block from the stored bytes (fp32 products and sums, as the kernels form them)
+        S = wq.scales.repeat_interleave(256)[:a.numel()]
+        if dq == q.DQ_SIGNED:
+            ap = (wq.absmax_q.view(torch.int8).float() * S) + wq.offset
+        else:
+            ap = wq.absmax_q.float() * S
+        out[name] = {"weight_rel_frobenius_error": round(float(d.norm() / Wq.double().norm()), 6),
+                     "block_constant_mean_abs_rel_error": round(float(((ap.double() - a).abs() / a).mean()), 6)}
+        del wq, d
+    out["note"] = "errors on the 4096x4096 Gaussian q-projection weight"
+    out["workload"] = "llama7b_projections_m4096_r64_fwd_bwd_signed_block_constants"
+    del rep, Wq
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_extras(q, rep, dev, pk, barrier):
+    """Standalone dequantizer, quantizer and few-token forward, each in GB/s."""
+    out = {"dequant": dequant_gbs(q, rep.cases, dev, pk, barrier),
+           "quantize": quantize_gbs(q, rep.cases, dev, pk, barrier)}
     # few-token forward: weights rotated over enough copies to exceed L2
     res = {}
     for M in qi.GEMV_TOKENS:

@@ -32,12 +32,17 @@ EXPORTS = (
     "qlora_codes_bytes", "qlora_absmax_bytes", "qlora_group_scale_bytes", "qlora_quantize_nf4", "qlora_dequantize",
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
     "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
-    "qlora_profile_read", "qlora_linear_fwd_noalloc", "qlora_format_codebook",
+    "qlora_profile_read", "qlora_linear_fwd_noalloc", "qlora_format_codebook", "qlora_group_scale_bytes_dq",
+    "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_ws",
 )
 
 # 4-bit code tables (QLORA_FORMAT_*): NF4 is the method's type; FP4 (e2m1) and
 # INT4 are the plain float and integer types it is compared against.
 FORMAT_NF4, FORMAT_FP4, FORMAT_INT4 = 0, 1, 2
+
+# Readings of the 8-bit block constants (QLORA_DQ_*): unsigned with no offset,
+# or signed around the tensor-wide mean constant (stored after the group scales).
+DQ_PLAIN, DQ_SIGNED = 0, 1
 
 # Kernel kinds of the timing hook (qlora_profile_read).
 PROF_ALL, PROF_GEMM_FWD, PROF_GEMM_DGRAD, PROF_LORA, PROF_QUANT, PROF_DEQUANT, PROF_GEMV = range(7)
@@ -52,7 +57,7 @@ class QloraError(RuntimeError):
 class Nf4WeightC(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p),
                 ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p), ("format", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("dq", ctypes.c_int32)]
 
 
 _lib = None
@@ -86,6 +91,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_profile_enable": (None, [i32]),
         "qlora_profile_read": (i32, [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
         "qlora_linear_fwd_noalloc": (i32, [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp]),
+        "qlora_group_scale_bytes_dq": (sz, [i64, i64, i32]),
+        "qlora_quantize_workspace_bytes": (sz, [i64, i64, i32]),
+        "qlora_quantize_nf4_ws": (i32, [vp, wp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -114,22 +122,35 @@ class NF4Weight:
     rows: int
     cols: int
     codes: torch.Tensor        # uint8 [ceil(rows*cols/2)]
-    absmax_q: torch.Tensor     # uint8 [ceil(rows*cols/64)]
-    group_scale: torch.Tensor  # float32 [ceil(rows*cols/16384)]
+    absmax_q: torch.Tensor     # uint8 [ceil(rows*cols/64)] (int8 bit patterns for DQ_SIGNED)
+    group_scale: torch.Tensor  # float32 [ceil(rows*cols/16384)] (+ mu last for DQ_SIGNED)
     format: int = FORMAT_NF4   # code table (FORMAT_*)
+    dq: int = DQ_PLAIN         # reading of the block constants (DQ_*)
 
     def c_struct(self) -> Nf4WeightC:
         return Nf4WeightC(self.rows, self.cols, self.codes.data_ptr(), self.absmax_q.data_ptr(),
-                          self.group_scale.data_ptr(), self.format, 0)
+                          self.group_scale.data_ptr(), self.format, self.dq)
 
     @staticmethod
-    def empty(rows: int, cols: int, device="cuda", format: int = FORMAT_NF4) -> "NF4Weight":
+    def empty(rows: int, cols: int, device="cuda", format: int = FORMAT_NF4, dq: int = DQ_PLAIN) -> "NF4Weight":
         lib = load()
+        gs = lib.qlora_group_scale_bytes_dq(rows, cols, dq)
+        if gs == 0:
+            raise QloraError(1, "NF4Weight.empty")
         return NF4Weight(rows, cols,
                          torch.empty(lib.qlora_codes_bytes(rows, cols), dtype=torch.uint8, device=device),
                          torch.empty(lib.qlora_absmax_bytes(rows, cols), dtype=torch.uint8, device=device),
-                         torch.empty(lib.qlora_group_scale_bytes(rows, cols) // 4, dtype=torch.float32,
-                                     device=device), format)
+                         torch.empty(gs // 4, dtype=torch.float32, device=device), format, dq)
+
+    @property
+    def scales(self) -> torch.Tensor:
+        """The per-group scales S_g (without the offset)."""
+        return self.group_scale[:-1] if self.dq == DQ_SIGNED else self.group_scale
+
+    @property
+    def offset(self) -> torch.Tensor | None:
+        """mu, the offset of DQ_SIGNED block constants (a 1-element view), else None."""
+        return self.group_scale[-1:] if self.dq == DQ_SIGNED else None
 
     def nbytes(self) -> int:
         return self.codes.numel() + self.absmax_q.numel() + 4 * self.group_scale.numel()
@@ -173,15 +194,24 @@ def profile_read(kind: int):
     return ms.value, n.value
 
 
-def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, format: int = FORMAT_NF4) -> NF4Weight:
+def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, format: int = FORMAT_NF4,
+                 dq: int = DQ_PLAIN, workspace: torch.Tensor | None = None) -> NF4Weight:
     """Quantize a contiguous fp32 CUDA tensor [rows, cols] (flat row-major) to a
-    4-bit table (NF4 unless `format` says otherwise, or `out.format` when given)."""
+    4-bit table (NF4 unless `format` says otherwise) with block constants as
+    `dq` reads them (`out.format` / `out.dq` when `out` is given).  DQ_SIGNED
+    uses a workspace of qlora_quantize_workspace_bytes (allocated here when not
+    given)."""
     lib = load()
     assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
     rows, cols = (W.shape[0], W[0].numel()) if W.dim() >= 2 else (1, W.numel())
-    w = out if out is not None else NF4Weight.empty(rows, cols, W.device, format)
+    w = out if out is not None else NF4Weight.empty(rows, cols, W.device, format, dq)
     s = w.c_struct()
-    _check(lib.qlora_quantize_nf4(_ptr(W), ctypes.byref(s), _stream()), "qlora_quantize_nf4")
+    need = int(lib.qlora_quantize_workspace_bytes(rows, cols, w.dq))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qlora_quantize_nf4_ws(_ptr(W), ctypes.byref(s), _ptr(workspace), nbytes, _stream()),
+           "qlora_quantize_nf4_ws")
     return w
 
 

@@ -107,6 +107,16 @@ const Nf4Table &format_table(int format) {
 
 const Nf4Table &nf4_table() { return format_table(QLORA_FORMAT_NF4); }
 
+Nf4Table weight_table(const qlora_nf4_weight *w) {
+  Nf4Table t = format_table(w->format);
+  if (w->dq == QLORA_DQ_SIGNED) {
+    const int64_t nb = ceil_div(w->rows * w->cols, kBlock);
+    t.qx = 128u;
+    t.offset = w->group_scale + ceil_div(nb, kGroup);
+  }
+  return t;
+}
+
 uint64_t wait_limit() { return g_wait_limit.load(); }
 
 // ----------------------------------------------------------------- device status word
@@ -257,7 +267,8 @@ T *at(void *ws, size_t off) {
 qlora_status check_weight(const qlora_nf4_weight *w) {
   if (!w || !w->codes || !w->absmax_q || !w->group_scale) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < 1) return QLORA_ERR_INVALID_ARG;
-  if (w->format < QLORA_FORMAT_NF4 || w->format > QLORA_FORMAT_INT4 || w->reserved != 0) return QLORA_ERR_INVALID_ARG;
+  if (w->format < QLORA_FORMAT_NF4 || w->format > QLORA_FORMAT_INT4) return QLORA_ERR_INVALID_ARG;
+  if (w->dq != QLORA_DQ_PLAIN && w->dq != QLORA_DQ_SIGNED) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale)) return QLORA_ERR_MISALIGNED;
   return QLORA_OK;
 }
@@ -327,6 +338,15 @@ size_t qlora_absmax_bytes(int64_t rows, int64_t cols) {
 size_t qlora_group_scale_bytes(int64_t rows, int64_t cols) {
   const int64_t nb = (rows * cols + kBlock - 1) / kBlock;
   return rows < 1 || cols < 1 ? 0 : static_cast<size_t>((nb + kGroup - 1) / kGroup) * 4;
+}
+size_t qlora_group_scale_bytes_dq(int64_t rows, int64_t cols, int dq) {
+  if (dq != QLORA_DQ_PLAIN && dq != QLORA_DQ_SIGNED) return 0;
+  const size_t b = qlora_group_scale_bytes(rows, cols);
+  return b == 0 ? 0 : b + (dq == QLORA_DQ_SIGNED ? 4 : 0);
+}
+size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols, int dq) {
+  if (rows < 1 || cols < 1 || dq != QLORA_DQ_SIGNED) return 0;
+  return quantize_workspace_bytes(rows * cols);
 }
 
 const char *qlora_status_string(qlora_status st) {
@@ -412,22 +432,33 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
   return make_plan(op, M, N, K, r).total;
 }
 
-qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream) {
+qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
+                                   void *stream) {
   if (!W) return QLORA_ERR_INVALID_ARG;
   QL_TRY(check_weight(out));
   if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  const int64_t numel = out->rows * out->cols;
+  if (out->dq == QLORA_DQ_SIGNED) {
+    if (numel >= (int64_t(1) << 38)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    if (!ws || ws_bytes < quantize_workspace_bytes(numel)) return QLORA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  }
   int *status = device_status_ptr();
   if (!status) return QLORA_ERR_CUDA;
-  QL_CUDA(launch_quantize(W, out->rows * out->cols, out->codes, out->absmax_q, out->group_scale, out->format,
-                          status, static_cast<cudaStream_t>(stream)));
+  QL_CUDA(launch_quantize(W, numel, out->codes, out->absmax_q, out->group_scale, weight_table(out),
+                          out->dq == QLORA_DQ_SIGNED ? ws : nullptr, status, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream) {
+  return qlora_quantize_nf4_ws(W, out, nullptr, 0, stream);
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream) {
   if (!W_out) return QLORA_ERR_INVALID_ARG;
   QL_TRY(check_weight(w));
   if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
-  QL_CUDA(launch_dequantize(w->codes, w->absmax_q, w->group_scale, w->rows * w->cols, w->format,
+  QL_CUDA(launch_dequantize(w->codes, w->absmax_q, w->group_scale, w->rows * w->cols, weight_table(w),
                             W_out, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
 }
@@ -445,11 +476,12 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int6
   float *H = H_out ? H_out : at<float>(ws, p.H);
   if (p.gemv) {
     GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<void>(ws, p.part),
-               w->format};
+               weight_table(w)};
     return launch_gemv(g, st);
   }
   QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
-  QGemmArgs g{false, M, N, K, X, w->codes, w->absmax_q, w->group_scale, at<uint16_t>(ws, p.sH), B, r, Y, w->format};
+  QGemmArgs g{false, M, N, K, X, w->codes, w->absmax_q, w->group_scale, at<uint16_t>(ws, p.sH), B, r, Y,
+              weight_table(w)};
   return launch_qgemm(g, st);
 }
 
@@ -529,7 +561,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
     }
   }
   // dX = dY W' + Gb A
-  QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX, w->format};
+  QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX, weight_table(w)};
   return launch_qgemm(g, st);
 }
 

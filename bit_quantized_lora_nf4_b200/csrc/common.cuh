@@ -17,11 +17,27 @@ namespace qlora {
 constexpr int kBlock = 64;     // weights per absmax block
 constexpr int kGroup = 256;    // blocks per double-quantization group
 
-// Values every kernel that touches NF4 needs, passed by value (constant bank).
+// Values every kernel that touches NF4 needs, passed by value (constant bank):
+// the 16-entry code table and the reading of the 8-bit block constants.
 struct Nf4Table {
   float level[16];       // ascending NF4 levels (fp32)
   float thresh[15];      // thresh[i] = midpoint(level[i], level[i+1]) rounded toward -inf
+  uint32_t qx;           // 0: unsigned block constants; 128: signed (int8) ones around an offset
+  const float *offset;   // signed constants: device address of the offset mu; nullptr otherwise
 };
+
+// The offset mu every block constant is stored relative to (+0 for unsigned
+// constants).  One load per thread, at kernel start.
+__device__ __forceinline__ float dq_offset(const Nf4Table &t) { return t.offset ? __ldg(t.offset) : 0.0f; }
+
+// Dequantized block constant a' from its stored byte q and group scale S:
+// fl32(fl32(v * S) + mu), v = q (unsigned) or the int8 value of q (signed,
+// qx = 128: (q ^ 128) - 128).  For unsigned constants mu = +0 and v * S >= +0,
+// so the sum is exact and a' = fl32(q * S) bit for bit.
+__device__ __forceinline__ float block_constant(uint32_t q, float S, uint32_t qx, float mu) {
+  const int v = static_cast<int>(q ^ qx) - static_cast<int>(qx);
+  return __fadd_rn(__fmul_rn(static_cast<float>(v), S), mu);
+}
 
 // ------------------------------------------------------------------ status word
 __device__ __forceinline__ void latch_status(int *status, int code) {

@@ -153,9 +153,14 @@ struct GemvParams {
 
 // Quantized constants of one position for rows n0 = 16 t + g and n0 + 8, block 4 step + c.
 struct PosConst {
-  uint32_t q0, q1;   // 8-bit block constants
-  float S0, S1;      // 32-bit group constants (0 for rows past N / blocks past K)
+  uint32_t q0, q1;   // 8-bit block constants; bit 8 set for rows past N / blocks past K
+  float S0, S1;      // 32-bit group constants
 };
+
+// a' of one position's block, and 0 for the padding positions (bit 8 of q set).
+__device__ __forceinline__ float pos_constant(uint32_t q, float S, uint32_t qx, float mu) {
+  return (q & 0x100u) ? 0.0f : block_constant(q, S, qx, mu);
+}
 
 // Where a thread reads its activation fragments: token rows past M read the
 // last live token (those output columns are never stored), blocks past K read
@@ -315,21 +320,20 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
   int g0 = range_owner(first_tile * S, p.U, p.G);   // first warp on the current tile
 
   // Block constants one position ahead in registers.  Rows past N and blocks
-  // past K read a clamped, valid address and get a zero group constant, so
+  // past K read a clamped, valid address and are marked in bit 8 of q, so
   // their weights decode to (signed) zero.
+  const float mu = dq_offset(p.tab);
   int ft = first_tile, fs = a - first_tile * S, fu = a;
   auto fetch = [&](PosConst &f) {
     const int kb = 4 * fs + c;
     const int kbc = min(kb, KB - 1);
     const int n0 = ft * 16 + g;
     const int bi0 = min(n0, N - 1) * KB + kbc, bi1 = min(n0 + 8, N - 1) * KB + kbc;   // < 2^31 (host check)
-    f.q0 = ldg_once_u8(p.absmax_q + bi0);
-    f.q1 = ldg_once_u8(p.absmax_q + bi1);
-    const float S0 = ldg_once_f32(p.group_scale + (bi0 >> 8));
-    const float S1 = ldg_once_f32(p.group_scale + (bi1 >> 8));
     const bool kv = kb < KB;
-    f.S0 = (kv && n0 < N) ? S0 : 0.0f;
-    f.S1 = (kv && n0 + 8 < N) ? S1 : 0.0f;
+    f.q0 = ldg_once_u8(p.absmax_q + bi0) | ((kv && n0 < N) ? 0u : 0x100u);
+    f.q1 = ldg_once_u8(p.absmax_q + bi1) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
+    f.S0 = ldg_once_f32(p.group_scale + (bi0 >> 8));
+    f.S1 = ldg_once_f32(p.group_scale + (bi1 >> 8));
     if (fu + 1 < b) {   // advance, staying on the last position of the range
       ++fu;
       if (++fs == S) {
@@ -359,8 +363,8 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
     for (int tt = 0; tt < NT; ++tt) xv[0][tt] = x.load(tt, kbc, 0);
 
     uint32_t LO[2][4], HI[2][4];
-    nf4_block_table(__fmul_rn(static_cast<float>(f.q0), f.S0), p.tab, LO[0], HI[0]);
-    nf4_block_table(__fmul_rn(static_cast<float>(f.q1), f.S1), p.tab, LO[1], HI[1]);
+    nf4_block_table(pos_constant(f.q0, f.S0, p.tab.qx, mu), p.tab, LO[0], HI[0]);
+    nf4_block_table(pos_constant(f.q1, f.S1, p.tab.qx, mu), p.tab, LO[1], HI[1]);
 
     // codes of rows g and g + 8, 32 bytes each at column 32 c: 16-byte chunks 2c
     // and 2c+1, stored at chunk ^ (row & 7) by the 128-byte swizzle
@@ -680,7 +684,7 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
                reinterpret_cast<float *>(ws + L.off_pieces), reinterpret_cast<float *>(ws + L.off_hpart),
                static_cast<int>(a.M), a.r, L.r16, L.JT, L.HS, static_cast<int>(G), static_cast<int>(L.S),
                static_cast<int>(L.U), static_cast<int>(L.T), L.P, xs ? xs_row_bytes(KB) : 0, a.wN, a.wK, status,
-               wait_limit(), format_table(a.format)};
+               wait_limit(), a.tab};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(GV_THREADS);

@@ -14,6 +14,10 @@ namespace qlora {
 const Nf4Table &nf4_table();
 // The table of a QLORA_FORMAT_* (the NF4 one for QLORA_FORMAT_NF4); format must be valid.
 const Nf4Table &format_table(int format);
+// The decode description of a validated weight: its format's table plus the
+// reading of its block constants (signed ones point `offset` at mu, stored
+// after the group scales).
+Nf4Table weight_table(const qlora_nf4_weight *w);
 
 // Address of the device status word on the current device (nullptr on error).
 int *device_status_ptr();
@@ -37,10 +41,13 @@ bool make_tmap_2d(CUtensorMap *tm, const void *base, CUtensorMapDataType dtype, 
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 // ---- kernels (launchers return the launch error) -------------------------------
+// Quantizer.  tab.qx != 0 selects signed block constants; those need `ws`
+// (quantize_workspace_bytes(numel) bytes) and write mu to tab.offset.
+size_t quantize_workspace_bytes(int64_t numel);
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
-                            int format, int *status, cudaStream_t st);
+                            const Nf4Table &tab, void *ws, int *status, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
-                              int64_t numel, int format, uint16_t *out, cudaStream_t st);
+                              int64_t numel, const Nf4Table &tab, uint16_t *out, cudaStream_t st);
 
 // Fused dequant-GEMM on tensor cores.
 //   forward: out[M, wN] = act[M, wK] . W'^T + lora_act[M, r] . lora_w[wN, r]^T
@@ -57,7 +64,7 @@ struct QGemmArgs {
   const uint16_t *lora_w;
   int r;
   uint16_t *out;
-  int format;          // QLORA_FORMAT_* of the weight
+  Nf4Table tab;        // weight_table() of the weight
 };
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
 // The same product on a CTA pair (256-row tiles); launch_qgemm dispatches to it for M > 128.
@@ -77,7 +84,7 @@ struct GemvArgs {
   uint16_t *Y;
   float *H_out;        // optional [M, r]
   void *workspace;     // gemv_workspace_bytes(M, N, K, r) bytes, 256-byte aligned
-  int format;          // QLORA_FORMAT_* of the weight
+  Nf4Table tab;        // weight_table() of the weight
 };
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st);

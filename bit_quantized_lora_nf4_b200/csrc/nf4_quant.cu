@@ -13,9 +13,20 @@
 //   a_b = max |w| over the 64-element block (exact)
 //   n   = fl32(w / a_b)            (0 when a_b == 0)
 //   code = #{ i : n > thresh[i] }  == nearest level, ties to the lower index
-//   c_g = max a_b over 256 blocks;  S_g = fl32(c_g / 255)
-//   q_b = min(255, rint(fl32(a_b / S_g)))  (0 when S_g == 0)
-//   W'  = bf16(fl32(level[code] * fl32(q_b * S_g)))
+//   plain block constants (QLORA_DQ_PLAIN):
+//     c_g = max a_b over 256 blocks;  S_g = fl32(c_g / 255)
+//     q_b = min(255, rint(fl32(a_b / S_g)))  (0 when S_g == 0);  a'_b = fl32(q_b * S_g)
+//   signed block constants around their mean (QLORA_DQ_SIGNED):
+//     mu  = fl32(fl64(fl64(exact sum of all a_b) / n_blocks))
+//     c_b = fl32(a_b - mu);  S_g = fl32(max |c_b| / 127)
+//     q_b = clamp(rint(fl32(c_b / S_g)), -127, 127)  (0 when S_g == 0), stored as int8
+//     a'_b = fl32(fl32(q_b * S_g) + mu)
+//   W'  = bf16(fl32(level[code] * a'_b))
+//
+// The signed constants take three launches: the quantizer writes the codes,
+// the fp32 a_b and an exact, order-free sum of the a_b (integer digits added
+// with 64-bit atomics); a second kernel turns the sum into mu and codes every
+// group's constants against it.
 #include "decode.cuh"
 #include "internal.h"
 
@@ -42,6 +53,72 @@ __device__ __forceinline__ bool finite4(float4 v) {
   return isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
 }
 
+// ---- exact sum of non-negative fp32 values ------------------------------------
+// Every finite fp32 value is an integer number of 2^-149 units; a value with
+// biased exponent E and significand m (hidden bit included) is m << max(E - 1, 0)
+// units, below 2^278.  The sum of fewer than 2^32 of them is below 2^310 and is
+// kept as kSumDigits base-2^32 digits, each held in a 64-bit word that absorbs
+// unnormalised additions (carries are propagated once, when the sum is read).
+constexpr int kSumDigits = 10;
+
+// Adds this warp's 32 values to the digit words `acc` (shared memory): per
+// digit the 32 contributions are summed as two 16-bit halves with warp
+// reductions, then one lane adds the total.
+__device__ __forceinline__ void warp_exact_add(float a, unsigned long long *acc) {
+  const uint32_t u = __float_as_uint(a);
+  const uint32_t E = u >> 23;
+  const uint32_t m = (u & 0x7FFFFFu) | (E ? 0x800000u : 0u);
+  const uint32_t shift = E ? E - 1 : 0;
+  const uint32_t d = shift >> 5;
+  const unsigned long long x = static_cast<unsigned long long>(m) << (shift & 31);   // < 2^55
+  const uint32_t lo = static_cast<uint32_t>(x), hi = static_cast<uint32_t>(x >> 32);
+  const uint32_t dmin = __reduce_min_sync(0xffffffffu, d);
+  const uint32_t dmax = __reduce_max_sync(0xffffffffu, d) + 1;
+  for (uint32_t k = dmin; k <= dmax; ++k) {
+    const uint32_t c = k == d ? lo : (k == d + 1 ? hi : 0u);
+    const unsigned long long sum = __reduce_add_sync(0xffffffffu, c & 0xFFFFu) +
+                                   (static_cast<unsigned long long>(__reduce_add_sync(0xffffffffu, c >> 16)) << 16);
+    if ((threadIdx.x & 31) == 0 && sum != 0) atomicAdd(acc + k, sum);
+  }
+}
+
+// 2^k as a double, -1022 <= k <= 1023.
+__device__ __forceinline__ double pow2d(int k) { return __longlong_as_double(static_cast<long long>(k + 1023) << 52); }
+
+// fl32(fl64(fl64(S) / n)) for the exact sum S held in the digit words (one thread).
+__device__ float exact_mean(const unsigned long long *acc, int64_t n) {
+  uint32_t dig[kSumDigits + 2];
+  unsigned long long carry = 0;
+  for (int i = 0; i < kSumDigits; ++i) {
+    const unsigned long long v = acc[i] + carry;
+    dig[i] = static_cast<uint32_t>(v);
+    carry = v >> 32;
+  }
+  dig[kSumDigits] = static_cast<uint32_t>(carry);
+  dig[kSumDigits + 1] = 0;
+  int top = kSumDigits;
+  while (top > 0 && dig[top] == 0) --top;
+  if (dig[top] == 0 || n <= 0) return 0.0f;
+  const int p = 32 * top + 31 - __clz(dig[top]);                  // highest set bit
+  unsigned long long w;
+  int lowbit = 0;
+  if (p < 64) {
+    w = (static_cast<unsigned long long>(dig[1]) << 32) | dig[0];
+  } else {
+    // the 64 bits p-63 .. p; anything set below them is folded into bit 0, which
+    // lies under the rounding position of a 53-bit significand (a sticky bit)
+    lowbit = p - 63;
+    const int i0 = lowbit >> 5, off = lowbit & 31;
+    const unsigned long long lo64 = (static_cast<unsigned long long>(dig[i0 + 1]) << 32) | dig[i0];
+    w = off ? (lo64 >> off) | (static_cast<unsigned long long>(dig[i0 + 2]) << (64 - off)) : lo64;
+    bool sticky = off && (dig[i0] & ((1u << off) - 1u)) != 0;
+    for (int j = 0; j < i0; ++j) sticky |= dig[j] != 0;
+    if (sticky) w |= 1ull;
+  }
+  const double s = __dmul_rn(__ull2double_rn(w), pow2d(lowbit - 149));   // exact scaling
+  return __double2float_rn(__ddiv_rn(s, static_cast<double>(n)));
+}
+
 // One CTA per group of 256 blocks (16384 weights).  Full, aligned groups take
 // the vectorised path: each half-warp streams one block per iteration with
 // 16-byte loads, reduces its absmax with shuffles and writes 8 bytes of codes
@@ -50,12 +127,16 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float
                                                                      uint8_t *__restrict__ codes,
                                                                      uint8_t *__restrict__ absmax_q,
                                                                      float *__restrict__ group_scale, Nf4Table tab,
+                                                                     float *__restrict__ dq_abs,
+                                                                     unsigned long long *__restrict__ dq_acc,
                                                                      int *status) {
   __shared__ float s_thr[16];
   __shared__ float s_abs[kGroup];
   __shared__ float s_wmax[kQuantThreads / 32];
+  __shared__ unsigned long long s_acc[kSumDigits];
   const int t = threadIdx.x;
   if (t < 15) s_thr[t] = tab.thresh[t];
+  if (t < kSumDigits) s_acc[t] = 0;
   __syncthreads();
 
   const int64_t g = blockIdx.x;
@@ -104,6 +185,18 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float
   }
   __syncthreads();
 
+  if (dq_abs != nullptr) {
+    // Signed constants: keep a_b for the second pass and add it to the exact sum.
+    const float a = s_abs[t];
+    const int64_t blk = g * kGroup + t;
+    if (blk < nblocks) dq_abs[blk] = a;
+    warp_exact_add(a, s_acc);
+    __syncthreads();
+    if (t < kSumDigits && s_acc[t] != 0) atomicAdd(dq_acc + t, s_acc[t]);
+    if (bad) latch_status(status, QLORA_ERR_NONFINITE);
+    return;
+  }
+
   // Double quantization of this group's 256 block constants.
   const float a = s_abs[t];
   float m = a;
@@ -125,6 +218,40 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float
   if (bad) latch_status(status, QLORA_ERR_NONFINITE);
 }
 
+// Signed block constants of one group (one thread per block) against the
+// tensor-wide mean; every CTA derives mu from the exact sum itself.
+__global__ void __launch_bounds__(kQuantThreads) nf4_dq_signed_kernel(const float *__restrict__ dq_abs,
+                                                                      const unsigned long long *__restrict__ dq_acc,
+                                                                      int64_t nblocks, uint8_t *__restrict__ absmax_q,
+                                                                      float *__restrict__ group_scale,
+                                                                      float *__restrict__ mu_out) {
+  __shared__ float s_mu;
+  __shared__ float s_wmax[kQuantThreads / 32];
+  const int t = threadIdx.x;
+  const int64_t g = blockIdx.x;
+  if (t == 0) s_mu = exact_mean(dq_acc, nblocks);
+  __syncthreads();
+  const float mu = s_mu;
+  const int64_t blk = g * kGroup + t;
+  const float c = blk < nblocks ? __fsub_rn(__ldg(dq_abs + blk), mu) : 0.0f;
+  float m = fabsf(c);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((t & 31) == 0) s_wmax[t >> 5] = m;
+  __syncthreads();
+  float cm = s_wmax[0];
+#pragma unroll
+  for (int w = 1; w < kQuantThreads / 32; ++w) cm = fmaxf(cm, s_wmax[w]);
+  const float S = __fdiv_rn(cm, 127.0f);
+  if (blk < nblocks) {
+    int q = 0;
+    if (S != 0.0f) q = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(c, S)), -127.0f), 127.0f));
+    absmax_q[blk] = static_cast<uint8_t>(q & 0xFF);
+  }
+  if (t == 0) group_scale[g] = S;
+  if (g == 0 && t == 0) *mu_out = mu;
+}
+
 // Each thread turns 16 bytes of codes (32 weights, half of one block) into
 // 64 bytes of bf16 through the block's byte-permute table (decode.cuh), so a
 // warp streams 512 B in and 2 KB out per iteration.
@@ -137,10 +264,11 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
                                                                      Nf4Table tab) {
   const int64_t nchunk = (numel + 31) / 32;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const float mu = dq_offset(tab);
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nchunk; i += stride) {
     const int64_t e0 = i * 32;
     const int64_t blk = e0 >> 6;
-    const float ap = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(group_scale + (blk >> 8)));
+    const float ap = block_constant(__ldg(absmax_q + blk), __ldg(group_scale + (blk >> 8)), tab.qx, mu);
     uint32_t LO[4], HI[4];
     nf4_block_table(ap, tab, LO, HI);
     if (e0 + 32 <= numel) {
@@ -213,6 +341,7 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
   }
   __syncthreads();
   int it = 0;
+  const float mu = dq_offset(tab);
   float S = first < nchunks ? __ldg(group_scale + (first >> 1)) : 0.0f;   // one group per two chunks
   for (int64_t ch = first; ch < nchunks; ch += step, ++it) {
     const int ls = it % kDqStages, ob = it & 1;
@@ -224,7 +353,7 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
     __syncthreads();
     if (*abort_flag) break;
     const uint8_t *stage = cbuf + ls * kDqStageBytes;
-    const float ap = __fmul_rn(static_cast<float>(stage[kDqCodeBytes + (t >> 1)]), S);
+    const float ap = block_constant(stage[kDqCodeBytes + (t >> 1)], S, tab.qx, mu);
     uint32_t LO[4], HI[4];
     nf4_block_table(ap, tab, LO, HI);
     const uint4 cw = ld_shared_v4(smem_addr(stage + t * 16));
@@ -256,19 +385,34 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
 
 }  // namespace
 
+size_t quantize_workspace_bytes(int64_t numel) {
+  const int64_t nblocks = (numel + kBlock - 1) / kBlock;
+  return static_cast<size_t>((128 + 4 * nblocks + 255) / 256 * 256);
+}
+
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
-                            int format, int *status, cudaStream_t st) {
+                            const Nf4Table &tab, void *ws, int *status, cudaStream_t st) {
   const int64_t ngroups = (numel + kGroupElems - 1) / kGroupElems;
+  const int64_t nblocks = (numel + kBlock - 1) / kBlock;
+  const bool sgn = tab.qx != 0;
+  unsigned long long *acc = sgn ? static_cast<unsigned long long *>(ws) : nullptr;
+  float *abs_ws = sgn ? reinterpret_cast<float *>(static_cast<char *>(ws) + 128) : nullptr;
   prof_mark(kProfQuant, true, st);
+  if (sgn) {
+    cudaError_t e = cudaMemsetAsync(acc, 0, kSumDigits * sizeof(unsigned long long), st);
+    if (e != cudaSuccess) return e;
+  }
   nf4_quantize_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(W, numel, codes, absmax_q,
-                                                                                 group_scale, format_table(format), status);
+                                                                                 group_scale, tab, abs_ws, acc, status);
+  if (sgn)
+    nf4_dq_signed_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(
+        abs_ws, acc, nblocks, absmax_q, group_scale, const_cast<float *>(tab.offset));
   prof_mark(kProfQuant, false, st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale, int64_t numel,
-                              int format,
-                              uint16_t *out, cudaStream_t st) {
+                              const Nf4Table &tab, uint16_t *out, cudaStream_t st) {
   // whole double-quantization groups (two chunks each) on the bulk path
   const int64_t nfull = (numel / (kBlock * kGroup)) * (kBlock * kGroup / kDqChunk);
   prof_mark(kProfDequant, true, st);
@@ -279,7 +423,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
                                          kDqSmem);
     if (e != cudaSuccess) return e;
     nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, kDqSmem, st>>>(
-        codes, absmax_q, group_scale, nfull, out, format_table(format), status, wait_limit());
+        codes, absmax_q, group_scale, nfull, out, tab, status, wait_limit());
   }
   const int64_t done = nfull * kDqChunk;
   if (done < numel) {
@@ -289,8 +433,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
     const int64_t nchunk = (rest + 31) / 32;
     int64_t blocks = (nchunk + kDeqThreads - 1) / kDeqThreads;
     nf4_dequantize_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(
-        codes + done / 2, absmax_q + done / kBlock, group_scale + done / (kBlock * kGroup), rest, out + done,
-        format_table(format));
+        codes + done / 2, absmax_q + done / kBlock, group_scale + done / (kBlock * kGroup), rest, out + done, tab);
   }
   prof_mark(kProfDequant, false, st);
   return cudaGetLastError();

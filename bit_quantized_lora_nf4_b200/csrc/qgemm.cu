@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       *idx = n * kblocks + kb;
       return n < p.wN && kb < kblocks;
     };
+    const float mu = dq_offset(tab);
     uint32_t q_next = 0;
     float s_next = 0.0f;
     {
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < nsteps; ++i) {
       const int s = i % STAGES;
       const uint32_t ph = (i / STAGES) & 1;
-      const float ap = __fmul_rn(static_cast<float>(q_next), s_next);
+      const float ap = block_constant(q_next, s_next, tab.qx, mu);
       q_next = 0;
       s_next = 0.0f;
       if (i + 1 < p.nkb) {
@@ -349,11 +350,11 @@ qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st) {
   if (a.dgrad) {
     e = cudaFuncSetAttribute(qgemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) qgemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, format_table(a.format));
+    if (e == cudaSuccess) qgemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, a.tab);
   } else {
     e = cudaFuncSetAttribute(qgemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) qgemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, format_table(a.format));
+    if (e == cudaSuccess) qgemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tm_act, tm_codes, tm_lact, p, a.tab);
   }
   prof_mark(kind, false, st);
   if (e == cudaSuccess) e = cudaGetLastError();

@@ -299,6 +299,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         b.S = __ldg(p.group_scale + (idx >> 8));
       }
     };
+    const float mu = dq_offset(tab);
     BlockLoad bq[PREFETCH];                   // this group's next PREFETCH K-steps
 #pragma unroll
     for (int j = 0; j < PREFETCH; ++j) fetch(grp + j * NACC, bq[j]);
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
       if (i < p.nkb) {
-        const float ap = __fmul_rn(static_cast<float>(cur.q), cur.S);
+        const float ap = block_constant(cur.q, cur.S, tab.qx, mu);
         uint32_t LO[4], HI[4];
         nf4_block_table(ap, tab, LO, HI);
         const uint32_t words[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
@@ -439,7 +440,7 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const Nf4Table tab = format_table(a.format);
+  const Nf4Table tab = a.tab;
   const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);

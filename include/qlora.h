@@ -64,8 +64,10 @@ typedef enum {
 /* The frozen base weight W [rows=N (out), cols=K (in)] in NF4 + double quant.
  * All three arrays are device memory owned by the caller.
  *   codes       : ceil(rows*cols/2) bytes
- *   absmax_q    : ceil(rows*cols/64) bytes, one unsigned 8-bit constant per block
- *   group_scale : ceil(rows*cols/16384) fp32, one per group of 256 blocks     */
+ *   absmax_q    : ceil(rows*cols/64) bytes, one 8-bit constant per block
+ *   group_scale : ceil(rows*cols/16384) fp32, one per group of 256 blocks, and
+ *                 with QLORA_DQ_SIGNED one more fp32 after them: the offset mu
+ *                 (qlora_group_scale_bytes_dq gives the size)               */
 /* 4-bit code tables.  NF4 is the method's type; the other two are the plain
  * 4-bit float and integer types the pages compare it against (the same
  * storage, block constants and kernels, another 16-entry table):
@@ -79,6 +81,24 @@ typedef enum {
 #define QLORA_FORMAT_FP4 1
 #define QLORA_FORMAT_INT4 2
 
+/* Two readings of the 8-bit block constants ("NormalFloat, double
+ * quantization, paged optimizers": the per-block constants are themselves
+ * stored in 8 bits under a coarser set of constants; the 8-bit format is not
+ * given).  a_b is the exact fp32 absmax of block b, g its group of 256 blocks.
+ *   QLORA_DQ_PLAIN   unsigned codes, no offset:
+ *                      S_g = fl32(max_g a_b / 255),
+ *                      q_b = min(255, rne(fl32(a_b / S_g)))      (0 if S_g = 0),
+ *                      a'_b = fl32(q_b * S_g)
+ *   QLORA_DQ_SIGNED  signed codes around the tensor-wide mean constant:
+ *                      mu = fl32(fl64(fl64(exact sum of all a_b) / n_blocks)),
+ *                      c_b = fl32(a_b - mu),  S_g = fl32(max_g |c_b| / 127),
+ *                      q_b = clamp(rne(fl32(c_b / S_g)), -127, 127) (0 if S_g = 0),
+ *                      stored as its int8 bit pattern; a'_b = fl32(fl32(q_b * S_g) + mu).
+ *                    The sum is exact (integer arithmetic), so mu, and with it
+ *                    every stored byte, does not depend on the order of work. */
+#define QLORA_DQ_PLAIN 0
+#define QLORA_DQ_SIGNED 1
+
 typedef struct {
   int64_t rows;
   int64_t cols;
@@ -86,30 +106,49 @@ typedef struct {
   uint8_t *absmax_q;
   float *group_scale;
   int32_t format;     /* QLORA_FORMAT_*; 0 (NF4) for a zero-initialised struct */
-  int32_t reserved;   /* must be 0 */
+  int32_t dq;         /* QLORA_DQ_*; 0 (plain) for a zero-initialised struct   */
 } qlora_nf4_weight;
 
-/* Sizes in bytes of the three arrays for a rows x cols weight. */
+/* Sizes in bytes of the three arrays for a rows x cols weight.
+ * qlora_group_scale_bytes is the QLORA_DQ_PLAIN size; qlora_group_scale_bytes_dq
+ * takes the variant (4 bytes more for QLORA_DQ_SIGNED; 0 for an unknown one). */
 size_t qlora_codes_bytes(int64_t rows, int64_t cols);
 size_t qlora_absmax_bytes(int64_t rows, int64_t cols);
 size_t qlora_group_scale_bytes(int64_t rows, int64_t cols);
+size_t qlora_group_scale_bytes_dq(int64_t rows, int64_t cols, int dq);
 
 /* qlora_quantize_nf4 -- quantize fp32 weights once, up front (in out->format;
- * NF4 unless the caller chose another table).
+ * NF4 unless the caller chose another table; block constants as out->dq).
  * ("Where the memory goes": the base never changes, so it is quantized once.)
  *   W   : device fp32 [out->rows * out->cols], flat row-major.
  *   out : rows/cols set by the caller; codes/absmax_q/group_scale receive the
  *         result.  Any rows*cols >= 1 is accepted (last block/group partial).
  * Per block b: a_b = max|w| (exact fp32); n = fl32(w / a_b) (n = 0 if a_b = 0);
  * code = index of the nearest level of the table, ties to the lower index.
- * Per group g: c_g = max a_b; S_g = fl32(c_g / 255);
- * q_b = min(255, round-half-even(fl32(a_b / S_g))) (0 if S_g = 0).
+ * The block constants a_b are then stored as QLORA_DQ_* describes.
+ * QLORA_DQ_SIGNED needs a workspace: this call returns QLORA_ERR_WORKSPACE for
+ * it; use qlora_quantize_nf4_ws.
  * A non-finite weight latches QLORA_ERR_NONFINITE (outputs then undefined). */
 qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream);
 
-/* qlora_dequantize -- W' = bf16(fl32(v_code * fl32(q_b * S_g))) into a device
- * bf16 buffer of rows*cols elements, row-major.  ("Where the memory goes":
- * the 16-bit form each pass works with.)  Bit-exact by construction. */
+/* Workspace bytes qlora_quantize_nf4_ws needs (0 for QLORA_DQ_PLAIN; for
+ * QLORA_DQ_SIGNED 128 + 4 bytes per block, rounded up to 256). */
+size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols, int dq);
+
+/* qlora_quantize_nf4_ws -- qlora_quantize_nf4 with a caller-owned device
+ * workspace (16-byte aligned, ws_bytes >= qlora_quantize_workspace_bytes;
+ * ws may be NULL when that is 0).  For QLORA_DQ_SIGNED it holds the fp32 block
+ * constants between the pass that finds them and the pass that codes them
+ * against mu, and the exact sum (ten 64-bit words of 32-bit digits, cleared
+ * by the call).  rows*cols < 2^38 for QLORA_DQ_SIGNED
+ * (QLORA_ERR_UNSUPPORTED_SHAPE beyond). */
+qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/* qlora_dequantize -- W' = bf16(fl32(v_code * a'_b)) into a device bf16 buffer
+ * of rows*cols elements, row-major, a'_b the dequantized block constant of
+ * w->dq.  ("Where the memory goes": the 16-bit form each pass works with.)
+ * Bit-exact by construction. */
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream);
 
 /* Operation ids for qlora_workspace_bytes(). */

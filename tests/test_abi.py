@@ -113,3 +113,25 @@ def test_quantize_dequantize_argument_errors():
 def test_wait_limit_roundtrip():
     old = q.set_wait_limit(12345)
     assert q.set_wait_limit(old) == 12345
+
+
+def test_signed_block_constant_sizes_and_errors():
+    lib = q.load()
+    for rows, cols in ((256, 256), (4096, 11008), (3, 5)):
+        n = rows * cols
+        assert lib.qlora_group_scale_bytes_dq(rows, cols, q.DQ_PLAIN) == 4 * nf4.num_groups(n)
+        assert lib.qlora_group_scale_bytes_dq(rows, cols, q.DQ_SIGNED) == 4 * nf4.num_groups(n) + 4
+        assert lib.qlora_quantize_workspace_bytes(rows, cols, q.DQ_PLAIN) == 0
+        ws = lib.qlora_quantize_workspace_bytes(rows, cols, q.DQ_SIGNED)
+        assert ws % 256 == 0 and ws >= 128 + 4 * nf4.num_blocks(n)
+    assert lib.qlora_group_scale_bytes_dq(4, 4, 2) == 0
+    w = q.Nf4WeightC(256, 256, FAKE, FAKE, FAKE, q.FORMAT_NF4, q.DQ_SIGNED)
+    assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(w), None) == 7          # needs the workspace call
+    assert lib.qlora_quantize_nf4_ws(FAKE, ctypes.byref(w), FAKE, 16, None) == 7
+    assert lib.qlora_quantize_nf4_ws(FAKE, ctypes.byref(w), MIS, 1 << 20, None) == 3
+    big = q.Nf4WeightC(1 << 20, 1 << 18, FAKE, FAKE, FAKE, q.FORMAT_NF4, q.DQ_SIGNED)
+    assert lib.qlora_quantize_nf4_ws(FAKE, ctypes.byref(big), FAKE, 1 << 62, None) == 2
+    bad = q.Nf4WeightC(256, 256, FAKE, FAKE, FAKE, q.FORMAT_NF4, 2)
+    assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(bad), None) == 1
+    assert lib.qlora_dequantize(ctypes.byref(bad), FAKE, None) == 1
+    assert _fwd(bad) == 1
