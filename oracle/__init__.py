@@ -18,6 +18,8 @@ Sources (web pages, cited by title and section):
                weight compression".
   [Cap-qlora]  same page, entry "qlora 4-bit quantization with nf4/fp4 data
                types and lora adapters".
+  [LQ-abs]     "LQ-LoRA: Low-rank Plus Quantized Matrix Decomposition for
+               Efficient Language Model Finetuning", abstract.
 
 Module map:
   nf4.py     codebook, blockwise absmax, nearest-code encode, double
@@ -25,6 +27,9 @@ Module map:
   linear.py  fp64 LoRA linear forward / backward on the dequantized weight.
   layer.py   fp64 LLaMA-shaped decoder layer around seven such linears
              (torch CPU fp64 with autograd), for the decoder-layer tests.
+  lq.py      low-rank plus quantized decomposition W ~ Q + L1 L2 ("LQ-LoRA",
+             abstract): residuals, truncated and randomized SVD, the
+             alternation.
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py`` except
 the quantitative equal-usage property of the codebook levels,
@@ -32,5 +37,5 @@ which is reported only (parity unpinned for that claim; absmax normalisation
 makes it approximate).
 """
 
-from . import nf4, linear  # noqa: F401
+from . import nf4, linear, lq  # noqa: F401
 # layer.py imports torch; it is imported where used (from oracle import layer).

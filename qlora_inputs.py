@@ -91,3 +91,28 @@ def make_weight(n_rows: int, n_cols: int, seed: int, std: float = 0.02) -> torch
     """Gaussian fp32 weight matrix (first draw of the case's generator)."""
     rng = np.random.default_rng(seed)
     return torch.from_numpy(rng.standard_normal((n_rows, n_cols), dtype=np.float32) * np.float32(std))
+
+
+def make_lowrank_weight(n_rows: int, n_cols: int, rank: int, seed: int, std: float = 0.02,
+                        strength: tuple = (4.0, 1.5)) -> torch.Tensor:
+    """Gaussian fp32 weight plus a planted rank-`rank` component, the structure a
+    low-rank plus quantized decomposition looks for.  Draw order: the Gaussian
+    [n_rows, n_cols] (scaled by std), then two Gaussian [n, rank] matrices whose
+    orthonormal bases (library QR, fp64) give the singular vectors.  The planted
+    singular values fall linearly from strength[0] to strength[1] times
+    std (sqrt(n_rows) + sqrt(n_cols)), the largest singular value of the
+    Gaussian part, so every planted direction stands out of it."""
+    rng = np.random.default_rng(seed)
+    G = rng.standard_normal((n_rows, n_cols), dtype=np.float32) * np.float32(std)
+    U, _ = np.linalg.qr(rng.standard_normal((n_rows, rank)))
+    V, _ = np.linalg.qr(rng.standard_normal((n_cols, rank)))
+    edge = std * (np.sqrt(n_rows) + np.sqrt(n_cols))
+    s = edge * np.linspace(strength[0], strength[1], rank)
+    return torch.from_numpy((G.astype(np.float64) + (U * s) @ V.T).astype(np.float32))
+
+
+def make_test_matrix(n_cols: int, width: int, seed: int) -> torch.Tensor:
+    """The Gaussian test matrix [n_cols, width] fp32 a randomized range finder
+    draws (passed in as an input, so both sides use the same numbers)."""
+    rng = np.random.default_rng(seed)
+    return torch.from_numpy(rng.standard_normal((n_cols, width), dtype=np.float32))
