@@ -252,6 +252,7 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     extras["llama65b"] = measure_65b(q, dev, pk, barrier)
     extras["decoder_layer"] = measure_layer(q, dev, pk, barrier)
     extras["dq_signed"] = measure_dq_signed(q, dev, pk, barrier)
+    extras["lq_decompose"] = measure_lq(q, dev, pk, barrier)
     e2e = measure_e2e(q, rep, dev, min(args.steps, 20), barrier, allmax, world)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -403,6 +404,53 @@ def measure_dq_signed(q, dev, pk, barrier):
     out["note"] = "errors on the 4096x4096 Gaussian q-projection weight"
     out["workload"] = "llama7b_projections_m4096_r64_fwd_bwd_signed_block_constants"
     del rep, Wq
+    torch.cuda.empty_cache()
+    return out
+
+
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x fp32 lanes x 2 flops x max SM clock
+
+
+def measure_lq(q, dev, pk, barrier):
+    """Low-rank plus quantized decomposition of the 4096 x 4096 q-projection-shaped weight with a
+    planted rank-64 part (r = 64, test matrix width 72, 2 power rounds, 2 alternation rounds):
+    time per decomposition and the residual products' fp32 rate against the CUDA-core peak."""
+    N = K = 4096
+    r, l, power, iters = 64, 72, 2, 2
+    W = qi.make_lowrank_weight(N, K, r, seed=99).to(dev)
+    Om = qi.make_test_matrix(K, l, seed=100).to(dev)
+    ws = torch.empty(q.load().qlora_lq_workspace_bytes(N, K, r, l, 0), dtype=torch.uint8, device=dev)
+
+    def run():
+        return q.lq_decompose(W, r, Om, power=power, iters=iters, workspace=ws)
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    reps = 3
+    ms = timed(run, reps, barrier) / reps
+    q.profile_enable(True)
+    w, L1, L2, err = run()
+    torch.cuda.synchronize()
+    pms, pn = q.profile_read(q.PROF_LQ_PRODUCT)
+    parts = {name: round(q.profile_read(k)[0], 3) for name, k in (
+        ("products", q.PROF_LQ_PRODUCT), ("residual_and_error", q.PROF_LQ_RESIDUAL), ("cholesky", q.PROF_LQ_CHOL),
+        ("jacobi", q.PROF_LQ_JACOBI), ("gram_small_sums", q.PROF_LQ_SMALL), ("quantizer", q.PROF_QUANT))}
+    q.profile_enable(False)
+    flops = pn * 2 * N * K * l
+    tf = flops / (pms * 1e-3) / 1e12
+    plain = q.quantize_nf4(W)
+    plain_err = float((q.dequantize(plain).double() - W.double()).norm() / W.double().norm())
+    e = err.cpu().numpy()
+    out = {"ms_per_decomposition": round(ms, 3),
+           "products": {"launches": int(pn), "ms": round(pms, 3), "achieved": round(tf, 2), "unit": "TFLOP/s",
+                        "bound": "alu", "peak": round(FP32_FMA_PEAK_TFLOPS, 1),
+                        "frac": round(tf / FP32_FMA_PEAK_TFLOPS, 4), "share": round(pms / ms, 3),
+                        "flops_per_launch": 2 * N * K * l},
+           "ms_by_kernel_kind": parts,
+           "rel_error": {"plain_nf4": round(plain_err, 5), "after_quantization": [round(x, 5) for x in e[:, 0]],
+                         "after_rank_r_step": [round(x, 5) for x in e[:, 1]]},
+           "workload": "lq_decompose_4096x4096_planted_rank64_r64_l72_power2_iters2"}
+    del W, Om, ws, w, L1, L2, plain
     torch.cuda.empty_cache()
     return out
 
@@ -582,6 +630,14 @@ def run_ncu_case(args):
         torch.cuda.synchronize()
         assert q.device_status() == 0
         return
+    if name == "lq":     # the low-rank plus quantized decomposition of a 4096 x 4096 weight
+        W = qi.make_lowrank_weight(4096, 4096, 64, seed=99).to(dev)
+        Om = qi.make_test_matrix(4096, 72, seed=100).to(dev)
+        for _ in range(args.warmup + args.steps):
+            q.lq_decompose(W, 64, Om, power=1, iters=1)
+        torch.cuda.synchronize()
+        assert q.device_status() == 0
+        return
     case = {"q": qi.LLAMA7B[0], "up": qi.LLAMA7B[1], "down": qi.LLAMA7B[2]}.get(name, qi.LLAMA7B[1])
     M = {"gemv1": 1, "gemv16": 16}.get(name, case.M)
     d = qi.make_linear(case, M=M)
@@ -607,7 +663,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--ncu-case", choices=["step", "q", "up", "down", "gemv1", "gemv16", "dequant"], default=None,
+    ap.add_argument("--ncu-case", choices=["step", "q", "up", "down", "gemv1", "gemv16", "dequant", "lq"], default=None,
                     help="profiling entry: run only one projection's calls (--warmup + --steps times), no JSON")
     args = ap.parse_args()
     if args.ncu_case:

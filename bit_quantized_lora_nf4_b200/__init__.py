@@ -33,7 +33,8 @@ EXPORTS = (
     "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
     "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
     "qlora_profile_read", "qlora_linear_fwd_noalloc", "qlora_format_codebook", "qlora_group_scale_bytes_dq",
-    "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_ws",
+    "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_ws", "qlora_lq_workspace_bytes", "qlora_lq_decompose",
+    "qlora_lq_quantize_residual", "qlora_lq_lowrank",
 )
 
 # 4-bit code tables (QLORA_FORMAT_*): NF4 is the method's type; FP4 (e2m1) and
@@ -45,7 +46,8 @@ FORMAT_NF4, FORMAT_FP4, FORMAT_INT4 = 0, 1, 2
 DQ_PLAIN, DQ_SIGNED = 0, 1
 
 # Kernel kinds of the timing hook (qlora_profile_read).
-PROF_ALL, PROF_GEMM_FWD, PROF_GEMM_DGRAD, PROF_LORA, PROF_QUANT, PROF_DEQUANT, PROF_GEMV = range(7)
+(PROF_ALL, PROF_GEMM_FWD, PROF_GEMM_DGRAD, PROF_LORA, PROF_QUANT, PROF_DEQUANT, PROF_GEMV, PROF_LQ_PRODUCT,
+ PROF_LQ_RESIDUAL, PROF_LQ_CHOL, PROF_LQ_JACOBI, PROF_LQ_SMALL) = range(12)
 
 
 class QloraError(RuntimeError):
@@ -94,6 +96,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_group_scale_bytes_dq": (sz, [i64, i64, i32]),
         "qlora_quantize_workspace_bytes": (sz, [i64, i64, i32]),
         "qlora_quantize_nf4_ws": (i32, [vp, wp, vp, sz, vp]),
+        "qlora_lq_workspace_bytes": (sz, [i64, i64, i32, i32, i32]),
+        "qlora_lq_decompose": (i32, [vp, wp, vp, vp, i32, vp, i32, i32, i32, vp, vp, sz, vp]),
+        "qlora_lq_quantize_residual": (i32, [vp, vp, vp, i32, wp, vp, sz, vp]),
+        "qlora_lq_lowrank": (i32, [vp, i64, i64, wp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -213,6 +219,59 @@ def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, format: int = FO
     _check(lib.qlora_quantize_nf4_ws(_ptr(W), ctypes.byref(s), _ptr(workspace), nbytes, _stream()),
            "qlora_quantize_nf4_ws")
     return w
+
+
+def lq_decompose(W: torch.Tensor, r: int, Omega: torch.Tensor, power: int = 2, iters: int = 4,
+                 format: int = FORMAT_NF4, dq: int = DQ_PLAIN, workspace: torch.Tensor | None = None):
+    """W ~ W'(Q) + L1 L2 (qlora_lq_decompose).  W: contiguous fp32 CUDA [N, K];
+    Omega: fp32 CUDA [K, l] test matrix.  Returns (NF4Weight Q, L1 fp32 [N, r],
+    L2 fp32 [r, K], err fp64 [iters, 2]: relative error after each round's
+    quantization and after its rank-r step)."""
+    lib = load()
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and W.dim() == 2
+    assert Omega.is_cuda and Omega.dtype == torch.float32 and Omega.is_contiguous()
+    N, K = W.shape
+    l = Omega.shape[1]
+    w = NF4Weight.empty(N, K, W.device, format, dq)
+    L1 = torch.empty((N, r), dtype=torch.float32, device=W.device)
+    L2 = torch.empty((r, K), dtype=torch.float32, device=W.device)
+    err = torch.empty((iters, 2), dtype=torch.float64, device=W.device)
+    need = int(lib.qlora_lq_workspace_bytes(N, K, r, l, dq))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=W.device)
+    s = w.c_struct()
+    _check(lib.qlora_lq_decompose(_ptr(W), ctypes.byref(s), _ptr(L1), _ptr(L2), r, _ptr(Omega), l, power, iters,
+                                  _ptr(err), _ptr(workspace), workspace.numel(), _stream()), "qlora_lq_decompose")
+    return w, L1, L2, err
+
+
+def lq_quantize_residual(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, format: int = FORMAT_NF4,
+                         dq: int = DQ_PLAIN) -> NF4Weight:
+    """Q = quantize(fl32(W - L1 L2)) with the fp64 low-rank product (qlora_lq_quantize_residual)."""
+    lib = load()
+    N, K = W.shape
+    r = L1.shape[1]
+    w = NF4Weight.empty(N, K, W.device, format, dq)
+    ws = torch.empty(max(16, int(lib.qlora_lq_workspace_bytes(N, K, r, 0, dq))), dtype=torch.uint8, device=W.device)
+    s = w.c_struct()
+    _check(lib.qlora_lq_quantize_residual(_ptr(W), _ptr(L1), _ptr(L2), r, ctypes.byref(s), _ptr(ws), ws.numel(),
+                                          _stream()), "qlora_lq_quantize_residual")
+    return w
+
+
+def lq_lowrank(W: torch.Tensor, Q: NF4Weight | None, Omega: torch.Tensor, r: int, power: int = 2):
+    """(L1 [N, r], L2 [r, K]) ~ rank-r part of W - W'(Q) (of W when Q is None) (qlora_lq_lowrank)."""
+    lib = load()
+    N, K = W.shape
+    l = Omega.shape[1]
+    L1 = torch.empty((N, r), dtype=torch.float32, device=W.device)
+    L2 = torch.empty((r, K), dtype=torch.float32, device=W.device)
+    dq = Q.dq if Q is not None else DQ_PLAIN
+    ws = torch.empty(max(16, int(lib.qlora_lq_workspace_bytes(N, K, r, l, dq))), dtype=torch.uint8, device=W.device)
+    s = Q.c_struct() if Q is not None else None
+    _check(lib.qlora_lq_lowrank(_ptr(W), N, K, ctypes.byref(s) if s is not None else None, _ptr(Omega), l, power, r,
+                                _ptr(L1), _ptr(L2), _ptr(ws), ws.numel(), _stream()), "qlora_lq_lowrank")
+    return L1, L2
 
 
 def dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:

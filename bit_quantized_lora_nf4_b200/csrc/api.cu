@@ -323,6 +323,9 @@ qlora_status run_h(const Plan &p, void *ws, const uint16_t *X, const uint16_t *A
 }
 
 }  // namespace
+
+qlora_status validate_weight(const qlora_nf4_weight *w) { return check_weight(w); }
+
 }  // namespace qlora
 
 using namespace qlora;

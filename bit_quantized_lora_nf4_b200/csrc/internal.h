@@ -18,6 +18,8 @@ const Nf4Table &format_table(int format);
 // reading of its block constants (signed ones point `offset` at mu, stored
 // after the group scales).
 Nf4Table weight_table(const qlora_nf4_weight *w);
+// Pointer, size, format and alignment checks of a weight header (QLORA_OK or the error).
+qlora_status validate_weight(const qlora_nf4_weight *w);
 
 // Address of the device status word on the current device (nullptr on error).
 int *device_status_ptr();
@@ -31,7 +33,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---- kernel timing hook (see qlora_profile_enable) --------------------------
 enum ProfKind { kProfAll = 0, kProfGemmFwd = 1, kProfGemmDgrad = 2, kProfLora = 3, kProfQuant = 4, kProfDequant = 5,
-                kProfGemv = 6, kProfKinds = 7 };
+                kProfGemv = 6, kProfLqProduct = 7, kProfLqResidual = 8, kProfLqChol = 9, kProfLqJacobi = 10,
+                kProfLqSmall = 11, kProfKinds = 12 };
 // Records an event before (begin=true) or after a launch of `kind` on `st` when profiling is on.
 void prof_mark(int kind, bool begin, cudaStream_t st);
 

@@ -1,0 +1,972 @@
+// Low-rank plus quantized decomposition of a frozen weight, W ~ Q + L1 L2.
+//
+// "LQ-LoRA: Low-rank Plus Quantized Matrix Decomposition for Efficient
+// Language Model Finetuning", abstract: each pretrained matrix is split by an
+// iterative algorithm into a high-precision low-rank part and a quantized
+// part; finetuning keeps the quantized part fixed and trains the low-rank one.
+// The alternation run here starts from the principal rank-r part of W and
+// then repeats
+//     Q = quantize(W - L1 L2);   L1 L2 = rank-r approximation of W - W'(Q)
+// with the library's own quantizer.  The rank-r step is randomized subspace
+// iteration (range finder with power iterations on a caller-given Gaussian
+// test matrix, then the eigen-decomposition of the small l x l matrix B B^T).
+//
+// Every pass over the N x K residual R = W - W' reads W (fp32) and the packed
+// weight and forms R on the fly; R is never stored.  The small l x l steps
+// (Gram sums, Cholesky, triangular inverse, Jacobi eigen-decomposition) run in
+// fp64 in one CTA each.  Reductions are split over CTAs with partial results
+// summed in a fixed order, so a run is bit-reproducible.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int kLqMaxL = 96;       // widest test matrix (l); keeps the l x l work in one CTA
+constexpr int kLqThreads = 256;
+
+// The quantized part as the kernels see it (absent for the first rank-r step,
+// which factors W itself).
+struct LqQuant {
+  const uint8_t *codes;      // nullptr: no quantized part, R = W
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  Nf4Table tab;
+};
+
+// W'[e] (the bf16 value of the dequantized weight, as fp32) for flat index e;
+// `lv` holds the 16 levels in shared memory.
+__device__ __forceinline__ float lq_wq(const LqQuant &q, const float *lv, int64_t e, float mu) {
+  const uint32_t code = (__ldg(q.codes + (e >> 1)) >> ((e & 1) * 4)) & 15u;
+  const int64_t blk = e >> 6;
+  const float ap = block_constant(__ldg(q.absmax_q + blk), __ldg(q.group_scale + (blk >> 8)), q.tab.qx, mu);
+  return __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[code], ap)));
+}
+
+__device__ __forceinline__ void lq_load_levels(const LqQuant &q, float *lv, float *mu_s) {
+  if (threadIdx.x < 16) lv[threadIdx.x] = q.tab.level[threadIdx.x];
+  if (threadIdx.x == 0) *mu_s = q.codes ? dq_offset(q.tab) : 0.0f;
+}
+
+// Fixed-order block sum of one fp64 value per thread (256 threads).
+__device__ double block_sum_f64(double v, double *red) {
+  red[threadIdx.x] = v;
+  __syncthreads();
+  for (int s = kLqThreads / 2; s > 0; s >>= 1) {
+    if (static_cast<int>(threadIdx.x) < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  const double out = red[0];
+  __syncthreads();
+  return out;
+}
+
+// ---- low-rank residual -------------------------------------------------------
+// Tile of 32 rows x 128 columns, thread (tx, ty) owns rows ty + 8 i and
+// columns tx + 32 c.  P = sum_j L1[n, j] L2[j, k] is accumulated in fp64 in
+// the order j = 0 .. r-1 (each product of two fp32 values is exact in fp64, so
+// an FMA gives the same sum as a product then an add).  Outputs, each optional:
+//   E[n, k] = fl32(fl64(W) - P)                       (quantizer input)
+//   part[cta] = sum over the tile of (fl64(W - W') - P)^2, fl64(W) - P without
+//   a quantized part (no L1: P = 0).
+constexpr int kResRows = 32, kResCols = 128, kResJ = 32;
+
+__global__ void __launch_bounds__(kLqThreads) lq_residual_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                                 const float *__restrict__ L1,
+                                                                 const float *__restrict__ L2, int r, LqQuant q,
+                                                                 float *__restrict__ E, double *__restrict__ part) {
+  __shared__ float l1s[kResRows][kResJ + 1];
+  __shared__ float l2s[kResJ][kResCols];
+  __shared__ float lv[16];
+  __shared__ float mu_s;
+  __shared__ double red[kLqThreads];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kResRows, k0 = static_cast<int64_t>(blockIdx.x) * kResCols;
+  lq_load_levels(q, lv, &mu_s);
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
+  if (L1 != nullptr) {
+    for (int j0 = 0; j0 < r; j0 += kResJ) {
+      for (int idx = threadIdx.x; idx < kResRows * kResJ; idx += kLqThreads) {
+        const int rr = idx / kResJ, jj = idx % kResJ;
+        const int64_t n = n0 + rr;
+        l1s[rr][jj] = (n < N && j0 + jj < r) ? __ldg(L1 + n * r + j0 + jj) : 0.0f;
+      }
+      for (int idx = threadIdx.x; idx < kResJ * kResCols; idx += kLqThreads) {
+        const int jj = idx / kResCols, cc = idx % kResCols;
+        const int64_t k = k0 + cc;
+        l2s[jj][cc] = (k < K && j0 + jj < r) ? __ldg(L2 + static_cast<int64_t>(j0 + jj) * K + k) : 0.0f;
+      }
+      __syncthreads();
+      const int jn = min(kResJ, r - j0);
+      for (int jj = 0; jj < jn; ++jj) {
+        double a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = static_cast<double>(l1s[ty + 8 * i][jj]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) b[c] = static_cast<double>(l2s[jj][tx + 32 * c]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[i][c] = __fma_rn(a[i], b[c], acc[i][c]);
+      }
+      __syncthreads();
+    }
+  } else {
+    __syncthreads();   // levels and mu are visible
+  }
+  const float mu = mu_s;
+  double sq = 0.0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t n = n0 + ty + 8 * i;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t k = k0 + tx + 32 * c;
+      if (n < N && k < K) {
+        const int64_t e = n * K + k;
+        const float w = __ldg(W + e);
+        if (E) E[e] = __double2float_rn(__dsub_rn(static_cast<double>(w), acc[i][c]));
+        if (part) {
+          double d = static_cast<double>(w);
+          if (q.codes) d = __dsub_rn(d, static_cast<double>(lq_wq(q, lv, e, mu)));
+          d = __dsub_rn(d, acc[i][c]);
+          sq = __fma_rn(d, d, sq);
+        }
+      }
+    }
+  }
+  if (part) {
+    const double s = block_sum_f64(sq, red);
+    if (threadIdx.x == 0) part[static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x] = s;
+  }
+}
+
+// out[0] = sum of part[0 .. n) in index order (sum mode), or
+// out[0] = sqrt(sum / *norm2) (relative error mode, norm2 != nullptr).
+__global__ void lq_sum_kernel(const double *__restrict__ part, int64_t n, const double *__restrict__ norm2,
+                              double *__restrict__ out) {
+  __shared__ double red[kLqThreads];
+  // thread t sums a contiguous stretch, then the stretches are added in order
+  const int64_t per = (n + kLqThreads - 1) / kLqThreads;
+  const int64_t a = static_cast<int64_t>(threadIdx.x) * per, b = min(n, a + per);
+  double s = 0.0;
+  for (int64_t i = a; i < b; ++i) s = __dadd_rn(s, part[i]);
+  const double tot = block_sum_f64(s, red);
+  if (threadIdx.x == 0) *out = norm2 ? (*norm2 > 0.0 ? sqrt(tot / *norm2) : 0.0) : tot;
+}
+
+// ---- residual tiles: 8 consecutive elements of one row per thread -------------
+// K % 64 == 0, so a run of 8 never leaves its 64-element block and its codes
+// are one aligned 32-bit word.  The raw loads are issued one chunk ahead and
+// decoded after the current chunk's arithmetic.
+struct Raw8 {
+  float4 w0, w1;
+  uint32_t codes, q;
+  float S;
+  bool valid;   // false past the matrix or the CTA's range: the run decodes to 0
+};
+
+__device__ __forceinline__ void raw8_load(const float *W, const LqQuant &q, int64_t n, int64_t N, int64_t k,
+                                          int64_t kend, int64_t K, Raw8 &r) {
+  r.valid = n < N && k < kend;
+  if (r.valid) {
+    const int64_t e = n * K + k;
+    r.w0 = __ldg(reinterpret_cast<const float4 *>(W + e));
+    r.w1 = __ldg(reinterpret_cast<const float4 *>(W + e) + 1);
+    if (q.codes) {
+      r.codes = __ldg(reinterpret_cast<const uint32_t *>(q.codes + (e >> 1)));
+      r.q = __ldg(q.absmax_q + (e >> 6));
+      r.S = __ldg(q.group_scale + (e >> 14));
+    }
+  } else {
+    r.w0 = r.w1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    r.codes = 0;
+    r.q = 0;
+    r.S = 0.0f;
+  }
+}
+
+// R = fl32(W - W') for the 8 elements (0 for an invalid run).
+__device__ __forceinline__ void raw8_decode(const Raw8 &r, const LqQuant &q, const float *lv, float mu,
+                                            float (&out)[8]) {
+  const float w[8] = {r.w0.x, r.w0.y, r.w0.z, r.w0.w, r.w1.x, r.w1.y, r.w1.z, r.w1.w};
+  if (!q.codes || !r.valid) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = w[i];   // W itself; zeros for an invalid run
+    return;
+  }
+  const float ap = block_constant(r.q, r.S, q.tab.qx, mu);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(r.codes >> (4 * i)) & 15u], ap)));
+    out[i] = __fsub_rn(w[i], wq);
+  }
+}
+
+// ---- Y = R M: tall-skinny product over K -------------------------------------
+// CTA (bx, split): 32 rows of R x all l (<= 96) columns over the split's range
+// of K, walked in chunks of 64 (one NF4 block per row); writes
+// part[split][n][c].  Thread (tx, ty): rows 4 ty .. 4 ty + 3, columns tx + 32 m.
+// Tile fill: thread t decodes row t / 8, columns 8 (t % 8) .. + 7.
+constexpr int kRmRows = 32, kRmChunk = 64;
+
+__global__ void __launch_bounds__(kLqThreads) lq_rmul_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                             LqQuant q, const float *__restrict__ M, int l,
+                                                             int64_t k_per, float *__restrict__ part) {
+  __shared__ __align__(16) float Rs[kRmRows][kRmChunk + 4];
+  __shared__ float Ms[kRmChunk][kLqMaxL];
+  __shared__ float lv[16];
+  __shared__ float mu_s;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int fr = threadIdx.x >> 3, fc = (threadIdx.x & 7) * 8;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kRmRows;
+  lq_load_levels(q, lv, &mu_s);
+  __syncthreads();
+  const float mu = mu_s;
+  float acc[4][3];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int m = 0; m < 3; ++m) acc[i][m] = 0.0f;
+  const int64_t ka = static_cast<int64_t>(blockIdx.y) * k_per, kb = min(K, ka + k_per);
+  Raw8 raw;
+  raw8_load(W, q, n0 + fr, N, ka + fc, kb, K, raw);
+  for (int64_t k0 = ka; k0 < kb; k0 += kRmChunk) {
+    float rv[8];
+    raw8_decode(raw, q, lv, mu, rv);
+    *reinterpret_cast<float4 *>(&Rs[fr][fc]) = make_float4(rv[0], rv[1], rv[2], rv[3]);
+    *reinterpret_cast<float4 *>(&Rs[fr][fc + 4]) = make_float4(rv[4], rv[5], rv[6], rv[7]);
+    for (int idx = threadIdx.x; idx < kRmChunk * l; idx += kLqThreads) {
+      const int kk = idx / l, c = idx % l;
+      Ms[kk][c] = (k0 + kk < kb) ? __ldg(M + (k0 + kk) * l + c) : 0.0f;
+    }
+    raw8_load(W, q, n0 + fr, N, k0 + kRmChunk + fc, kb, K, raw);   // next chunk, in flight meanwhile
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < kRmChunk; kk += 4) {
+      float4 a[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4 *>(&Rs[4 * ty + i][kk]);
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const int c = tx + 32 * m;
+        if (c < l) {
+          const float b0 = Ms[kk][c], b1 = Ms[kk + 1][c], b2 = Ms[kk + 2][c], b3 = Ms[kk + 3][c];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[i][m] = fmaf(a[i].x, b0, acc[i][m]);
+            acc[i][m] = fmaf(a[i].y, b1, acc[i][m]);
+            acc[i][m] = fmaf(a[i].z, b2, acc[i][m]);
+            acc[i][m] = fmaf(a[i].w, b3, acc[i][m]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  float *Y = part + static_cast<int64_t>(blockIdx.y) * N * l;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t n = n0 + 4 * ty + i;
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const int c = tx + 32 * m;
+      if (n < N && c < l) Y[n * l + c] = acc[i][m];
+    }
+  }
+}
+
+// ---- Z = R^T Y: tall-skinny product over N, split over row ranges ------------
+// CTA (bx, split): columns 64 bx .. 64 bx + 63 of R x all l columns of Y, rows
+// [rows_per * split, ...) walked 32 at a time.  Thread (tx, ty): R columns
+// 8 ty .. 8 ty + 7, Y columns tx + 32 m.  Writes part[split][k][c].
+constexpr int kRtCols = 64, kRtRows = 32;
+
+__global__ void __launch_bounds__(kLqThreads) lq_rtmul_kernel(const float *__restrict__ W, int64_t N, int64_t K,
+                                                              LqQuant q, const float *__restrict__ Y, int l,
+                                                              int64_t rows_per, float *__restrict__ part) {
+  __shared__ __align__(16) float Rs[kRtRows][kRtCols + 4];
+  __shared__ float Ys[kRtRows][kLqMaxL];
+  __shared__ float lv[16];
+  __shared__ float mu_s;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int fr = threadIdx.x >> 3, fc = (threadIdx.x & 7) * 8;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kRtCols;
+  const int64_t na = static_cast<int64_t>(blockIdx.y) * rows_per, nb = min(N, na + rows_per);
+  lq_load_levels(q, lv, &mu_s);
+  __syncthreads();
+  const float mu = mu_s;
+  float acc[8][3];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int m = 0; m < 3; ++m) acc[i][m] = 0.0f;
+  Raw8 raw;
+  raw8_load(W, q, na + fr, nb, k0 + fc, K, K, raw);
+  for (int64_t n0 = na; n0 < nb; n0 += kRtRows) {
+    float rv[8];
+    raw8_decode(raw, q, lv, mu, rv);
+    *reinterpret_cast<float4 *>(&Rs[fr][fc]) = make_float4(rv[0], rv[1], rv[2], rv[3]);
+    *reinterpret_cast<float4 *>(&Rs[fr][fc + 4]) = make_float4(rv[4], rv[5], rv[6], rv[7]);
+    for (int idx = threadIdx.x; idx < kRtRows * l; idx += kLqThreads) {
+      const int rr = idx / l, c = idx % l;
+      Ys[rr][c] = (n0 + rr < nb) ? __ldg(Y + (n0 + rr) * l + c) : 0.0f;
+    }
+    raw8_load(W, q, n0 + kRtRows + fr, nb, k0 + fc, K, K, raw);   // next rows, in flight meanwhile
+    __syncthreads();
+#pragma unroll 2
+    for (int rr = 0; rr < kRtRows; ++rr) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&Rs[rr][8 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&Rs[rr][8 * ty + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const int c = tx + 32 * m;
+        if (c < l) {
+          const float b = Ys[rr][c];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i][m] = fmaf(a[i], b, acc[i][m]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  float *out = part + static_cast<int64_t>(blockIdx.y) * K * l;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t k = k0 + 8 * ty + i;
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const int c = tx + 32 * m;
+      if (k < K && c < l) out[k * l + c] = acc[i][m];
+    }
+  }
+}
+
+// Z[e] = sum over splits s = 0 .. ns-1 (in order) of part[s][e].
+__global__ void lq_sum_splits_kernel(const float *__restrict__ part, int ns, int64_t n, float *__restrict__ Z) {
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = part[e];
+    for (int i = 1; i < ns; ++i) s = __fadd_rn(s, part[static_cast<int64_t>(i) * n + e]);
+    Z[e] = s;
+  }
+}
+
+// ---- Gram matrices of tall fp32 matrices, in fp64 -----------------------------
+// CTA (g, part): entries g * per_group + t + 256 m (t the thread) of the l x l
+// matrix X^T X over the part's rows; each product of two fp32 values is exact
+// in fp64.  part[p][e] holds the part sums; lq_gram_sum_kernel adds the parts
+// in part order.
+constexpr int kGramRows = 32;
+constexpr int kGramGroups = 4;
+constexpr int kGramMaxParts = 64;
+constexpr int kGramPer = (kLqMaxL * kLqMaxL / kGramGroups + kLqThreads - 1) / kLqThreads;   // 9
+
+__global__ void __launch_bounds__(kLqThreads) lq_gram_kernel(const float *__restrict__ X, int64_t rows, int l,
+                                                             int64_t rows_per, double *__restrict__ part) {
+  __shared__ float Xs[kGramRows][kLqMaxL];
+  const int64_t na = static_cast<int64_t>(blockIdx.y) * rows_per, nb = min(rows, na + rows_per);
+  const int ll = l * l;
+  const int per_group = (ll + kGramGroups - 1) / kGramGroups;
+  const int e0 = blockIdx.x * per_group, e1 = min(ll, e0 + per_group);
+  double acc[kGramPer];
+  int ea[kGramPer], eb[kGramPer];
+#pragma unroll
+  for (int m = 0; m < kGramPer; ++m) {
+    const int e = e0 + threadIdx.x + kLqThreads * m;
+    acc[m] = 0.0;
+    ea[m] = e < e1 ? e / l : 0;
+    eb[m] = e < e1 ? e % l : 0;
+  }
+  for (int64_t n0 = na; n0 < nb; n0 += kGramRows) {
+    for (int idx = threadIdx.x; idx < kGramRows * l; idx += kLqThreads) {
+      const int rr = idx / l, c = idx % l;
+      Xs[rr][c] = (n0 + rr < nb) ? __ldg(X + (n0 + rr) * l + c) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rr = 0; rr < kGramRows; ++rr) {
+#pragma unroll
+      for (int m = 0; m < kGramPer; ++m)
+        acc[m] = __fma_rn(static_cast<double>(Xs[rr][ea[m]]), static_cast<double>(Xs[rr][eb[m]]), acc[m]);
+    }
+    __syncthreads();
+  }
+  double *out = part + static_cast<int64_t>(blockIdx.y) * ll;
+#pragma unroll
+  for (int m = 0; m < kGramPer; ++m) {
+    const int e = e0 + threadIdx.x + kLqThreads * m;
+    if (e < e1) out[e] = acc[m];
+  }
+}
+
+__global__ void lq_gram_sum_kernel(const double *__restrict__ part, int nparts, int ll, double *__restrict__ G) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= ll) return;
+  double s = 0.0;
+  for (int p = 0; p < nparts; ++p) s = __dadd_rn(s, part[static_cast<int64_t>(p) * ll + e]);
+  G[e] = s;
+}
+
+// Row pitch of l x l fp64 matrices in shared memory: odd, so that a warp
+// walking down a column touches every bank pair once.
+__host__ __device__ __forceinline__ int lq_pitch(int l) { return l | 1; }
+
+// G (global, l x l, dense) into shared memory with row pitch lp.
+__device__ void lq_load_gram(const double *__restrict__ Gg, int l, int lp, double *G) {
+  for (int e = threadIdx.x; e < l * l; e += blockDim.x) G[(e / l) * lp + e % l] = Gg[e];
+  __syncthreads();
+}
+
+// ---- Cholesky and triangular inverse (one CTA) ---------------------------------
+// G = L L^T (right-looking, column by column); a column whose pivot is not
+// above 1e-24 of the largest diagonal entry is numerically dependent and is
+// dropped (zero in L and in the inverse).  T = L^-T, so that X T has
+// orthonormal columns when G = X^T X.
+__global__ void __launch_bounds__(kLqThreads) lq_chol_inv_kernel(const double *__restrict__ Gg, int l,
+                                                                 double *__restrict__ T) {
+  extern __shared__ __align__(16) double lq_smem[];
+  const int lp = lq_pitch(l);
+  double *G = lq_smem;               // [l][lp]: lower triangle becomes L
+  double *Xi = lq_smem + l * lp;     // [l][lp]: L^-1 (lower)
+  __shared__ double dmax;
+  __shared__ int dead[kLqMaxL];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  lq_load_gram(Gg, l, lp, G);
+  if (threadIdx.x == 0) {
+    double m = 0.0;
+    for (int a = 0; a < l; ++a) m = fmax(m, G[a * lp + a]);
+    dmax = m;
+  }
+  __syncthreads();
+  const double tol = 1e-24 * dmax;
+  for (int j = 0; j < l; ++j) {
+    const double piv = G[j * lp + j];
+    const bool dj = !(piv > tol);
+    const double d = dj ? 0.0 : sqrt(piv);
+    __syncthreads();   // every thread has read the pivot
+    // column j of L below the diagonal
+    for (int a = j + 1 + threadIdx.x; a < l; a += blockDim.x) G[a * lp + j] = dj ? 0.0 : G[a * lp + j] / d;
+    if (threadIdx.x == 0) {
+      G[j * lp + j] = d;
+      dead[j] = dj;
+    }
+    __syncthreads();
+    // trailing update of the lower triangle: G[a][b] -= L[a][j] L[b][j], j < b <= a (a row per warp)
+    for (int a = j + 1 + warp; a < l; a += nwarps) {
+      const double laj = G[a * lp + j];
+      for (int b = j + 1 + lane; b <= a; b += 32) G[a * lp + b] = __fma_rn(-laj, G[b * lp + j], G[a * lp + b]);
+    }
+    __syncthreads();
+  }
+  // L^-1 by forward substitution, one column per thread (four partial sums per dot product)
+  for (int c = threadIdx.x; c < l; c += blockDim.x) {
+    for (int j = 0; j < l; ++j) {
+      double v = 0.0;
+      if (j >= c && !dead[j]) {
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        int i = c;
+        for (; i + 3 < j; i += 4) {
+          s0 = __fma_rn(G[j * lp + i], Xi[i * lp + c], s0);
+          s1 = __fma_rn(G[j * lp + i + 1], Xi[(i + 1) * lp + c], s1);
+          s2 = __fma_rn(G[j * lp + i + 2], Xi[(i + 2) * lp + c], s2);
+          s3 = __fma_rn(G[j * lp + i + 3], Xi[(i + 3) * lp + c], s3);
+        }
+        for (; i < j; ++i) s0 = __fma_rn(G[j * lp + i], Xi[i * lp + c], s0);
+        v = ((j == c ? 1.0 : 0.0) - ((s0 + s1) + (s2 + s3))) / G[j * lp + j];
+      }
+      Xi[j * lp + c] = v;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < l * l; e += blockDim.x) {
+    const int a = e / l, b = e % l;
+    T[e] = Xi[b * lp + a];
+  }
+}
+
+// ---- small right factor: out = X S (X fp32 [rows, l], S fp64 [l, cols]) -------
+// fp64 accumulation, fp32 result; `transposed` stores out[c][n] ([cols, rows]).
+constexpr int kSgRows = 32;
+
+__global__ void __launch_bounds__(kLqThreads) lq_small_gemm_kernel(const float *__restrict__ X, int64_t rows, int l,
+                                                                   const double *__restrict__ S, int cols,
+                                                                   float *__restrict__ out, int transposed) {
+  extern __shared__ __align__(16) double lq_smem[];
+  double *Ss = lq_smem;                                        // [l][cols]
+  float *Xs = reinterpret_cast<float *>(lq_smem + l * cols);   // [kSgRows][l]
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kSgRows;
+  for (int e = threadIdx.x; e < l * cols; e += blockDim.x) Ss[e] = S[e];
+  for (int idx = threadIdx.x; idx < kSgRows * l; idx += blockDim.x) {
+    const int rr = idx / l, c = idx % l;
+    Xs[idx] = (n0 + rr < rows) ? __ldg(X + (n0 + rr) * l + c) : 0.0f;
+  }
+  __syncthreads();
+  for (int c = tx; c < cols; c += 32) {
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int j = 0; j < l; ++j) {
+      const double s = Ss[j * cols + c];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = __fma_rn(static_cast<double>(Xs[(4 * ty + i) * l + j]), s, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t n = n0 + 4 * ty + i;
+      if (n < rows) {
+        if (transposed)
+          out[static_cast<int64_t>(c) * rows + n] = __double2float_rn(acc[i]);
+        else
+          out[n * cols + c] = __double2float_rn(acc[i]);
+      }
+    }
+  }
+}
+
+// ---- symmetric eigen-decomposition (one CTA), parallel cyclic Jacobi ------------
+// C = sum of Gram parts (l x l, l even).  Each sweep pairs all indices in l - 1
+// rounds (circle method: index l-1 stays, the others rotate), the l/2 disjoint
+// rotations of a round are applied together: A <- J^T A J, V <- V J, with
+// c, s from the symmetric 2x2 Schur step (t = sign(tau) / (|tau| + sqrt(1 +
+// tau^2)), tau = (a_qq - a_pp) / (2 a_pq)).  Sweeps stop when the off-diagonal
+// mass is below 1e-24 of the total (entries about 1e-12 of the matrix; fp64
+// rounding alone leaves about l^2 1e-32), at most kJacobiSweeps.  Then the r largest
+// eigenvalues lam (ties to the lower index), s = sqrt(lam), and
+//   M1[:, i] = v_i sqrt(s_i),  M2[:, i] = v_i / sqrt(s_i)
+// (zero for s_i <= 1e-12 s_0), so that with C = B B^T and B = Q^T R:
+// L1 = Q M1, L2^T = B^T M2.
+constexpr int kJacobiSweeps = 30;
+
+__global__ void __launch_bounds__(kLqThreads) lq_jacobi_kernel(const double *__restrict__ Gg, int l, int r,
+                                                               double *__restrict__ M1, double *__restrict__ M2,
+                                                               double *__restrict__ sv) {
+  extern __shared__ __align__(16) double lq_smem[];
+  const int lp = lq_pitch(l);
+  double *A = lq_smem;               // [l][lp]
+  double *V = lq_smem + l * lp;      // [l][lp]
+  __shared__ double cs[kLqMaxL / 2][2];
+  __shared__ int pr[kLqMaxL / 2][2];
+  __shared__ double red[kLqThreads];
+  __shared__ int order[kLqMaxL];
+  __shared__ int taken[kLqMaxL];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  lq_load_gram(Gg, l, lp, A);
+  for (int e = threadIdx.x; e < l * l; e += blockDim.x) V[(e / l) * lp + e % l] = (e / l == e % l) ? 1.0 : 0.0;
+  __syncthreads();
+  const int h = l / 2;
+  for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
+    double off = 0.0, tot = 0.0;
+    for (int a = warp; a < l; a += nwarps)
+      for (int b = lane; b < l; b += 32) {
+        const double v = A[a * lp + b] * A[a * lp + b];
+        tot += v;
+        if (a != b) off += v;
+      }
+    off = block_sum_f64(off, red);
+    tot = block_sum_f64(tot, red);
+    if (!(off > 1e-24 * tot)) break;
+    for (int round = 0; round < l - 1; ++round) {
+      if (static_cast<int>(threadIdx.x) < h) {
+        const int i = threadIdx.x;
+        int p, q;
+        if (i == 0) {
+          p = round;
+          q = l - 1;
+        } else {
+          p = (round + i) % (l - 1);
+          q = (round - i + (l - 1)) % (l - 1);
+        }
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
+        const double apq = A[p * lp + q];
+        double c = 1.0, s = 0.0;
+        if (apq != 0.0) {
+          const double tau = (A[q * lp + q] - A[p * lp + p]) / (2.0 * apq);
+          const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+          c = 1.0 / sqrt(1.0 + t * t);
+          s = t * c;
+        }
+        pr[i][0] = p;
+        pr[i][1] = q;
+        cs[i][0] = c;
+        cs[i][1] = s;
+      }
+      __syncthreads();
+      // rows: A <- J^T A (a pair per warp, its columns over the lanes)
+      for (int i = warp; i < h; i += nwarps) {
+        const int p = pr[i][0], q = pr[i][1];
+        const double c = cs[i][0], s = cs[i][1];
+        for (int j = lane; j < l; j += 32) {
+          const double ap = A[p * lp + j], aq = A[q * lp + j];
+          A[p * lp + j] = c * ap - s * aq;
+          A[q * lp + j] = s * ap + c * aq;
+        }
+      }
+      __syncthreads();
+      // columns: A <- A J, V <- V J
+      for (int i = warp; i < h; i += nwarps) {
+        const int p = pr[i][0], q = pr[i][1];
+        const double c = cs[i][0], s = cs[i][1];
+        for (int j = lane; j < l; j += 32) {
+          const double ap = A[j * lp + p], aq = A[j * lp + q];
+          A[j * lp + p] = c * ap - s * aq;
+          A[j * lp + q] = s * ap + c * aq;
+          const double vp = V[j * lp + p], vq = V[j * lp + q];
+          V[j * lp + p] = c * vp - s * vq;
+          V[j * lp + q] = s * vp + c * vq;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x == 0) {
+    // the r largest eigenvalues, ties to the lower index
+    for (int a = 0; a < l; ++a) taken[a] = 0;
+    for (int i = 0; i < r; ++i) {
+      int best = -1;
+      for (int a = 0; a < l; ++a)
+        if (!taken[a] && (best < 0 || A[a * lp + a] > A[best * lp + best])) best = a;
+      taken[best] = 1;
+      order[i] = best;
+    }
+  }
+  __syncthreads();
+  const double s0 = sqrt(fmax(A[order[0] * lp + order[0]], 0.0));
+  for (int e = threadIdx.x; e < l * r; e += blockDim.x) {
+    const int a = e / r, i = e % r;
+    const double si = sqrt(fmax(A[order[i] * lp + order[i]], 0.0));
+    const bool keep = s0 > 0.0 && si > 1e-12 * s0;
+    const double hh = keep ? sqrt(si) : 0.0;
+    const double v = V[a * lp + order[i]];
+    M1[e] = keep ? v * hh : 0.0;
+    M2[e] = keep ? v / hh : 0.0;
+    if (sv && a == 0) sv[i] = si;
+  }
+}
+
+}  // namespace
+
+// ---- host side ------------------------------------------------------------------
+namespace {
+
+struct LqPlan {
+  int64_t N, K;
+  int r, l;
+  int64_t rt_rows, rt_splits;      // row range per split and number of splits of R^T Y
+  int64_t rm_cols, rm_splits;      // K range per split and number of splits of R M
+  int64_t res_ctas;                // CTAs of the residual kernel (error parts)
+  int64_t gram_parts_max;
+  size_t E, qws, Ya, Yb, Za, Zb, Zpart, Gpart, G, T, M1, M2, sv, errpart, norm2, total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// at most kGramMaxParts parts of a multiple of kGramRows rows each
+void gram_split(int64_t rows, int64_t *parts, int64_t *per) {
+  const int64_t q = ceil_div(ceil_div(rows, kGramMaxParts), kGramRows) * kGramRows;
+  *per = q;
+  *parts = ceil_div(rows, q);
+}
+
+LqPlan lq_plan(int64_t N, int64_t K, int r, int l, int dq) {
+  LqPlan p{};
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.l = l;
+  // both products aim at about four CTAs per SM
+  const int64_t col_tiles = ceil_div(K, kRtCols);
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(ceil_div(4 * 148, col_tiles), ceil_div(N, kRtRows)));
+  p.rt_rows = ceil_div(ceil_div(N, splits), kRtRows) * kRtRows;
+  p.rt_splits = ceil_div(N, p.rt_rows);
+  const int64_t row_tiles = ceil_div(N, kRmRows);
+  splits = std::max<int64_t>(1, std::min<int64_t>(ceil_div(4 * 148, row_tiles), ceil_div(K, kRmChunk)));
+  p.rm_cols = ceil_div(ceil_div(K, splits), kRmChunk) * kRmChunk;
+  p.rm_splits = ceil_div(K, p.rm_cols);
+  p.res_ctas = ceil_div(K, kResCols) * ceil_div(N, kResRows);
+  p.gram_parts_max = kGramMaxParts;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  p.E = take(4 * static_cast<size_t>(N * K));
+  p.qws = take(dq == QLORA_DQ_SIGNED ? quantize_workspace_bytes(N * K) : 0);
+  p.Ya = take(4 * static_cast<size_t>(N) * l);
+  p.Yb = take(4 * static_cast<size_t>(N) * l);
+  p.Za = take(4 * static_cast<size_t>(K) * l);
+  p.Zb = take(4 * static_cast<size_t>(K) * l);
+  p.Zpart = take(4 * std::max(static_cast<size_t>(p.rt_splits) * K, static_cast<size_t>(p.rm_splits) * N) * l);
+  p.Gpart = take(8 * static_cast<size_t>(p.gram_parts_max) * l * l);
+  p.G = take(8 * static_cast<size_t>(l) * l);
+  p.T = take(8 * static_cast<size_t>(l) * l);
+  p.M1 = take(8 * static_cast<size_t>(l) * r);
+  p.M2 = take(8 * static_cast<size_t>(l) * r);
+  p.sv = take(8 * static_cast<size_t>(r));
+  p.errpart = take(8 * static_cast<size_t>(p.res_ctas));
+  p.norm2 = take(8);
+  p.total = off;
+  return p;
+}
+
+template <typename T>
+T *wsp(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+struct LqRun {
+  const LqPlan &p;
+  void *ws;
+  const float *W;
+  cudaStream_t st;
+  cudaError_t err = cudaSuccess;
+
+  void check() {
+    if (err == cudaSuccess) err = cudaGetLastError();
+  }
+
+  // part[] = squared-error parts of W - W'(q) - L1 L2 (and E when given)
+  void residual(const float *L1, const float *L2, const LqQuant &q, float *E, double *part) {
+    const dim3 grid(static_cast<unsigned>(ceil_div(p.K, kResCols)), static_cast<unsigned>(ceil_div(p.N, kResRows)));
+    prof_mark(kProfLqResidual, true, st);
+    lq_residual_kernel<<<grid, kLqThreads, 0, st>>>(W, p.N, p.K, L1, L2, p.r, q, E, part);
+    prof_mark(kProfLqResidual, false, st);
+    check();
+  }
+  void sum(const double *part, int64_t n, const double *norm2, double *out) {
+    lq_sum_kernel<<<1, kLqThreads, 0, st>>>(part, n, norm2, out);
+    check();
+  }
+  void rmul(const LqQuant &q, const float *M, float *Y) {
+    const dim3 grid(static_cast<unsigned>(ceil_div(p.N, kRmRows)), static_cast<unsigned>(p.rm_splits));
+    float *part = wsp<float>(ws, p.Zpart);
+    prof_mark(kProfLqProduct, true, st);
+    lq_rmul_kernel<<<grid, kLqThreads, 0, st>>>(W, p.N, p.K, q, M, p.l, p.rm_cols, part);
+    prof_mark(kProfLqProduct, false, st);
+    check();
+    sum_splits(part, static_cast<int>(p.rm_splits), p.N * p.l, Y);
+  }
+  void sum_splits(const float *part, int ns, int64_t n, float *out) {
+    prof_mark(kProfLqSmall, true, st);
+    lq_sum_splits_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 148 * 8)), 256, 0, st>>>(
+        part, ns, n, out);
+    prof_mark(kProfLqSmall, false, st);
+    check();
+  }
+  void rtmul(const LqQuant &q, const float *Y, float *Z) {
+    const dim3 grid(static_cast<unsigned>(ceil_div(p.K, kRtCols)), static_cast<unsigned>(p.rt_splits));
+    float *part = wsp<float>(ws, p.Zpart);
+    prof_mark(kProfLqProduct, true, st);
+    lq_rtmul_kernel<<<grid, kLqThreads, 0, st>>>(W, p.N, p.K, q, Y, p.l, p.rt_rows, part);
+    prof_mark(kProfLqProduct, false, st);
+    check();
+    sum_splits(part, static_cast<int>(p.rt_splits), p.K * p.l, Z);
+  }
+  // G = X^T X (fp64, l x l) of X [rows, l]
+  void gram(const float *X, int64_t rows) {
+    int64_t parts, per;
+    gram_split(rows, &parts, &per);
+    prof_mark(kProfLqSmall, true, st);
+    const dim3 grid(kGramGroups, static_cast<unsigned>(parts));
+    lq_gram_kernel<<<grid, kLqThreads, 0, st>>>(X, rows, p.l, per, wsp<double>(ws, p.Gpart));
+    const int ll = p.l * p.l;
+    lq_gram_sum_kernel<<<static_cast<unsigned>(ceil_div(ll, 256)), 256, 0, st>>>(
+        wsp<double>(ws, p.Gpart), static_cast<int>(parts), ll, wsp<double>(ws, p.G));
+    prof_mark(kProfLqSmall, false, st);
+    check();
+  }
+  void small_gemm(const float *X, int64_t rows, const double *S, int cols, float *out, bool transposed) {
+    const size_t smem = 8 * static_cast<size_t>(p.l) * cols + 4 * static_cast<size_t>(kSgRows) * p.l;
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(lq_small_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+    if (err != cudaSuccess) return;
+    prof_mark(kProfLqSmall, true, st);
+    lq_small_gemm_kernel<<<static_cast<unsigned>(ceil_div(rows, kSgRows)), kLqThreads, smem, st>>>(
+        X, rows, p.l, S, cols, out, transposed ? 1 : 0);
+    prof_mark(kProfLqSmall, false, st);
+    check();
+  }
+  // the columns of *X [rows, l] made orthonormal by Cholesky QR, `passes`
+  // times (the span is unchanged; a second pass restores orthogonality to
+  // working precision).  The result lands in *X or *tmp; the pointers are
+  // swapped so that *X names it.
+  void orth(float **X, float **tmp, int64_t rows, int passes) {
+    const size_t smem = 16 * static_cast<size_t>(p.l) * lq_pitch(p.l);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(lq_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+    for (int pass = 0; pass < passes; ++pass) {
+      gram(*X, rows);
+      if (err != cudaSuccess) return;
+      prof_mark(kProfLqChol, true, st);
+      lq_chol_inv_kernel<<<1, kLqThreads, smem, st>>>(wsp<double>(ws, p.G), p.l, wsp<double>(ws, p.T));
+      prof_mark(kProfLqChol, false, st);
+      check();
+      small_gemm(*X, rows, wsp<double>(ws, p.T), p.l, *tmp, false);
+      std::swap(*X, *tmp);
+    }
+  }
+  // L1 L2 = rank-r approximation of R (randomized subspace iteration)
+  void rsvd(const LqQuant &q, const float *Omega, int power, float *L1, float *L2) {
+    float *Ya = wsp<float>(ws, p.Ya), *Yb = wsp<float>(ws, p.Yb);
+    float *Za = wsp<float>(ws, p.Za), *Zb = wsp<float>(ws, p.Zb);
+    // one Cholesky QR pass between power rounds, two for the basis B is formed from
+    rmul(q, Omega, Ya);
+    orth(&Ya, &Yb, p.N, power == 0 ? 2 : 1);
+    for (int i = 0; i < power; ++i) {
+      rtmul(q, Ya, Za);
+      orth(&Za, &Zb, p.K, 1);
+      rmul(q, Za, Ya);
+      orth(&Ya, &Yb, p.N, i + 1 == power ? 2 : 1);
+    }
+    rtmul(q, Ya, Za);   // B^T = R^T Q
+    gram(Za, p.K);
+    const size_t smem = 16 * static_cast<size_t>(p.l) * lq_pitch(p.l);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(lq_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+    if (err != cudaSuccess) return;
+    prof_mark(kProfLqJacobi, true, st);
+    lq_jacobi_kernel<<<1, kLqThreads, smem, st>>>(wsp<double>(ws, p.G), p.l, p.r, wsp<double>(ws, p.M1),
+                                                  wsp<double>(ws, p.M2), wsp<double>(ws, p.sv));
+    prof_mark(kProfLqJacobi, false, st);
+    check();
+    small_gemm(Ya, p.N, wsp<double>(ws, p.M1), p.r, L1, false);
+    small_gemm(Za, p.K, wsp<double>(ws, p.M2), p.r, L2, true);
+  }
+};
+
+}  // namespace
+
+}  // namespace qlora
+
+using namespace qlora;
+
+#define LQ_TRY(expr)                          \
+  do {                                        \
+    const qlora_status lq_st_ = (expr);       \
+    if (lq_st_ != QLORA_OK) return lq_st_;    \
+  } while (0)
+
+namespace {
+
+// Shared argument checks; fills the plan.  l = 0 means "no rank-r step" (the
+// residual quantizer alone), checked as l = r.
+qlora_status lq_args(const float *W, int64_t N, int64_t K, int r, int l, int dq, void *ws, size_t ws_bytes,
+                     LqPlan *plan) {
+  if (!W || N < 1 || K < 1) return QLORA_ERR_INVALID_ARG;
+  const int lc = l == 0 ? r : l;
+  if (r < 1 || lc < r || lc > kLqMaxL || (lc & 1)) return QLORA_ERR_INVALID_ARG;
+  if (N < lc || K < lc) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (l != 0 && K % kBlock != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;   // the products walk whole blocks
+  if (dq == QLORA_DQ_SIGNED && N * K >= (int64_t(1) << 38)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  *plan = lq_plan(N, K, r, lc, dq);
+  if (!ws || ws_bytes < plan->total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qlora_lq_workspace_bytes(int64_t rows, int64_t cols, int r, int l, int dq) {
+  const int lc = l == 0 ? r : l;
+  if (rows < 1 || cols < 1 || r < 1 || lc < r || lc > kLqMaxL || (dq != QLORA_DQ_PLAIN && dq != QLORA_DQ_SIGNED))
+    return 0;
+  return lq_plan(rows, cols, r, lc, dq).total;
+}
+
+qlora_status qlora_lq_quantize_residual(const float *W, const float *L1, const float *L2, int r,
+                                        const qlora_nf4_weight *Q, void *ws, size_t ws_bytes, void *stream) {
+  if (!Q || !L1 || !L2) return QLORA_ERR_INVALID_ARG;
+  LQ_TRY(validate_weight(Q));
+  LqPlan p;
+  LQ_TRY(lq_args(W, Q->rows, Q->cols, r, 0, Q->dq, ws, ws_bytes, &p));
+  if (!aligned16(L1) || !aligned16(L2)) return QLORA_ERR_MISALIGNED;
+  int *status = device_status_ptr();
+  if (!status) return QLORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LqRun run{p, ws, W, st};
+  const Nf4Table tab = weight_table(Q);
+  float *E = wsp<float>(ws, p.E);
+  run.residual(L1, L2, LqQuant{nullptr, nullptr, nullptr, tab}, E, nullptr);
+  if (run.err == cudaSuccess)
+    run.err = launch_quantize(E, p.N * p.K, Q->codes, Q->absmax_q, Q->group_scale, tab,
+                              Q->dq == QLORA_DQ_SIGNED ? wsp<void>(ws, p.qws) : nullptr, status, st);
+  return run.err == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_lq_lowrank(const float *W, int64_t rows, int64_t cols, const qlora_nf4_weight *Q,
+                              const float *Omega, int l, int power, int r, float *L1, float *L2, void *ws,
+                              size_t ws_bytes, void *stream) {
+  if (!Omega || !L1 || !L2 || power < 0 || power > 16) return QLORA_ERR_INVALID_ARG;
+  if (l < 1) return QLORA_ERR_INVALID_ARG;
+  if (Q) {
+    LQ_TRY(validate_weight(Q));
+    if (Q->rows != rows || Q->cols != cols) return QLORA_ERR_INVALID_ARG;
+  }
+  LqPlan p;
+  LQ_TRY(lq_args(W, rows, cols, r, l, Q ? Q->dq : QLORA_DQ_PLAIN, ws, ws_bytes, &p));
+  if (!aligned16(Omega) || !aligned16(L1) || !aligned16(L2)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LqRun run{p, ws, W, st};
+  const Nf4Table tab = Q ? weight_table(Q) : format_table(QLORA_FORMAT_NF4);
+  const LqQuant q = Q ? LqQuant{Q->codes, Q->absmax_q, Q->group_scale, tab} : LqQuant{nullptr, nullptr, nullptr, tab};
+  run.rsvd(q, Omega, power, L1, L2);
+  return run.err == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_lq_decompose(const float *W, const qlora_nf4_weight *Q, float *L1, float *L2, int r,
+                                const float *Omega, int l, int power, int iters, double *err, void *ws,
+                                size_t ws_bytes, void *stream) {
+  if (!Q || !L1 || !L2 || !Omega || !err || l < 1) return QLORA_ERR_INVALID_ARG;
+  if (power < 0 || power > 16 || iters < 1 || iters > 1000) return QLORA_ERR_INVALID_ARG;
+  LQ_TRY(validate_weight(Q));
+  LqPlan p;
+  LQ_TRY(lq_args(W, Q->rows, Q->cols, r, l, Q->dq, ws, ws_bytes, &p));
+  if (!aligned16(L1) || !aligned16(L2) || !aligned16(Omega) || !aligned16(err)) return QLORA_ERR_MISALIGNED;
+  int *status = device_status_ptr();
+  if (!status) return QLORA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  LqRun run{p, ws, W, st};
+  const Nf4Table tab = weight_table(Q);
+  const LqQuant none{nullptr, nullptr, nullptr, tab};
+  const LqQuant quant{Q->codes, Q->absmax_q, Q->group_scale, tab};
+  double *part = wsp<double>(ws, p.errpart);
+  double *norm2 = wsp<double>(ws, p.norm2);
+  float *E = wsp<float>(ws, p.E);
+
+  run.residual(nullptr, nullptr, none, nullptr, part);   // ||W||^2
+  run.sum(part, p.res_ctas, nullptr, norm2);
+  run.rsvd(none, Omega, power, L1, L2);                   // principal rank-r part of W
+  for (int t = 0; t < iters && run.err == cudaSuccess; ++t) {
+    run.residual(L1, L2, none, E, nullptr);               // E = W - L1 L2
+    if (run.err == cudaSuccess)
+      run.err = launch_quantize(E, p.N * p.K, Q->codes, Q->absmax_q, Q->group_scale, tab,
+                                Q->dq == QLORA_DQ_SIGNED ? wsp<void>(ws, p.qws) : nullptr, status, st);
+    run.residual(L1, L2, quant, nullptr, part);           // before the rank-r step
+    run.sum(part, p.res_ctas, norm2, err + 2 * t);
+    run.rsvd(quant, Omega, power, L1, L2);
+    run.residual(L1, L2, quant, nullptr, part);           // after it
+    run.sum(part, p.res_ctas, norm2, err + 2 * t + 1);
+  }
+  return run.err == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // extern "C"

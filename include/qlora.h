@@ -229,6 +229,58 @@ qlora_status qlora_nf4_codebook(float *out);
  * unknown format or a NULL levels pointer. */
 qlora_status qlora_format_codebook(int format, float *levels, float *thresh);
 
+/* ---- Low-rank plus quantized decomposition ------------------------------
+ * ("LQ-LoRA: Low-rank Plus Quantized Matrix Decomposition for Efficient
+ * Language Model Finetuning", abstract: an iterative algorithm splits each
+ * pretrained matrix into a high-precision low-rank part and a quantized part;
+ * finetuning keeps the quantized part fixed and trains the low-rank one.)
+ *
+ * qlora_lq_decompose -- W ~ W'(Q) + L1 L2.  Starts from the principal rank-r
+ * part of W, then `iters` rounds of
+ *     E = fl32(fl64(W) - P)  (P = L1 L2 summed in fp64 over j = 0 .. r-1),
+ *     Q = qlora_quantize_nf4(E) in Q->format / Q->dq,
+ *     L1 L2 = rank-r approximation of R = fl32(W - W'(Q)).
+ * The rank-r step is randomized subspace iteration on R: Y = orth(R Omega),
+ * `power` times Y = orth(R orth(R^T Y)), B = Y^T R, B B^T = U diag(lam) U^T
+ * (lam descending), s = sqrt(lam[:r]), L1 = Y U_r diag(sqrt(s)),
+ * L2 = diag(1/sqrt(s)) U_r^T B; components with s_i <= 1e-12 s_0 are zero.
+ * orth() is Cholesky QR done twice; the l x l steps run in fp64.
+ *   W     : device fp32 [N, K] (N = Q->rows, K = Q->cols), not modified.
+ *   Q     : the weight header; its arrays receive the final quantized part
+ *           (sized for Q->dq, as for qlora_quantize_nf4).
+ *   L1    : device fp32 [N, r];  L2 : device fp32 [r, K]  (outputs).
+ *   Omega : device fp32 [K, l] Gaussian test matrix (the random numbers the
+ *           method draws; the caller supplies them).  r <= l <= 96, l even,
+ *           N >= l, K >= l.  0 <= power <= 16, 1 <= iters <= 1000.
+ *   err   : device fp64 [2 iters]: err[2t] = ||W - W' - L1 L2||_F / ||W||_F
+ *           after round t's quantization, err[2t+1] after its rank-r step.
+ *   ws    : device workspace of qlora_lq_workspace_bytes(N, K, r, l, Q->dq)
+ *           bytes (about 4 N K + 8 (N + K) l bytes).
+ * Every reduction is split over CTAs with parts added in a fixed order: the
+ * same inputs give the same bits.  Returns QLORA_ERR_UNSUPPORTED_SHAPE for
+ * N < l, K < l or K % 64 != 0 (the rank-r step walks whole 64-element blocks). */
+size_t qlora_lq_workspace_bytes(int64_t rows, int64_t cols, int r, int l, int dq);
+
+/* qlora_lq_quantize_residual -- one quantization step of the decomposition:
+ * Q = qlora_quantize_nf4(fl32(fl64(W) - P)), P = L1 L2 summed in fp64 over
+ * j = 0 .. r-1 (each product of two fp32 values is exact in fp64).  W fp32
+ * [N, K], L1 fp32 [N, r], L2 fp32 [r, K] (device); Q as for the quantizer.
+ * ws: qlora_lq_workspace_bytes(N, K, r, 0, Q->dq) bytes or more.  Bit-exact. */
+qlora_status qlora_lq_quantize_residual(const float *W, const float *L1, const float *L2, int r,
+                                        const qlora_nf4_weight *Q, void *ws, size_t ws_bytes, void *stream);
+
+/* qlora_lq_lowrank -- one rank-r step: L1 L2 ~ R with R = fl32(W - W'(Q)), or
+ * R = W when Q is NULL, by the randomized subspace iteration described above
+ * (Omega [cols, l], `power` rounds).  rows/cols give W's shape (and must match
+ * Q's).  ws: qlora_lq_workspace_bytes(rows, cols, r, l, dq) bytes or more. */
+qlora_status qlora_lq_lowrank(const float *W, int64_t rows, int64_t cols, const qlora_nf4_weight *Q,
+                              const float *Omega, int l, int power, int r, float *L1, float *L2, void *ws,
+                              size_t ws_bytes, void *stream);
+
+qlora_status qlora_lq_decompose(const float *W, const qlora_nf4_weight *Q, float *L1, float *L2, int r,
+                                const float *Omega, int l, int power, int iters, double *err, void *ws,
+                                size_t ws_bytes, void *stream);
+
 /* Synchronize `stream`, return the latched device status and clear it. */
 qlora_status qlora_device_status(void *stream);
 
@@ -249,7 +301,10 @@ qlora_status qlora_selftest_wait_timeout(uint64_t cycles, void *stream);
  * counts the launches, per kind:
  *   0 all kernels, 1 fused dequant-GEMM forward, 2 fused dequant-GEMM dgrad,
  *   3 adapter (low-rank) GEMMs and their reductions, 4 quantizer,
- *   5 dequantizer, 6 dequant-GEMV.
+ *   5 dequantizer, 6 dequant-GEMV; the decomposition (qlora_lq_*): 7 the
+ *   residual products R M and R^T Y, 8 the low-rank residual and error
+ *   kernel, 9 Cholesky and triangular inverse, 10 Jacobi eigen-decomposition,
+ *   11 Gram, small-factor and split-sum kernels.
  * qlora_profile_enable(1) clears the records; qlora_profile_read()
  * synchronizes the device and returns the summed event time (ms) and the
  * launch count of one kind.  Not thread-safe; off by default. */

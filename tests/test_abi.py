@@ -135,3 +135,32 @@ def test_signed_block_constant_sizes_and_errors():
     assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(bad), None) == 1
     assert lib.qlora_dequantize(ctypes.byref(bad), FAKE, None) == 1
     assert _fwd(bad) == 1
+
+
+def test_lq_sizes_and_argument_errors():
+    lib = q.load()
+    assert lib.qlora_lq_workspace_bytes(256, 512, 16, 24, 0) >= 4 * 256 * 512
+    assert lib.qlora_lq_workspace_bytes(256, 512, 16, 0, 0) > 0          # residual quantizer alone
+    assert lib.qlora_lq_workspace_bytes(256, 512, 16, 8, 0) == 0         # l < r
+    assert lib.qlora_lq_workspace_bytes(256, 512, 16, 98, 0) == 0        # l > 96
+    assert lib.qlora_lq_workspace_bytes(256, 512, 16, 24, 5) == 0        # unknown dq
+    w = q.Nf4WeightC(256, 512, FAKE, FAKE, FAKE, 0, 0)
+    big = 1 << 40
+
+    def dec(W=FAKE, Q=w, L1=FAKE, L2=FAKE, r=16, Om=FAKE, l=24, power=2, iters=2, err=FAKE, ws=FAKE, wsb=big):
+        return lib.qlora_lq_decompose(W, ctypes.byref(Q), L1, L2, r, Om, l, power, iters, err, ws, wsb, None)
+    assert dec(W=None) == 1
+    assert dec(err=None) == 1
+    assert dec(l=23) == 1                      # odd test-matrix width
+    assert dec(l=8) == 1                       # l < r
+    assert dec(iters=0) == 1
+    assert dec(power=-1) == 1
+    assert dec(Q=q.Nf4WeightC(20, 512, FAKE, FAKE, FAKE, 0, 0)) == 2      # fewer rows than l
+    assert dec(wsb=1024) == 7
+    assert dec(W=MIS) == 3
+    assert dec(Om=MIS) == 3
+    assert lib.qlora_lq_lowrank(FAKE, 256, 512, ctypes.byref(q.Nf4WeightC(256, 256, FAKE, FAKE, FAKE, 0, 0)),
+                                FAKE, 24, 2, 16, FAKE, FAKE, FAKE, big, None) == 1       # shape mismatch
+    assert lib.qlora_lq_lowrank(FAKE, 10, 512, None, FAKE, 24, 2, 16, FAKE, FAKE, FAKE, big, None) == 2
+    assert lib.qlora_lq_quantize_residual(FAKE, None, FAKE, 16, ctypes.byref(w), FAKE, big, None) == 1
+    assert lib.qlora_lq_quantize_residual(FAKE, FAKE, FAKE, 16, ctypes.byref(w), FAKE, 64, None) == 7
