@@ -253,6 +253,7 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     extras["decoder_layer"] = measure_layer(q, dev, pk, barrier)
     extras["dq_signed"] = measure_dq_signed(q, dev, pk, barrier)
     extras["lq_decompose"] = measure_lq(q, dev, pk, barrier)
+    extras["dense_base"] = measure_dense(q, rep, dev, pk, barrier)
     e2e = measure_e2e(q, rep, dev, min(args.steps, 20), barrier, allmax, world)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -451,6 +452,61 @@ def measure_lq(q, dev, pk, barrier):
                          "after_rank_r_step": [round(x, 5) for x in e[:, 1]]},
            "workload": "lq_decompose_4096x4096_planted_rank64_r64_l72_power2_iters2"}
     del W, Om, ws, w, L1, L2, plain
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_dense(q, rep, dev, pk, barrier):
+    """The LLaMA-7B projection step (M = 4096, r = 64, fwd + bwd) on dense bf16 base weights (the
+    call a weight from any quantizer takes): once with W' already materialized, once re-materializing
+    it in every pass through qlora_linear_*_materialized with the library's dequantizer as the
+    black box."""
+    import ctypes
+    lib = q.load()
+    dense = [q.dequantize(c["w"]) for c in rep.cases]
+    scratch = [torch.empty_like(W) for W in dense]
+    wsf = [torch.empty(lib.qlora_workspace_bytes(q.QLORA_OP_FWD_DENSE, c["case"].M, c["case"].N, c["case"].K,
+                                                 c["case"].r), dtype=torch.uint8, device=dev) for c in rep.cases]
+    wsb = [torch.empty(lib.qlora_workspace_bytes(q.QLORA_OP_BWD_DENSE, c["case"].M, c["case"].N, c["case"].K,
+                                                 c["case"].r), dtype=torch.uint8, device=dev) for c in rep.cases]
+    st = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)   # noqa: E731
+    P = lambda t: ctypes.c_void_p(t.data_ptr())                              # noqa: E731
+    structs = [c["w"].c_struct() for c in rep.cases]
+
+    def mat(ctx, w_out, n, k, stream):
+        i = int(ctx)
+        return lib.qlora_dequantize(ctypes.byref(structs[i]), ctypes.c_void_p(w_out), ctypes.c_void_p(stream))
+    fn = q.MATERIALIZE_FN(mat)
+
+    def step(materialize):
+        for i, c in enumerate(rep.cases):
+            M, N, K, r = c["case"].M, c["case"].N, c["case"].K, c["case"].r
+            if materialize:
+                q._check(lib.qlora_linear_fwd_materialized(fn, ctypes.c_void_p(i), P(scratch[i]), N, K, P(c["X"]), M,
+                                                           P(c["A"]), P(c["B"]), r, c["s"], P(c["Y"]), P(c["H"]),
+                                                           P(wsf[i]), wsf[i].numel(), st()), "fwd_materialized")
+                q._check(lib.qlora_linear_bwd_materialized(fn, ctypes.c_void_p(i), P(scratch[i]), N, K, P(c["X"]),
+                                                           P(c["dY"]), M, P(c["A"]), P(c["B"]), r, c["s"], P(c["H"]),
+                                                           P(c["dX"]), P(c["dA"]), P(c["dB"]), P(wsb[i]),
+                                                           wsb[i].numel(), st()), "bwd_materialized")
+            else:
+                q._check(lib.qlora_linear_fwd_dense(P(dense[i]), N, K, P(c["X"]), M, P(c["A"]), P(c["B"]), r, c["s"],
+                                                    P(c["Y"]), P(c["H"]), P(wsf[i]), wsf[i].numel(), st()),
+                         "fwd_dense")
+                q._check(lib.qlora_linear_bwd_dense(P(dense[i]), N, K, P(c["X"]), P(c["dY"]), M, P(c["A"]),
+                                                    P(c["B"]), r, c["s"], P(c["H"]), P(c["dX"]), P(c["dA"]),
+                                                    P(c["dB"]), P(wsb[i]), wsb[i].numel(), st()), "bwd_dense")
+    out = {}
+    for name, m in (("dense_weight", False), ("materialized_each_pass", True)):
+        for _ in range(3):
+            step(m)
+        torch.cuda.synchronize()
+        ms = timed(lambda: step(m), 20, barrier) / 20
+        out[name] = {"ms_per_step": round(ms, 4), "value": round(rep.flops() / (ms * 1e-3) / 1e12, 1),
+                     "unit": "TFLOP/s"}
+    assert q.device_status() == 0
+    out["workload"] = "llama7b_projections_m4096_r64_fwd_bwd_dense_bf16_base"
+    del dense, scratch, wsf, wsb
     torch.cuda.empty_cache()
     return out
 

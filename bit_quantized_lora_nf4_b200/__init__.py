@@ -21,6 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libqlora.so")
 
 QLORA_OP_FWD = 0
 QLORA_OP_BWD = 1
+QLORA_OP_FWD_DENSE = 2      # the linear on a dense bf16 base weight (any quantizer's output)
+QLORA_OP_BWD_DENSE = 3
 
 STATUS_NAMES = {
     0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED_SHAPE", 3: "QLORA_ERR_MISALIGNED",
@@ -34,7 +36,8 @@ EXPORTS = (
     "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
     "qlora_profile_read", "qlora_linear_fwd_noalloc", "qlora_format_codebook", "qlora_group_scale_bytes_dq",
     "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_ws", "qlora_lq_workspace_bytes", "qlora_lq_decompose",
-    "qlora_lq_quantize_residual", "qlora_lq_lowrank",
+    "qlora_lq_quantize_residual", "qlora_lq_lowrank", "qlora_linear_fwd_dense", "qlora_linear_bwd_dense",
+    "qlora_linear_fwd_materialized", "qlora_linear_bwd_materialized",
 )
 
 # 4-bit code tables (QLORA_FORMAT_*): NF4 is the method's type; FP4 (e2m1) and
@@ -63,6 +66,10 @@ class Nf4WeightC(ctypes.Structure):
 
 
 _lib = None
+
+# qlora_materialize_fn: (ctx, W_out, N, K, stream) -> status
+MATERIALIZE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                  ctypes.c_void_p)
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -100,6 +107,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_lq_decompose": (i32, [vp, wp, vp, vp, i32, vp, i32, i32, i32, vp, vp, sz, vp]),
         "qlora_lq_quantize_residual": (i32, [vp, vp, vp, i32, wp, vp, sz, vp]),
         "qlora_lq_lowrank": (i32, [vp, i64, i64, wp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
+        "qlora_linear_fwd_dense": (i32, [vp, i64, i64, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_linear_bwd_dense": (i32, [vp, i64, i64, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
+        "qlora_linear_fwd_materialized": (i32, [MATERIALIZE_FN, vp, vp, i64, i64, vp, i64, vp, vp, i32, f32, vp, vp,
+                                                vp, sz, vp]),
+        "qlora_linear_bwd_materialized": (i32, [MATERIALIZE_FN, vp, vp, i64, i64, vp, vp, i64, vp, vp, i32, f32, vp,
+                                                vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -297,6 +310,58 @@ def linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, 
     st = w.c_struct()
     _check(lib.qlora_linear_fwd(ctypes.byref(st), _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(Y), _ptr(H), _ptr(ws),
                                 ws.numel(), _stream()), "qlora_linear_fwd")
+    return Y, H
+
+
+def linear_fwd_dense(W: torch.Tensor, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float,
+                     save_h: bool = True):
+    """The forward on a dense bf16 base W [N, K] from any quantizer (qlora_linear_fwd_dense)."""
+    lib = load()
+    N, K = W.shape
+    M, r = X.shape[0], A.shape[0]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    H = torch.empty((M, r), dtype=torch.float32, device=X.device) if save_h else None
+    ws = torch.empty(lib.qlora_workspace_bytes(QLORA_OP_FWD_DENSE, M, N, K, r), dtype=torch.uint8, device=X.device)
+    _check(lib.qlora_linear_fwd_dense(_ptr(W), N, K, _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(Y), _ptr(H), _ptr(ws),
+                                      ws.numel(), _stream()), "qlora_linear_fwd_dense")
+    return Y, H
+
+
+def linear_bwd_dense(W: torch.Tensor, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor, s: float,
+                     H: torch.Tensor | None = None):
+    """The backward on a dense bf16 base W [N, K] (qlora_linear_bwd_dense): (dX, dA, dB)."""
+    lib = load()
+    N, K = W.shape
+    M, r = X.shape[0], A.shape[0]
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=X.device)
+    dA = torch.empty((r, K), dtype=torch.float32, device=X.device)
+    dB = torch.empty((N, r), dtype=torch.float32, device=X.device)
+    ws = torch.empty(lib.qlora_workspace_bytes(QLORA_OP_BWD_DENSE, M, N, K, r), dtype=torch.uint8, device=X.device)
+    _check(lib.qlora_linear_bwd_dense(_ptr(W), N, K, _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B), r, s, _ptr(H), _ptr(dX),
+                                      _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream()), "qlora_linear_bwd_dense")
+    return dX, dA, dB
+
+
+def linear_fwd_materialized(materialize, N: int, K: int, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                            s: float, save_h: bool = True):
+    """The forward with the base produced by `materialize(W_out)` (a callable that fills a bf16 CUDA
+    tensor [N, K] on the current stream) through qlora_linear_fwd_materialized."""
+    lib = load()
+    M, r = X.shape[0], A.shape[0]
+    scratch = torch.empty((N, K), dtype=torch.bfloat16, device=X.device)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    H = torch.empty((M, r), dtype=torch.float32, device=X.device) if save_h else None
+    ws = torch.empty(lib.qlora_workspace_bytes(QLORA_OP_FWD_DENSE, M, N, K, r), dtype=torch.uint8, device=X.device)
+
+    def cb(ctx, w_out, n, k, stream):
+        if w_out != scratch.data_ptr() or (n, k) != (N, K):
+            return 1
+        materialize(scratch)
+        return 0
+    fn = MATERIALIZE_FN(cb)
+    _check(lib.qlora_linear_fwd_materialized(fn, None, _ptr(scratch), N, K, _ptr(X), M, _ptr(A), _ptr(B), r, s,
+                                             _ptr(Y), _ptr(H), _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_fwd_materialized")
     return Y, H
 
 

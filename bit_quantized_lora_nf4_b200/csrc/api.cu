@@ -221,7 +221,7 @@ struct Plan {
   bool gemv = false;
 };
 
-Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r) {
+Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, bool allow_gemv = true) {
   Plan p;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -230,7 +230,7 @@ Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r) {
     return o;
   };
   const size_t Mr = static_cast<size_t>(M) * r;
-  if (op == QLORA_OP_FWD && M <= kGemvMaxTokens && gemv_enabled()) {
+  if (op == QLORA_OP_FWD && allow_gemv && M <= kGemvMaxTokens && gemv_enabled()) {
     p.gemv = true;
     p.part = take(gemv_workspace_bytes(M, N, K, r));
     p.total = off;
@@ -274,17 +274,54 @@ qlora_status check_weight(const qlora_nf4_weight *w) {
 }
 
 // Shape, pointer and alignment checks shared by the linear calls (no workspace).
+qlora_status check_linear_shape(int64_t N, int64_t K, int64_t M, int r, float s, const void *X, const void *A,
+                                const void *B, const void *out) {
+  if (!X || !A || !B || !out) return QLORA_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || M < 1 || r < 8 || r > 256 || !std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (r % 8 != 0 || K % 64 != 0 || N % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1)
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(out)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
 qlora_status check_linear(const qlora_nf4_weight *w, int64_t M, int r, float s, const void *X, const void *A,
                           const void *B, const void *out) {
   qlora_status st = check_weight(w);
   if (st != QLORA_OK) return st;
-  if (!X || !A || !B || !out) return QLORA_ERR_INVALID_ARG;
-  if (M < 1 || r < 8 || r > 256 || !std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
-  if (r % 8 != 0 || w->cols % 64 != 0 || w->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (M > (int64_t(1) << 31) - 1 || w->rows > (int64_t(1) << 31) - 1 || w->cols > (int64_t(1) << 31) - 1)
-    return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(out)) return QLORA_ERR_MISALIGNED;
-  return QLORA_OK;
+  return check_linear_shape(w->rows, w->cols, M, r, s, X, A, B, out);
+}
+
+// Where the fused GEMMs take the base weight from: a packed NF4 weight, or a
+// dense bf16 W' [N, K] the caller materialized (any quantizer's output).
+struct WeightSrc {
+  const qlora_nf4_weight *w;
+  const uint16_t *dense;
+  int64_t N, K;
+};
+
+QGemmArgs gemm_args(const WeightSrc &src, bool dgrad, int64_t M, const uint16_t *act, const uint16_t *lora_act,
+                    const uint16_t *lora_w, int r, uint16_t *out) {
+  QGemmArgs g{};
+  g.dgrad = dgrad;
+  g.M = M;
+  g.wN = src.N;
+  g.wK = src.K;
+  g.act = act;
+  g.lora_act = lora_act;
+  g.lora_w = lora_w;
+  g.r = r;
+  g.out = out;
+  if (src.w) {
+    g.codes = src.w->codes;
+    g.absmax_q = src.w->absmax_q;
+    g.group_scale = src.w->group_scale;
+    g.tab = weight_table(src.w);
+  } else {
+    g.tab = format_table(QLORA_FORMAT_NF4);
+    g.wdense = src.dense;
+  }
+  return g;
 }
 
 qlora_status check_ws(const void *ws, size_t ws_bytes, size_t need) {
@@ -431,8 +468,10 @@ qlora_status qlora_device_status(void *stream) {
 }
 
 size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
-  if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || M < 1 || N < 1 || K < 1 || r < 1) return 0;
-  return make_plan(op, M, N, K, r).total;
+  if (op < QLORA_OP_FWD || op > QLORA_OP_BWD_DENSE || M < 1 || N < 1 || K < 1 || r < 1) return 0;
+  const bool dense = op == QLORA_OP_FWD_DENSE || op == QLORA_OP_BWD_DENSE;
+  const int base = dense ? op - QLORA_OP_FWD_DENSE : op;
+  return make_plan(base, M, N, K, r, !dense).total;
 }
 
 qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
@@ -466,34 +505,33 @@ qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *
   return QLORA_OK;
 }
 
-qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
-                              const uint16_t *B, int r, float s, uint16_t *Y, float *H_out, void *ws,
-                              size_t ws_bytes, void *stream) {
-  if (!w) return QLORA_ERR_INVALID_ARG;
-  QL_TRY(check_linear(w, M, r, s, X, A, B, Y));
-  const int64_t N = w->rows, K = w->cols;
-  const Plan p = make_plan(QLORA_OP_FWD, M, N, K, r);
+}  // extern "C"
+
+namespace {
+
+qlora_status linear_fwd_impl(const WeightSrc &src, const uint16_t *X, int64_t M, const uint16_t *A,
+                             const uint16_t *B, int r, float s, uint16_t *Y, float *H_out, void *ws, size_t ws_bytes,
+                             void *stream) {
+  const int64_t N = src.N, K = src.K;
+  const Plan p = make_plan(QLORA_OP_FWD, M, N, K, r, src.w != nullptr);
   QL_TRY(check_ws(ws, ws_bytes, p.total));
   if (H_out && !aligned16(H_out)) return QLORA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *H = H_out ? H_out : at<float>(ws, p.H);
   if (p.gemv) {
+    const qlora_nf4_weight *w = src.w;
     GemvArgs g{M, N, K, X, w->codes, w->absmax_q, w->group_scale, A, B, r, s, Y, H_out, at<void>(ws, p.part),
                weight_table(w)};
     return launch_gemv(g, st);
   }
   QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
-  QGemmArgs g{false, M, N, K, X, w->codes, w->absmax_q, w->group_scale, at<uint16_t>(ws, p.sH), B, r, Y,
-              weight_table(w)};
-  return launch_qgemm(g, st);
+  return launch_qgemm(gemm_args(src, false, M, X, at<uint16_t>(ws, p.sH), B, r, Y), st);
 }
 
-qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
-                              const uint16_t *A, const uint16_t *B, int r, float s, const float *H_saved,
-                              uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream) {
-  if (!w || !dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-  QL_TRY(check_linear(w, M, r, s, X, A, B, dX));
-  const int64_t N = w->rows, K = w->cols;
+qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint16_t *dY, int64_t M,
+                             const uint16_t *A, const uint16_t *B, int r, float s, const float *H_saved,
+                             uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream) {
+  const int64_t N = src.N, K = src.K;
   const Plan p = make_plan(QLORA_OP_BWD, M, N, K, r);
   QL_TRY(check_ws(ws, ws_bytes, p.total));
   if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_MISALIGNED;
@@ -564,8 +602,73 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
     }
   }
   // dX = dY W' + Gb A
-  QGemmArgs g{true, M, N, K, dY, w->codes, w->absmax_q, w->group_scale, Gb, A, r, dX, weight_table(w)};
-  return launch_qgemm(g, st);
+  return launch_qgemm(gemm_args(src, true, M, dY, Gb, A, r, dX), st);
+}
+
+}  // namespace
+
+extern "C" {
+
+qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t M, const uint16_t *A,
+                              const uint16_t *B, int r, float s, uint16_t *Y, float *H_out, void *ws,
+                              size_t ws_bytes, void *stream) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear(w, M, r, s, X, A, B, Y));
+  return linear_fwd_impl(WeightSrc{w, nullptr, w->rows, w->cols}, X, M, A, B, r, s, Y, H_out, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t M,
+                              const uint16_t *A, const uint16_t *B, int r, float s, const float *H_saved,
+                              uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream) {
+  if (!w || !dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear(w, M, r, s, X, A, B, dX));
+  return linear_bwd_impl(WeightSrc{w, nullptr, w->rows, w->cols}, X, dY, M, A, B, r, s, H_saved, dX, dA, dB, ws,
+                         ws_bytes, stream);
+}
+
+qlora_status qlora_linear_fwd_dense(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X, int64_t M,
+                                    const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y, float *H_out,
+                                    void *ws, size_t ws_bytes, void *stream) {
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear_shape(N, K, M, r, s, X, A, B, Y));
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  return linear_fwd_impl(WeightSrc{nullptr, W, N, K}, X, M, A, B, r, s, Y, H_out, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_dense(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X, const uint16_t *dY,
+                                    int64_t M, const uint16_t *A, const uint16_t *B, int r, float s,
+                                    const float *H_saved, uint16_t *dX, float *dA, float *dB, void *ws,
+                                    size_t ws_bytes, void *stream) {
+  if (!W || !dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear_shape(N, K, M, r, s, X, A, B, dX));
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  return linear_bwd_impl(WeightSrc{nullptr, W, N, K}, X, dY, M, A, B, r, s, H_saved, dX, dA, dB, ws, ws_bytes,
+                         stream);
+}
+
+qlora_status qlora_linear_fwd_materialized(qlora_materialize_fn materialize, void *ctx, uint16_t *W_scratch,
+                                           int64_t N, int64_t K, const uint16_t *X, int64_t M, const uint16_t *A,
+                                           const uint16_t *B, int r, float s, uint16_t *Y, float *H_out, void *ws,
+                                           size_t ws_bytes, void *stream) {
+  if (!materialize || !W_scratch) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear_shape(N, K, M, r, s, X, A, B, Y));
+  if (!aligned16(W_scratch)) return QLORA_ERR_MISALIGNED;
+  QL_TRY(check_ws(ws, ws_bytes, make_plan(QLORA_OP_FWD, M, N, K, r, false).total));
+  QL_TRY(materialize(ctx, W_scratch, N, K, stream));
+  return qlora_linear_fwd_dense(W_scratch, N, K, X, M, A, B, r, s, Y, H_out, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_materialized(qlora_materialize_fn materialize, void *ctx, uint16_t *W_scratch,
+                                           int64_t N, int64_t K, const uint16_t *X, const uint16_t *dY, int64_t M,
+                                           const uint16_t *A, const uint16_t *B, int r, float s,
+                                           const float *H_saved, uint16_t *dX, float *dA, float *dB, void *ws,
+                                           size_t ws_bytes, void *stream) {
+  if (!materialize || !W_scratch || !dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  QL_TRY(check_linear_shape(N, K, M, r, s, X, A, B, dX));
+  if (!aligned16(W_scratch)) return QLORA_ERR_MISALIGNED;
+  QL_TRY(check_ws(ws, ws_bytes, make_plan(QLORA_OP_BWD, M, N, K, r).total));
+  QL_TRY(materialize(ctx, W_scratch, N, K, stream));
+  return qlora_linear_bwd_dense(W_scratch, N, K, X, dY, M, A, B, r, s, H_saved, dX, dA, dB, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

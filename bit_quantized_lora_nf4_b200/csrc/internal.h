@@ -68,6 +68,7 @@ struct QGemmArgs {
   int r;
   uint16_t *out;
   Nf4Table tab;        // weight_table() of the weight
+  const uint16_t *wdense = nullptr;   // dense bf16 W' [wN, wK] instead of the packed weight (pair kernel only)
 };
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
 // The same product on a CTA pair (256-row tiles); launch_qgemm dispatches to it for M > 128.

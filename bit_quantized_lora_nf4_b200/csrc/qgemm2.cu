@@ -86,6 +86,7 @@ struct Params {
   const uint8_t *absmax_q;
   const float *group_scale;
   const uint16_t *lora_w;
+  const uint16_t *wdense;   // DENSE: the bf16 weight [wN, wK]
   int r;
   int nkb;           // weight K-steps (of 128)
   int nls;           // adapter K-steps (of 128)
@@ -132,7 +133,12 @@ struct BlockLoad {
   float S;
 };
 
-template <bool DGRAD, int NACC>
+// One weight run of a DENSE operand row: 8 x 16 bytes of bf16 W'.
+struct DenseLoad {
+  uint4 v[8];
+};
+
+template <bool DGRAD, int NACC, bool DENSE>
 __global__ void __launch_bounds__(THREADS, 1)
     qgemm2_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lact,
                   const Params p, const Nf4Table tab) {
@@ -299,22 +305,59 @@ __global__ void __launch_bounds__(THREADS, 1)
         b.S = __ldg(p.group_scale + (idx >> 8));
       }
     };
-    const float mu = dq_offset(tab);
-    BlockLoad bq[PREFETCH];                   // this group's next PREFETCH K-steps
+    // DENSE: the operand row's 64 weights of this thread's run, 8 x 16 bytes
+    // (zero past the matrix), loaded one of the group's K-steps ahead.
+    auto fetch_dense = [&](int i, DenseLoad &d) {
 #pragma unroll
-    for (int j = 0; j < PREFETCH; ++j) fetch(grp + j * NACC, bq[j]);
+      for (int c = 0; c < 8; ++c) d.v[c] = make_uint4(0, 0, 0, 0);
+      if (i >= p.nkb) return;
+      int64_t n, k;
+      if (DGRAD) {
+        n = static_cast<int64_t>(i) * BK + row;
+        k = nb0 + 64 * jb;
+      } else {
+        n = nb0 + row;
+        k = static_cast<int64_t>(i) * BK + 64 * jb;
+      }
+      if (n < p.wN && k < p.wK) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.wdense + n * p.wK + k);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) d.v[c] = __ldg(src + c);
+      }
+    };
+    const float mu = DENSE ? 0.0f : dq_offset(tab);
+    BlockLoad bq[DENSE ? 1 : PREFETCH];       // this group's next PREFETCH K-steps
+    DenseLoad dnext;
+    if (DENSE) {
+      fetch_dense(grp, dnext);
+    } else {
+#pragma unroll
+      for (int j = 0; j < PREFETCH; ++j) fetch(grp + j * NACC, bq[j]);
+    }
     const uint32_t swz = row & 7;             // 128B swizzle of the operand
     for (int i = grp; i < nsteps; i += NACC) {
       const int sd = i % D_STAGES;
-      const BlockLoad cur = bq[0];
+      BlockLoad cur{};
+      DenseLoad dcur;
+      if (DENSE) {
+        dcur = dnext;
+        fetch_dense(i + NACC, dnext);
+      } else {
+        cur = bq[0];
 #pragma unroll
-      for (int j = 0; j + 1 < PREFETCH; ++j) bq[j] = bq[j + 1];
-      fetch(i + PREFETCH * NACC, bq[PREFETCH - 1]);
+        for (int j = 0; j + 1 < (DENSE ? 1 : PREFETCH); ++j) bq[j] = bq[j + 1];
+        fetch(i + PREFETCH * NACC, bq[(DENSE ? 1 : PREFETCH) - 1]);
+      }
       if (i >= D_STAGES &&
           !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
         break;
       const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
-      if (i < p.nkb) {
+      if (DENSE && i < p.nkb) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), dcur.v[c].x, dcur.v[c].y, dcur.v[c].z,
+                       dcur.v[c].w);
+      } else if (i < p.nkb) {
         const float ap = block_constant(cur.q, cur.S, tab.qx, mu);
         uint32_t LO[4], HI[4];
         nf4_block_table(ap, tab, LO, HI);
@@ -414,6 +457,7 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   p.absmax_q = a.absmax_q;
   p.group_scale = a.group_scale;
   p.lora_w = a.lora_w;
+  p.wdense = a.wdense;
   p.r = a.r;
   p.out = a.out;
   p.status = device_status_ptr();
@@ -450,10 +494,16 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
     return e;
   };
   cudaError_t e;
-  if (a.dgrad)
-    e = nacc == 2 ? go(qgemm2_kernel<true, 2>) : go(qgemm2_kernel<true, 1>);
-  else
-    e = nacc == 2 ? go(qgemm2_kernel<false, 2>) : go(qgemm2_kernel<false, 1>);
+  if (a.wdense) {
+    if (a.dgrad)
+      e = nacc == 2 ? go(qgemm2_kernel<true, 2, true>) : go(qgemm2_kernel<true, 1, true>);
+    else
+      e = nacc == 2 ? go(qgemm2_kernel<false, 2, true>) : go(qgemm2_kernel<false, 1, true>);
+  } else if (a.dgrad) {
+    e = nacc == 2 ? go(qgemm2_kernel<true, 2, false>) : go(qgemm2_kernel<true, 1, false>);
+  } else {
+    e = nacc == 2 ? go(qgemm2_kernel<false, 2, false>) : go(qgemm2_kernel<false, 1, false>);
+  }
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

@@ -151,9 +151,12 @@ qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, 
  * Bit-exact by construction. */
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream);
 
-/* Operation ids for qlora_workspace_bytes(). */
+/* Operation ids for qlora_workspace_bytes(): the linear on a packed weight,
+ * and on a dense bf16 weight (qlora_linear_*_dense / _materialized). */
 #define QLORA_OP_FWD 0
 #define QLORA_OP_BWD 1
+#define QLORA_OP_FWD_DENSE 2
+#define QLORA_OP_BWD_DENSE 3
 
 /* Workspace bytes the linear calls need for the given sizes (0 never means
  * "no workspace" for the linear; it is at least 256). */
@@ -189,6 +192,42 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
                               int64_t M, const uint16_t *A, const uint16_t *B, int r, float s,
                               const float *H_saved, uint16_t *dX, float *dA, float *dB,
                               void *ws, size_t ws_bytes, void *stream);
+
+/* ---- Linear on a base weight from any quantizer ----------------------------
+ * ("ModuLoRA", abstract: a quantization-agnostic backward that materializes the
+ * low-precision weights of a black-box quantization module in each pass.)
+ * The base W' arrives as a dense bf16 matrix [N, K] (device, row-major) that
+ * the caller's dequantizer produced; the same fused tensor-core GEMM, adapter
+ * products and precision rules as qlora_linear_fwd / qlora_linear_bwd apply
+ * (the operand is copied into the GEMM's shared-memory ring instead of being
+ * decoded; the pair kernel serves every M).  With W' = qlora_dequantize(w) the
+ * results equal the packed calls' bit for bit whenever those take the pair
+ * kernel (M > 128).  Workspace: qlora_workspace_bytes(QLORA_OP_FWD_DENSE /
+ * QLORA_OP_BWD_DENSE, M, N, K, r).  Shape rules as for the packed calls. */
+qlora_status qlora_linear_fwd_dense(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X, int64_t M,
+                                    const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y, float *H_out,
+                                    void *ws, size_t ws_bytes, void *stream);
+qlora_status qlora_linear_bwd_dense(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X, const uint16_t *dY,
+                                    int64_t M, const uint16_t *A, const uint16_t *B, int r, float s,
+                                    const float *H_saved, uint16_t *dX, float *dA, float *dB, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/* The black-box boundary itself: `materialize(ctx, W_out, N, K, stream)`
+ * enqueues, on `stream`, whatever writes the bf16 base weight [N, K] into the
+ * device buffer W_out and returns QLORA_OK (any other status aborts the call
+ * and is returned).  The _materialized calls run it into the caller's scratch
+ * buffer W_scratch (2 N K bytes, 16-byte aligned) and then the dense linear, so
+ * the full-precision weight exists only for the duration of one pass. */
+typedef qlora_status (*qlora_materialize_fn)(void *ctx, uint16_t *W_out, int64_t N, int64_t K, void *stream);
+qlora_status qlora_linear_fwd_materialized(qlora_materialize_fn materialize, void *ctx, uint16_t *W_scratch,
+                                           int64_t N, int64_t K, const uint16_t *X, int64_t M, const uint16_t *A,
+                                           const uint16_t *B, int r, float s, uint16_t *Y, float *H_out, void *ws,
+                                           size_t ws_bytes, void *stream);
+qlora_status qlora_linear_bwd_materialized(qlora_materialize_fn materialize, void *ctx, uint16_t *W_scratch,
+                                           int64_t N, int64_t K, const uint16_t *X, const uint16_t *dY, int64_t M,
+                                           const uint16_t *A, const uint16_t *B, int r, float s,
+                                           const float *H_saved, uint16_t *dX, float *dA, float *dB, void *ws,
+                                           size_t ws_bytes, void *stream);
 
 /* Size of the library-owned scratch array used by qlora_linear_fwd_noalloc(). */
 #define QLORA_STATIC_SCRATCH_BYTES (8u << 20)

@@ -18,6 +18,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "ql
 def _declared():
     txt = open(HEADER).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    txt = re.sub(r"typedef[^;]*;", "", txt)         # function-pointer types are not exports
     return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", txt)))
 
 
@@ -164,3 +165,30 @@ def test_lq_sizes_and_argument_errors():
     assert lib.qlora_lq_lowrank(FAKE, 10, 512, None, FAKE, 24, 2, 16, FAKE, FAKE, FAKE, big, None) == 2
     assert lib.qlora_lq_quantize_residual(FAKE, None, FAKE, 16, ctypes.byref(w), FAKE, big, None) == 1
     assert lib.qlora_lq_quantize_residual(FAKE, FAKE, FAKE, 16, ctypes.byref(w), FAKE, 64, None) == 7
+
+
+def test_dense_linear_sizes_and_argument_errors():
+    lib = q.load()
+    for op in (q.QLORA_OP_FWD_DENSE, q.QLORA_OP_BWD_DENSE):
+        assert lib.qlora_workspace_bytes(op, 4, 512, 512, 16) >= 256
+    assert lib.qlora_workspace_bytes(4, 4, 512, 512, 16) == 0
+    big = 1 << 40
+    f = lib.qlora_linear_fwd_dense
+    assert f(None, 256, 256, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, big, None) == 1
+    assert f(FAKE, 256, 200, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, big, None) == 2     # K % 64
+    assert f(MIS, 256, 256, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, big, None) == 3
+    assert f(FAKE, 256, 256, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, 16, None) == 7
+    b = lib.qlora_linear_bwd_dense
+    assert b(FAKE, 256, 256, FAKE, None, 64, FAKE, FAKE, 16, 1.0, None, FAKE, FAKE, FAKE, FAKE, big, None) == 1
+    calls = []
+
+    def cb(ctx, w_out, n, k, stream):
+        calls.append((n, k))
+        return 0
+    fn = q.MATERIALIZE_FN(cb)
+    m = lib.qlora_linear_fwd_materialized
+    assert m(fn, None, FAKE, 256, 200, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, big, None) == 2
+    assert m(fn, None, FAKE, 256, 256, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, 16, None) == 7
+    assert calls == []          # argument errors are found before the weight is materialized
+    bad = q.MATERIALIZE_FN(lambda ctx, w_out, n, k, stream: 4)
+    assert m(bad, None, FAKE, 256, 256, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, big, None) == 4
