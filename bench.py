@@ -474,7 +474,7 @@ def measure_dense(q, rep, dev, pk, barrier):
     structs = [c["w"].c_struct() for c in rep.cases]
 
     def mat(ctx, w_out, n, k, stream):
-        i = int(ctx)
+        i = ctx or 0          # ctypes hands a NULL context (case 0) over as None
         return lib.qlora_dequantize(ctypes.byref(structs[i]), ctypes.c_void_p(w_out), ctypes.c_void_p(stream))
     fn = q.MATERIALIZE_FN(mat)
 
