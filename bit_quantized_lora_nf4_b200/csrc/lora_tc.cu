@@ -85,6 +85,8 @@ __device__ __forceinline__ uint16_t t_bf16(float x) {
 }
 __device__ __forceinline__ float t_bf16_val(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
 
+constexpr int kMaxZ = 8;   // most slices of one tile (the portable cluster size)
+
 // After every slice of the tile is staged: CTA z of the Z in the cluster adds
 // its share of the rows over all Z staged tiles in slice order (distributed
 // shared memory) and writes the epilogue's outputs; a second cluster barrier
@@ -105,21 +107,46 @@ __device__ __forceinline__ void cluster_finish(const TParams &p, float *stage, i
   const int tcols = kind == kSkinnyCols ? half_j : static_cast<int>(J - j0 < p.bn ? J - j0 : p.bn);
   const int per = (trows + Z - 1) / Z;
   const int rbeg = z * per, rend = rbeg + per < trows ? rbeg + per : trows;
-  const int n = rend > rbeg ? (rend - rbeg) * tcols : 0;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const int row = rbeg + e / tcols, col = e - (e / tcols) * tcols;
-    const int64_t gi = i0 + row, gj = j0 + col;
+  // four consecutive columns per item: every slice's values are fetched with
+  // independent 16-byte loads before they are added (one round trip through
+  // distributed shared memory instead of one per slice)
+  const int tc4 = tcols / 4;   // tcols % 4 == 0 for every kind (J, r multiples of 4)
+  const int n4 = rend > rbeg ? (rend - rbeg) * tc4 : 0;
+  const bool paired = kind == kSkinnyCols || kind == kSkinnyRows;
+  const int off2 = kind == kSkinnyCols ? half_j : half_i * pitch;   // the second half's offset
+  for (int e4 = threadIdx.x; e4 < n4; e4 += blockDim.x) {
+    const int row = rbeg + e4 / tc4, col0 = (e4 - (e4 / tc4) * tc4) * 4;
+    const int64_t gi = i0 + row;
     if (kind != kSkinnyRows && gi >= p.I) continue;
-    float v = 0.0f;
-    for (int q = 0; q < Z; ++q) {   // slice order: fixed, so the result is deterministic
-      const float *t = cl.map_shared_rank(stage, q);
-      if (kind == kSkinnyCols)
-        v = __fadd_rn(v, __fadd_rn(t[row * pitch + col], t[row * pitch + col + half_j]));
-      else if (kind == kSkinnyRows)
-        v = __fadd_rn(v, __fadd_rn(t[row * pitch + col], t[(row + half_i) * pitch + col]));
-      else
-        v = __fadd_rn(v, t[row * pitch + col]);
+    float4 a[kMaxZ], b[kMaxZ];
+#pragma unroll
+    for (int q = 0; q < kMaxZ; ++q) {
+      if (q < Z) {
+        const float *t = cl.map_shared_rank(stage, q) + row * pitch + col0;
+        a[q] = *reinterpret_cast<const float4 *>(t);
+        if (paired) b[q] = *reinterpret_cast<const float4 *>(t + off2);
+      }
     }
+    float v4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int q = 0; q < kMaxZ; ++q) {   // slice order: fixed, so the result is deterministic
+      if (q < Z) {
+        const float av[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
+        if (paired) {
+          const float bv[4] = {b[q].x, b[q].y, b[q].z, b[q].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v4[c] = __fadd_rn(v4[c], __fadd_rn(av[c], bv[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v4[c] = __fadd_rn(v4[c], av[c]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+    const int col = col0 + c;
+    const int64_t gj = j0 + col;
+    const float v = v4[c];
     if (kind == kSkinnyH) {
       const int64_t idx = gi * J + gj;
       ep.out_f[idx] = v;
@@ -146,6 +173,7 @@ __device__ __forceinline__ void cluster_finish(const TParams &p, float *stage, i
       ep.out_f[gi * half_j + gj] = __fmul_rn(ep.s, v);
     } else {   // kSkinnyRows
       ep.out_f[static_cast<int64_t>(row) * J + gj] = v;
+    }
     }
   }
   cluster_sync_all();
@@ -305,10 +333,14 @@ __global__ void __launch_bounds__(TTHREADS, 1)
 }  // namespace
 
 namespace {
-constexpr int kMaxSkinnyCluster = 8;   // portable cluster size
+constexpr int kMaxSkinnyCluster = kMaxZ;   // portable cluster size
+// Tile width: the whole J up to 128 columns.  Wider matrices (dA, J = K) take
+// 128-column tiles: twice the tiles of 256-column ones, so more of the
+// machine at the same number of splits, and the staged tile of a cluster
+// epilogue still fits the ring.
 int64_t tc_bn(int64_t J) {
   const int64_t b = ceil_div(J, 64) * 64;
-  return b > TBN_MAX ? TBN_MAX : b;
+  return b > 128 ? 128 : b;
 }
 }  // namespace
 
@@ -334,8 +366,9 @@ bool skinny_fused_ok(const SkinnyArgs &a) {
   switch (a.ep.kind) {
     case kSkinnyH:
     case kSkinnyG:
+      return a.J <= bn && a.J % 4 == 0;           // one tile covers every column
     case kSkinnyCols:
-      return a.J <= bn && a.J % 2 == 0;           // one tile covers every column (and both halves)
+      return a.J <= bn && a.J % 8 == 0;           // ... and both halves, in runs of four
     case kSkinnyRows:
       return a.I <= TBM && a.I % 2 == 0 && a.J % 4 == 0;   // one tile covers both row halves
     default:
