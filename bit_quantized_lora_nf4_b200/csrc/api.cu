@@ -136,6 +136,36 @@ int *device_status_ptr() {
   return ptrs[dev];
 }
 
+// ----------------------------------------------------------------- side stream
+// A low-priority stream per (host thread, device) on which the backward runs
+// the dB and dA products while the dgrad GEMM occupies the main stream: the
+// GEMM's CTAs are dispatched first, the adapter products fill the SMs its
+// last, partial wave leaves idle.  Fork and join are event record / wait, so
+// the pattern is also legal inside stream capture.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SideStream *side_stream() {
+  thread_local SideStream per_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream &ss = per_dev[dev];
+  if (!ss.s) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking, lo) != cudaSuccess) {
+      ss.s = nullptr;
+      return nullptr;
+    }
+    if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+  }
+  return &ss;
+}
+
 // ----------------------------------------------------------------- kernel timing hook
 namespace {
 struct Prof {
@@ -160,6 +190,8 @@ cudaEvent_t prof_event() {
   return P.pool[P.next++];
 }
 }  // namespace
+
+bool prof_on() { return prof().on; }
 
 void prof_mark(int kind, bool begin, cudaStream_t st) {
   Prof &P = prof();
@@ -572,34 +604,44 @@ qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint
     }
   }
   if (hs_pending) QL_CUDA(launch_split_hilo(H_saved, M, r, Hs, st));
-  // dB = s dY^T H
-  {
-    SkinnyArgs a{dY, N, false, Hs, 2 * static_cast<int64_t>(r), false, N, 2 * static_cast<int64_t>(r), M, p.spB,
-                 p.kpsB, part};
-    a.ep.kind = kSkinnyCols;
-    a.ep.s = s;
-    a.ep.out_f = dB;
-    if (skinny_fused_ok(a)) {
-      QL_CUDA(launch_skinny(a, st));
-    } else {
-      a.ep = SkinnyEpilogue{};
-      QL_CUDA(launch_skinny(a, st));
-      QL_CUDA(launch_finalize_cols(part, p.spB, N, r, s, dB, st));
-    }
+  // dB = s dY^T H  and  dA = G^T X
+  SkinnyArgs aB{dY, N, false, Hs, 2 * static_cast<int64_t>(r), false, N, 2 * static_cast<int64_t>(r), M, p.spB,
+                p.kpsB, part};
+  aB.ep.kind = kSkinnyCols;
+  aB.ep.s = s;
+  aB.ep.out_f = dB;
+  SkinnyArgs aA{Gs, 2 * static_cast<int64_t>(r), false, X, K, false, 2 * static_cast<int64_t>(r), K, M, p.spA,
+                p.kpsA, part};
+  aA.ep.kind = kSkinnyRows;
+  aA.ep.out_f = dA;
+  // Both finishing in-kernel (no shared partial buffer): they run on the side
+  // stream, beside the dgrad GEMM.
+  // (Off while the timing hook records, so that every kernel's events time it alone.)
+  SideStream *side = (skinny_fused_ok(aB) && skinny_fused_ok(aA) && !prof_on()) ? side_stream() : nullptr;
+  if (side) {
+    QL_CUDA(cudaEventRecord(side->fork, st));
+    QL_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    // dX = dY W' + Gb A first, so that its CTAs are dispatched ahead of the products'
+    const qlora_status gst = launch_qgemm(gemm_args(src, true, M, dY, Gb, A, r, dX), st);
+    QL_CUDA(launch_skinny(aB, side->s));
+    QL_CUDA(launch_skinny(aA, side->s));
+    QL_CUDA(cudaEventRecord(side->join, side->s));
+    QL_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+    return gst;
   }
-  // dA = G^T X
-  {
-    SkinnyArgs a{Gs, 2 * static_cast<int64_t>(r), false, X, K, false, 2 * static_cast<int64_t>(r), K, M, p.spA,
-                 p.kpsA, part};
-    a.ep.kind = kSkinnyRows;
-    a.ep.out_f = dA;
-    if (skinny_fused_ok(a)) {
-      QL_CUDA(launch_skinny(a, st));
-    } else {
-      a.ep = SkinnyEpilogue{};
-      QL_CUDA(launch_skinny(a, st));
-      QL_CUDA(launch_finalize_rows(part, p.spA, r, K, dA, st));
-    }
+  if (skinny_fused_ok(aB)) {
+    QL_CUDA(launch_skinny(aB, st));
+  } else {
+    aB.ep = SkinnyEpilogue{};
+    QL_CUDA(launch_skinny(aB, st));
+    QL_CUDA(launch_finalize_cols(part, p.spB, N, r, s, dB, st));
+  }
+  if (skinny_fused_ok(aA)) {
+    QL_CUDA(launch_skinny(aA, st));
+  } else {
+    aA.ep = SkinnyEpilogue{};
+    QL_CUDA(launch_skinny(aA, st));
+    QL_CUDA(launch_finalize_rows(part, p.spA, r, K, dA, st));
   }
   // dX = dY W' + Gb A
   return launch_qgemm(gemm_args(src, true, M, dY, Gb, A, r, dX), st);

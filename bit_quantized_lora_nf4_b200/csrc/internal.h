@@ -37,6 +37,8 @@ enum ProfKind { kProfAll = 0, kProfGemmFwd = 1, kProfGemmDgrad = 2, kProfLora = 
                 kProfLqSmall = 11, kProfKinds = 12 };
 // Records an event before (begin=true) or after a launch of `kind` on `st` when profiling is on.
 void prof_mark(int kind, bool begin, cudaStream_t st);
+// Whether the timing hook is recording (the backward then keeps every launch on the caller's stream).
+bool prof_on();
 
 // ---- tensor maps ------------------------------------------------------------
 // 2D tiled map over a row-major [outer, inner] array.

@@ -185,6 +185,9 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int6
  *   dB = s dY^T (X A^T)         device fp32 [N, r]
  * ("QLoRA" Abstract: gradients flow through the frozen 4-bit model into the
  * adapters; "Where the memory goes": through the dequantized weights.)
+ * dB and dA run on a library-owned low-priority stream (one per host thread
+ * and device, forked from and joined back into `stream` by events, so the
+ * call stays stream-ordered and capturable) beside the dgrad GEMM.
  *   H_saved : optional device fp32 [M, r] from qlora_linear_fwd; NULL makes the
  *             call recompute X A^T.
  * Same shape rules as the forward; M >= 1. */
@@ -344,6 +347,8 @@ qlora_status qlora_selftest_wait_timeout(uint64_t cycles, void *stream);
  *   residual products R M and R^T Y, 8 the low-rank residual and error
  *   kernel, 9 Cholesky and triangular inverse, 10 Jacobi eigen-decomposition,
  *   11 Gram, small-factor and split-sum kernels.
+ * While recording, the backward keeps every launch on the caller's stream
+ * (no side stream), so each event pair times its kernel alone.
  * qlora_profile_enable(1) clears the records; qlora_profile_read()
  * synchronizes the device and returns the summed event time (ms) and the
  * launch count of one kind.  Not thread-safe; off by default. */
