@@ -222,7 +222,7 @@ def run_ours(args, rank, world, dev, barrier, allmax):
     assert q.device_status() == 0
     ms_max = allmax(ms)
     ms_step = ms_max / args.steps
-    value = world * rep.flops() / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(world, rep.flops(), ms_step) / 1e12
 
     # kernel-level roofline pass: the library records events around its own launches
     kp = min(args.steps, 50)
@@ -712,6 +712,34 @@ def run_ncu_case(args):
     assert q.device_status() == 0
 
 
+# --------------------------------------------------------------------------- ranks
+def make_comm(world: int, dev, backend: str = "nccl"):
+    """(barrier, allmax, dist module or None) for one process per GPU.  Replicas only:
+    the ranks share no data-path collective, only the barriers around the timed region
+    and the max over ranks of its duration.  Short process-group timeout, so that ranks
+    waiting for a rank that died end with an error instead of hanging."""
+    if world <= 1:
+        return (lambda: None), (lambda x: x), None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        dist.barrier()
+
+    def allmax(x):
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return barrier, allmax, dist
+
+
+def whole_job_rate(world: int, units_per_rank: float, max_ms: float) -> float:
+    """Units per second of all ranks together: every rank processes units_per_rank in
+    the timed region, whose length is the slowest rank's (max over ranks)."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 # --------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -734,26 +762,9 @@ def main():
         run_reference(args, rank, world)
         return
 
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def allmax(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
+    barrier, allmax, dist = make_comm(world, dev, "nccl")
     try:
         run_ours(args, rank, world, dev, barrier, allmax)
     finally:
