@@ -53,7 +53,6 @@ def test_two_gloo_ranks_max_and_whole_job_rate():
         assert rate == pytest.approx(2 * 1e9 / 15e-3)      # both ranks' units over that time
 
 
-
 def test_single_rank_needs_no_process_group():
     barrier, allmax, dist = bench.make_comm(1, torch.device("cpu"))
     assert dist is None
