@@ -686,6 +686,15 @@ def run_ncu_case(args):
         torch.cuda.synchronize()
         assert q.device_status() == 0
         return
+    if name == "quant_signed":   # the quantizer with signed block constants, up-projection weight
+        case = qi.LLAMA7B[1]
+        W = qi.make_weight(case.N, case.K, case.seed).to(dev)
+        out = q.NF4Weight.empty(case.N, case.K, dev, dq=q.DQ_SIGNED)
+        for _ in range(args.warmup + args.steps):
+            q.quantize_nf4(W, out=out)
+        torch.cuda.synchronize()
+        assert q.device_status() == 0
+        return
     if name == "lq":     # the low-rank plus quantized decomposition of a 4096 x 4096 weight
         W = qi.make_lowrank_weight(4096, 4096, 64, seed=99).to(dev)
         Om = qi.make_test_matrix(4096, 72, seed=100).to(dev)
@@ -747,7 +756,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--ncu-case", choices=["step", "q", "up", "down", "gemv1", "gemv16", "dequant", "lq"], default=None,
+    ap.add_argument("--ncu-case", choices=["step", "q", "up", "down", "gemv1", "gemv16", "dequant", "lq", "quant_signed"], default=None,
                     help="profiling entry: run only one projection's calls (--warmup + --steps times), no JSON")
     args = ap.parse_args()
     if args.ncu_case:
