@@ -572,27 +572,87 @@ def measure_extras(q, rep, dev, pk, barrier):
 
 
 def measure_e2e(q, rep, dev, steps, barrier, allmax, world):
-    """Same step through the C-ABI with host buffers: H2D of X and dY, D2H of Y, dX, dA, dB."""
+    """Same step through the C-ABI with host buffers: every step copies X and dY in from pinned host
+    memory and Y, dX, dA, dB back out.  The copies run on their own streams (host-to-device and
+    device-to-host use separate copy engines, and the link is full duplex) and the device buffers
+    are double-buffered, so one projection's copies overlap another's compute; every byte of every
+    step still crosses the link inside the timed region."""
     host = []
     for c in rep.cases:
         host.append({k: c[k].cpu().pin_memory() for k in ("X", "dY")} |
                     {k: torch.empty_like(c[k], device="cpu").pin_memory() for k in ("Y", "dX", "dA", "dB")})
     h2d = sum(h["X"].numel() * 2 + h["dY"].numel() * 2 for h in host)
     d2h = sum(h["Y"].numel() * 2 + h["dX"].numel() * 2 + h["dA"].numel() * 4 + h["dB"].numel() * 4 for h in host)
+    keys_in, keys_out = ("X", "dY"), ("Y", "dX", "dA", "dB")
+    # two device buffer sets per projection
+    bufs = [[{k: torch.empty_like(c[k]) for k in keys_in + keys_out + ("H",)} for _ in range(2)] for c in rep.cases]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {}
+
+    def event(key):
+        if key not in ev:
+            ev[key] = torch.cuda.Event()
+        return ev[key]
+
+    state = {"u": 0}
+
+    def unit(ci):
+        c, h = rep.cases[ci], host[ci]
+        u = state["u"]
+        state["u"] += 1
+        bset = (ci, u // len(rep.cases) % 2)
+        dbuf = bufs[ci][bset[1]]
+        with torch.cuda.stream(s_in):        # inputs may be overwritten once the compute that read them is done
+            if ("comp", bset) in ev:
+                s_in.wait_event(ev[("comp", bset)])
+            for k in keys_in:
+                dbuf[k].copy_(h[k], non_blocking=True)
+            event(("in", bset)).record(s_in)
+        comp.wait_event(ev[("in", bset)])
+        if ("out", bset) in ev:              # outputs may be overwritten once they are copied out
+            comp.wait_event(ev[("out", bset)])
+        q.linear_fwd(c["w"], dbuf["X"], c["A"], c["B"], c["s"], out=dbuf["Y"], h_out=dbuf["H"], workspace=c["wsf"])
+        q.linear_bwd(c["w"], dbuf["X"], dbuf["dY"], c["A"], c["B"], c["s"], H=dbuf["H"],
+                     outs=(dbuf["dX"], dbuf["dA"], dbuf["dB"]), workspace=c["wsb"])
+        event(("comp", bset)).record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev[("comp", bset)])
+            for k in keys_out:
+                h[k].copy_(dbuf[k], non_blocking=True)
+            event(("out", bset)).record(s_out)
 
     def st():
-        for c, h in zip(rep.cases, host):
-            c["X"].copy_(h["X"], non_blocking=True)
-            c["dY"].copy_(h["dY"], non_blocking=True)
-            q.linear_fwd(c["w"], c["X"], c["A"], c["B"], c["s"], out=c["Y"], h_out=c["H"], workspace=c["wsf"])
-            q.linear_bwd(c["w"], c["X"], c["dY"], c["A"], c["B"], c["s"], H=c["H"],
-                         outs=(c["dX"], c["dA"], c["dB"]), workspace=c["wsb"])
-            for k in ("Y", "dX", "dA", "dB"):
-                h[k].copy_(c[k], non_blocking=True)
-    st()
-    ms = allmax(timed(st, steps, barrier)) / steps
+        for ci in range(len(rep.cases)):
+            unit(ci)
+
+    def run(n):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        start.record(comp)
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
+        for _ in range(n):
+            st()
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)               # the last outputs are on the host
+        end.record(comp)
+        torch.cuda.synchronize()
+        barrier()
+        return start.elapsed_time(end)
+    run(2)
+    ms = allmax(run(steps)) / steps
+    # the pipeline computes what the plain step computes
+    for c, h in zip(rep.cases, host):
+        q.linear_fwd(c["w"], c["X"], c["A"], c["B"], c["s"], out=c["Y"], h_out=c["H"], workspace=c["wsf"])
+    torch.cuda.synchronize()
+    for c, h in zip(rep.cases, host):
+        assert torch.equal(h["Y"].to(dev), c["Y"]), "end-to-end pipeline output differs from the device step"
     return {"value": round(world * rep.flops() / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4),
+            "note": "inputs copied in and outputs copied out every step (pinned host memory); copies on "
+                    "their own streams, device buffers double-buffered"}
 
 
 # --------------------------------------------------------------------------- oracle (CPU) arm
