@@ -105,6 +105,14 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *t
       : "memory");
 }
 
+// Bring a 2D tile into L2 ahead of its load (no shared-memory destination, no
+// barrier; the same coordinate rules as a load).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *tm, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tm)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // 1-D bulk copies (16-byte aligned addresses, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
   asm volatile(

@@ -31,7 +31,9 @@
 // does the same with its two.  Measured per K-step on the LLaMA-7B projections
 // the issuer spends ~1150 clocks issuing MMAs and 70-350 clocks on its inputs,
 // almost all of it on the forwarded signal; the shallower operand ring and code
-// prefetch (fewer loads in flight) took 2-6 % off the step time.
+// prefetch (fewer loads in flight) took 2-6 % off the step time, and an L2
+// prefetch of the activation tile A_STAGES steps ahead 4-5 % off the launches
+// whose large activation operand comes from DRAM.
 // Waits are bounded; on expiry a CTA latches QLORA_ERR_DEVICE_TIMEOUT, lets
 // its outstanding loads and the pair's MMAs land, frees TMEM and exits.
 #include "decode.cuh"
@@ -221,6 +223,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int kh = 0; kh < C::KH; ++kh)
               tma_load_2d(st + (t * C::KH + kh) * HALF, &tm_act, &sm->afull[s], i * BK + 64 * kh,
                           static_cast<int>(mbase + 256 * t));
+          // the tile A_STAGES steps further on goes to L2 now: its load waits for a free
+          // slot, and for the operands read from DRAM the wait would otherwise add the
+          // DRAM latency to the step
+          const int ipf = i + A_STAGES;
+          if (ipf < p.nkb)
+            for (int t = 0; t < NACC; ++t)
+              for (int kh = 0; kh < C::KH; ++kh)
+                tma_prefetch_2d(&tm_act, ipf * BK + 64 * kh, static_cast<int>(mbase + 256 * t));
         } else {
           const int ls = i - p.nkb;
           const int rem = p.r - ls * BK;
