@@ -448,25 +448,31 @@ __global__ void __launch_bounds__(kLqThreads) lq_chol_inv_kernel(const double *_
   }
   __syncthreads();
   const double tol = 1e-24 * dmax;
+  // Right-looking elimination on the unscaled columns (one barrier per column):
+  // G[a][b] -= G[a][j] G[b][j] / G[j][j] for j < b <= a; column j and the pivot
+  // are not written in step j, so every thread reads them after the previous
+  // step's barrier.  Afterwards L[a][j] = G[a][j] / sqrt(G[j][j]).
   for (int j = 0; j < l; ++j) {
     const double piv = G[j * lp + j];
-    const bool dj = !(piv > tol);
-    const double d = dj ? 0.0 : sqrt(piv);
-    __syncthreads();   // every thread has read the pivot
-    // column j of L below the diagonal
-    for (int a = j + 1 + threadIdx.x; a < l; a += blockDim.x) G[a * lp + j] = dj ? 0.0 : G[a * lp + j] / d;
-    if (threadIdx.x == 0) {
-      G[j * lp + j] = d;
-      dead[j] = dj;
-    }
-    __syncthreads();
-    // trailing update of the lower triangle: G[a][b] -= L[a][j] L[b][j], j < b <= a (a row per warp)
+    const double inv = piv > tol ? 1.0 / piv : 0.0;   // a dependent column is dropped
     for (int a = j + 1 + warp; a < l; a += nwarps) {
-      const double laj = G[a * lp + j];
-      for (int b = j + 1 + lane; b <= a; b += 32) G[a * lp + b] = __fma_rn(-laj, G[b * lp + j], G[a * lp + b]);
+      const double gaj = G[a * lp + j] * inv;
+      for (int b = j + 1 + lane; b <= a; b += 32) G[a * lp + b] = __fma_rn(-gaj, G[b * lp + j], G[a * lp + b]);
     }
     __syncthreads();
   }
+  __shared__ double rinv[kLqMaxL];
+  for (int j = threadIdx.x; j < l; j += blockDim.x) {
+    const double piv = G[j * lp + j];
+    dead[j] = !(piv > tol);
+    const double d = dead[j] ? 0.0 : sqrt(piv);
+    rinv[j] = dead[j] ? 0.0 : 1.0 / d;
+    G[j * lp + j] = d;
+  }
+  __syncthreads();
+  for (int a = warp; a < l; a += nwarps)
+    for (int j = lane; j < a; j += 32) G[a * lp + j] *= rinv[j];
+  __syncthreads();
   // L^-1 by forward substitution, one column per thread (four partial sums per dot product)
   for (int c = threadIdx.x; c < l; c += blockDim.x) {
     for (int j = 0; j < l; ++j) {
