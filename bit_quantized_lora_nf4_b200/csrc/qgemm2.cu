@@ -16,7 +16,8 @@
 //               64-column boxes) into a 4-deep ring.
 //   warp 1      TMEM allocation for the pair; in the even CTA one lane issues
 //               the pair MMA and commits to both CTAs' barriers (multicast);
-//               in the odd CTA one lane forwards "decoded" to the even CTA.
+//               in the odd CTA two lanes, taking the K-steps in turn, forward
+//               "decoded" to the even CTA.
 //   warps 2-9   decode: thread (row = t % 128, j = t / 128) owns block j of its
 //               row.  Its 32 bytes of codes and its 8-bit constant are loaded
 //               from global memory into registers two of its K-steps ahead; it
@@ -30,7 +31,9 @@
 // to bounded waits only for one that is not complete; the odd CTA's forwarder
 // does the same with its two.  Measured per K-step on the LLaMA-7B projections
 // the issuer spends ~1150 clocks issuing MMAs and 70-350 clocks on its inputs,
-// almost all of it on the forwarded signal; the shallower operand ring and code
+// almost all of it on the forwarded signal (one forwarding lane could not keep
+// ahead: its cluster-scope arrive takes ~1100 clocks; two lanes can); the
+// shallower operand ring and code
 // prefetch (fewer loads in flight) took 2-6 % off the step time, and an L2
 // prefetch of the activation tile A_STAGES steps ahead 4-5 % off the launches
 // whose large activation operand comes from DRAM.
@@ -84,6 +87,7 @@ constexpr int MAX_D_STAGES = 8;
 static_assert(Cfg<1>::D_STAGES >= 2 && Cfg<2>::D_STAGES <= MAX_D_STAGES, "operand ring depth");
 static_assert(A_STAGES * A_BYTES + D_RING + 1280 <= 232448, "shared memory budget");
 constexpr uint64_t kDrainLimit = 4000000000ull;
+constexpr int kFwdLanes = 2;                // odd CTA: lanes forwarding readiness, steps in turn
 constexpr int kGroupM = 8;                  // M-pairs per raster group
 
 struct Params {
@@ -283,15 +287,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_commit_pair_mc(&sm->dfree[sd], 0x3);
       }
       tc_commit_pair_mc(&sm->acc_full, 0x3);
-    } else if (lane == 0) {
+    } else if (rank != 0 && lane < kFwdLanes) {
       // ---------------------------------------------------------- odd CTA: forward readiness
       // The even CTA's MMA reads this CTA's activation tile and operand half:
       // once both are in place, one cluster-scope release per stage.  (The
       // decode warps arrive only locally: a cluster-scope release from them
       // would also wait for the code loads they keep in flight for later steps.)
       // Both barriers are probed together; the bounded waits only for one that
-      // is not complete yet.
-      for (int i = 0; i < nsteps; ++i) {
+      // is not complete yet.  A cluster-scope release arrive takes about as long
+      // as a K-step's MMAs, so kFwdLanes lanes take the steps in turn and their
+      // arrives overlap.
+      for (int i = lane; i < nsteps; i += kFwdLanes) {
         const int sa = i % A_STAGES, sd = i % D_STAGES;
         const uint32_t pa = (i / A_STAGES) & 1, pd = (i / D_STAGES) & 1;
         const bool ra = mbar_test(smem_addr(&sm->afull[sa]), pa), rd = mbar_test(smem_addr(&sm->decoded[sd]), pd);
