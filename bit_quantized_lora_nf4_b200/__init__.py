@@ -23,6 +23,8 @@ QLORA_OP_FWD = 0
 QLORA_OP_BWD = 1
 QLORA_OP_FWD_DENSE = 2      # the linear on a dense bf16 base weight (any quantizer's output)
 QLORA_OP_BWD_DENSE = 3
+# Stream-K split of the fused GEMM's last partial wave (qlora_set_stream_k).
+STREAM_K_OFF, STREAM_K_AUTO, STREAM_K_ALWAYS = 0, 1, 2
 
 STATUS_NAMES = {
     0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED_SHAPE", 3: "QLORA_ERR_MISALIGNED",
@@ -32,7 +34,7 @@ STATUS_NAMES = {
 # Every symbol include/qlora.h declares.
 EXPORTS = (
     "qlora_codes_bytes", "qlora_absmax_bytes", "qlora_group_scale_bytes", "qlora_quantize_nf4", "qlora_dequantize",
-    "qlora_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
+    "qlora_workspace_bytes", "qlora_workspace_min_bytes", "qlora_set_stream_k", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
     "qlora_status_string", "qlora_set_wait_limit", "qlora_selftest_wait_timeout", "qlora_profile_enable",
     "qlora_profile_read", "qlora_linear_fwd_noalloc", "qlora_format_codebook", "qlora_group_scale_bytes_dq",
     "qlora_quantize_workspace_bytes", "qlora_quantize_nf4_ws", "qlora_lq_workspace_bytes", "qlora_lq_decompose",
@@ -89,6 +91,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_quantize_nf4": (i32, [vp, wp, vp]),
         "qlora_dequantize": (i32, [wp, vp, vp]),
         "qlora_workspace_bytes": (sz, [i32, i64, i64, i64, i32]),
+        "qlora_workspace_min_bytes": (sz, [i32, i64, i64, i64, i32]),
+        "qlora_set_stream_k": (i32, [i32]),
         "qlora_linear_fwd": (i32, [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
         "qlora_linear_bwd": (i32, [wp, vp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]),
         "qlora_nf4_codebook": (i32, [ctypes.POINTER(ctypes.c_float)]),
@@ -194,6 +198,14 @@ def device_status() -> int:
 
 def set_wait_limit(cycles: int) -> int:
     return int(load().qlora_set_wait_limit(cycles))
+
+
+def set_stream_k(mode: int) -> int:
+    """STREAM_K_OFF / _AUTO (default) / _ALWAYS; returns the previous mode."""
+    prev = int(load().qlora_set_stream_k(mode))
+    if prev < 0:
+        raise ValueError(f"unknown stream-K mode {mode}")
+    return prev
 
 
 def selftest_wait_timeout(cycles: int) -> int:

@@ -119,6 +119,9 @@ Nf4Table weight_table(const qlora_nf4_weight *w) {
 
 uint64_t wait_limit() { return g_wait_limit.load(); }
 
+std::atomic<int> g_stream_k{QLORA_STREAM_K_AUTO};
+int stream_k_mode() { return g_stream_k.load(); }
+
 // ----------------------------------------------------------------- device status word
 __device__ int g_device_status;
 
@@ -247,13 +250,21 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Plan {
   // byte offsets into the workspace
-  size_t part = 0, H = 0, sH = 0, Hs = 0, Gb = 0, Gs = 0, total = 0;
+  size_t part = 0, H = 0, sH = 0, Hs = 0, Gb = 0, Gs = 0, sk = 0, total = 0;
+  bool has_sk = false;   // the fused GEMMs run on CTA pairs: room for their stream-K tail
+  size_t min_total = 0;  // without the stream-K tail (the last region, optional)
+  // the stream-K region when the caller's workspace holds it, else null
+  void *sk_region(void *ws, size_t ws_bytes) const {
+    return has_sk && ws_bytes >= total ? static_cast<char *>(ws) + sk : nullptr;
+  }
   int spH = 1, spG = 1, spB = 1, spA = 1;
   int64_t kpsH = 0, kpsG = 0, kpsB = 0, kpsA = 0;
   bool gemv = false;
 };
 
-Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, bool allow_gemv = true) {
+// `packed`: the base weight is a packed NF4 weight (the few-token and
+// one-CTA kernels may run); a dense W' always takes the pair kernel.
+Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, bool packed = true) {
   Plan p;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -262,10 +273,10 @@ Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, bool allow_gemv =
     return o;
   };
   const size_t Mr = static_cast<size_t>(M) * r;
-  if (op == QLORA_OP_FWD && allow_gemv && M <= kGemvMaxTokens && gemv_enabled()) {
+  if (op == QLORA_OP_FWD && packed && M <= kGemvMaxTokens && gemv_enabled()) {
     p.gemv = true;
     p.part = take(gemv_workspace_bytes(M, N, K, r));
-    p.total = off;
+    p.total = p.min_total = off;
     return p;
   }
   skinny_plan(M, r, K, &p.spH, &p.kpsH);
@@ -286,6 +297,11 @@ Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, bool allow_gemv =
     p.Hs = take(Mr * 2 * 2);
     p.Gb = take(Mr * 2);
     p.Gs = take(Mr * 2 * 2);
+  }
+  p.min_total = off;
+  if (!packed || M > kPairMinRows) {
+    p.has_sk = true;
+    p.sk = take(pair_sk_workspace_bytes(M));
   }
   p.total = off;
   return p;
@@ -451,6 +467,11 @@ qlora_status qlora_format_codebook(int format, float *levels, float *thresh) {
 
 uint64_t qlora_set_wait_limit(uint64_t cycles) { return g_wait_limit.exchange(cycles); }
 
+int qlora_set_stream_k(int mode) {
+  if (mode < QLORA_STREAM_K_OFF || mode > QLORA_STREAM_K_ALWAYS) return -1;
+  return g_stream_k.exchange(mode);
+}
+
 void qlora_profile_enable(int on) {
   Prof &P = prof();
   P.on = on != 0;
@@ -506,6 +527,13 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
   return make_plan(base, M, N, K, r, !dense).total;
 }
 
+size_t qlora_workspace_min_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
+  if (op < QLORA_OP_FWD || op > QLORA_OP_BWD_DENSE || M < 1 || N < 1 || K < 1 || r < 1) return 0;
+  const bool dense = op == QLORA_OP_FWD_DENSE || op == QLORA_OP_BWD_DENSE;
+  const int base = dense ? op - QLORA_OP_FWD_DENSE : op;
+  return make_plan(base, M, N, K, r, !dense).min_total;
+}
+
 qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
                                    void *stream) {
   if (!W) return QLORA_ERR_INVALID_ARG;
@@ -546,7 +574,7 @@ qlora_status linear_fwd_impl(const WeightSrc &src, const uint16_t *X, int64_t M,
                              void *stream) {
   const int64_t N = src.N, K = src.K;
   const Plan p = make_plan(QLORA_OP_FWD, M, N, K, r, src.w != nullptr);
-  QL_TRY(check_ws(ws, ws_bytes, p.total));
+  QL_TRY(check_ws(ws, ws_bytes, p.min_total));
   if (H_out && !aligned16(H_out)) return QLORA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *H = H_out ? H_out : at<float>(ws, p.H);
@@ -557,16 +585,20 @@ qlora_status linear_fwd_impl(const WeightSrc &src, const uint16_t *X, int64_t M,
     return launch_gemv(g, st);
   }
   QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
-  return launch_qgemm(gemm_args(src, false, M, X, at<uint16_t>(ws, p.sH), B, r, Y), st);
+  QGemmArgs g = gemm_args(src, false, M, X, at<uint16_t>(ws, p.sH), B, r, Y);
+  g.sk_ws = p.sk_region(ws, ws_bytes);
+  return launch_qgemm(g, st);
 }
 
 qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint16_t *dY, int64_t M,
                              const uint16_t *A, const uint16_t *B, int r, float s, const float *H_saved,
                              uint16_t *dX, float *dA, float *dB, void *ws, size_t ws_bytes, void *stream) {
   const int64_t N = src.N, K = src.K;
-  const Plan p = make_plan(QLORA_OP_BWD, M, N, K, r);
-  QL_TRY(check_ws(ws, ws_bytes, p.total));
+  const Plan p = make_plan(QLORA_OP_BWD, M, N, K, r, src.w != nullptr);
+  QL_TRY(check_ws(ws, ws_bytes, p.min_total));
   if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_MISALIGNED;
+  QGemmArgs dgrad = gemm_args(src, true, M, dY, at<uint16_t>(ws, p.Gb), A, r, dX);
+  dgrad.sk_ws = p.sk_region(ws, ws_bytes);
   if (H_saved && !aligned16(H_saved)) return QLORA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float *part = at<float>(ws, p.part);
@@ -622,7 +654,7 @@ qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint
     QL_CUDA(cudaEventRecord(side->fork, st));
     QL_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
     // dX = dY W' + Gb A first, so that its CTAs are dispatched ahead of the products'
-    const qlora_status gst = launch_qgemm(gemm_args(src, true, M, dY, Gb, A, r, dX), st);
+    const qlora_status gst = launch_qgemm(dgrad, st);
     QL_CUDA(launch_skinny(aB, side->s));
     QL_CUDA(launch_skinny(aA, side->s));
     QL_CUDA(cudaEventRecord(side->join, side->s));
@@ -644,7 +676,7 @@ qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint
     QL_CUDA(launch_finalize_rows(part, p.spA, r, K, dA, st));
   }
   // dX = dY W' + Gb A
-  return launch_qgemm(gemm_args(src, true, M, dY, Gb, A, r, dX), st);
+  return launch_qgemm(dgrad, st);
 }
 
 }  // namespace
@@ -695,7 +727,7 @@ qlora_status qlora_linear_fwd_materialized(qlora_materialize_fn materialize, voi
   if (!materialize || !W_scratch) return QLORA_ERR_INVALID_ARG;
   QL_TRY(check_linear_shape(N, K, M, r, s, X, A, B, Y));
   if (!aligned16(W_scratch)) return QLORA_ERR_MISALIGNED;
-  QL_TRY(check_ws(ws, ws_bytes, make_plan(QLORA_OP_FWD, M, N, K, r, false).total));
+  QL_TRY(check_ws(ws, ws_bytes, make_plan(QLORA_OP_FWD, M, N, K, r, false).min_total));
   QL_TRY(materialize(ctx, W_scratch, N, K, stream));
   return qlora_linear_fwd_dense(W_scratch, N, K, X, M, A, B, r, s, Y, H_out, ws, ws_bytes, stream);
 }
@@ -708,7 +740,7 @@ qlora_status qlora_linear_bwd_materialized(qlora_materialize_fn materialize, voi
   if (!materialize || !W_scratch || !dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
   QL_TRY(check_linear_shape(N, K, M, r, s, X, A, B, dX));
   if (!aligned16(W_scratch)) return QLORA_ERR_MISALIGNED;
-  QL_TRY(check_ws(ws, ws_bytes, make_plan(QLORA_OP_BWD, M, N, K, r).total));
+  QL_TRY(check_ws(ws, ws_bytes, make_plan(QLORA_OP_BWD, M, N, K, r, false).min_total));
   QL_TRY(materialize(ctx, W_scratch, N, K, stream));
   return qlora_linear_bwd_dense(W_scratch, N, K, X, dY, M, A, B, r, s, H_saved, dX, dA, dB, ws, ws_bytes, stream);
 }

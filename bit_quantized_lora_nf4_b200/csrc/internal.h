@@ -71,9 +71,16 @@ struct QGemmArgs {
   uint16_t *out;
   Nf4Table tab;        // weight_table() of the weight
   const uint16_t *wdense = nullptr;   // dense bf16 W' [wN, wK] instead of the packed weight (pair kernel only)
+  void *sk_ws = nullptr;              // pair kernel: pair_sk_workspace_bytes(M) for its stream-K tail (null: none)
 };
+// Workspace of the pair kernel's stream-K tail (fp32 pieces of shared tiles and their counters).
+size_t pair_sk_workspace_bytes(int64_t M);
+// QLORA_STREAM_K_* set by qlora_set_stream_k.
+int stream_k_mode();
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
-// The same product on a CTA pair (256-row tiles); launch_qgemm dispatches to it for M > 128.
+// The same product on a CTA pair (256-row tiles); launch_qgemm dispatches to it
+// for M > kPairMinRows and for a dense W'.
+constexpr int64_t kPairMinRows = 128;
 qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st);
 
 // Few-token forward: Y[M, N] = X W'^T + (s X A^T) B^T for M <= 16.

@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace
 
 qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st) {
-  if (a.M > BM || a.wdense) return launch_qgemm_pair(a, st);
+  if (a.M > kPairMinRows || a.wdense) return launch_qgemm_pair(a, st);
   CUtensorMap tm_act, tm_codes, tm_lact;
   const int64_t kred = a.dgrad ? a.wN : a.wK;      // reduction length of the weight segment
   const int64_t n_out = a.dgrad ? a.wK : a.wN;

@@ -39,6 +39,9 @@
 // whose large activation operand comes from DRAM.
 // Waits are bounded; on expiry a CTA latches QLORA_ERR_DEVICE_TIMEOUT, lets
 // its outstanding loads and the pair's MMAs land, frees TMEM and exits.
+#include <algorithm>
+#include <atomic>
+
 #include "decode.cuh"
 #include "internal.h"
 
@@ -67,7 +70,6 @@ constexpr int D_RING = QLORA_PAIR_D_RING_KB * 1024;   // decoded-operand stages
 constexpr int PREFETCH = QLORA_PAIR_PREFETCH;
 constexpr int NUM_DEC_WARPS = 8;
 constexpr int THREADS = 32 * (2 + NUM_DEC_WARPS);
-constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + 256;
 
 // NACC = accumulators per CTA: the pair tile covers 256 * NACC rows.  With
 // NACC = 2 every decoded operand half feeds two MMAs (rows 0-255 and 256-511
@@ -85,10 +87,22 @@ struct Cfg {
 };
 constexpr int MAX_D_STAGES = 8;
 static_assert(Cfg<1>::D_STAGES >= 2 && Cfg<2>::D_STAGES <= MAX_D_STAGES, "operand ring depth");
-static_assert(A_STAGES * A_BYTES + D_RING + 1280 <= 232448, "shared memory budget");
 constexpr uint64_t kDrainLimit = 4000000000ull;
 constexpr int kFwdLanes = 2;                // odd CTA: lanes forwarding readiness, steps in turn
 constexpr int kGroupM = 8;                  // M-pairs per raster group
+// Stream-K tail: the tiles left after the last full wave have their K-steps
+// split evenly over the cluster slots; a workspace provides for kSkMaxUnits
+// such clusters, and none takes fewer than kSkMinSteps K-steps.  Measured on
+// the LLaMA-7B projections (0.85 us per K-step), a cluster sharing tiles spends
+// about kSkCostSteps K-steps' time beyond its own steps (accumulator drain and
+// refill at a tile boundary, writing its 256 KB fp32 piece, the finisher
+// reading the others' pieces at ~50 GB/s per SM), and a whole tile about
+// kTileCostSteps (fill, drain, epilogue); the automatic mode splits only when
+// that comes out shorter.
+constexpr int kSkMaxUnits = 80;
+constexpr int kSkMinSteps = 16;
+constexpr int kSkCostSteps = 33;
+constexpr int kTileCostSteps = 8;
 
 struct Params {
   int64_t M;
@@ -107,6 +121,13 @@ struct Params {
   uint16_t *out;
   int *status;
   uint64_t wait_limit;
+  int ns;            // K-steps per tile (nkb + nls)
+  int dp_tiles;      // tiles taken whole, one per cluster (the full waves)
+  int sk_units;      // clusters sharing the remaining tiles' K-steps (0: none)
+  int64_t sk_steps;  // K-steps of the shared tiles
+  int *sk_count;     // [shared tile][rank]: CTAs that finished accumulating a piece
+  int *sk_ready;     // [shared tile][rank]: pieces written to sk_part
+  float *sk_part;    // [unit][first, last piece][rank][NACC x 128 x 256] fp32
 };
 
 struct Smem {
@@ -116,9 +137,34 @@ struct Smem {
   uint64_t decoded[MAX_D_STAGES];      // this CTA's decode group wrote the operand half
   uint64_t peer_decoded[MAX_D_STAGES]; // even CTA only: the odd CTA's A tile and operand half are ready
   uint64_t acc_full;               // the pair's accumulation completed (multicast commit)
+  uint64_t tmem_empty;             // even CTA: both CTAs read the accumulators (next tile may start)
   uint32_t tmem_base;
   int abort_flag;
+  int sk_role;                     // this CTA's arrival order on a shared tile
+  int sk_ok;                       // the other pieces were written in time
 };
+constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + static_cast<int>(sizeof(Smem));
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(A_STAGES * A_BYTES >= NUM_DEC_WARPS * 16384, "epilogue staging fits the activation ring");
+
+// Tile t of the grouped raster: consecutive tiles walk kGroupM M-pairs before
+// moving to the next N tile, so a wave reuses both operands from L2.
+__device__ __forceinline__ void tile_coords(const Params &p, int t, int &pm, int &pn) {
+  const int in_group = kGroupM * p.num_n;
+  const int first_m = (t / in_group) * kGroupM;
+  const int gsz = min(p.num_m - first_m, kGroupM);
+  pm = first_m + (t % in_group) % gsz;
+  pn = (t % in_group) / gsz;
+}
+
+// Stream-K partition of the shared tiles' K-steps: unit u takes
+// [sk_begin(u), sk_begin(u + 1)); sk_unit_of inverts it.
+__host__ __device__ __forceinline__ int64_t sk_begin(int64_t steps, int units, int u) {
+  return static_cast<int64_t>(u) * steps / units;
+}
+__device__ __forceinline__ int sk_unit_of(const Params &p, int64_t g) {
+  return static_cast<int>(((g + 1) * p.sk_units - 1) / p.sk_steps);
+}
 
 template <bool CLUSTER_SCOPE>
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const Params &p, Smem *sm) {
@@ -154,7 +200,7 @@ struct DenseLoad {
 template <bool DGRAD, int NACC, bool DENSE>
 __global__ void __launch_bounds__(THREADS, 1)
     qgemm2_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lact,
-                  const Params p, const Nf4Table tab) {
+                  const __grid_constant__ CUtensorMap tm_out, const Params p, const Nf4Table tab) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *a_ring = smem;
@@ -168,22 +214,71 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();                              // 0 = even (MMA-issuing) CTA
-  // Grouped raster over pair tiles: consecutive clusters walk kGroupM M-pairs
-  // before moving to the next N tile, so a wave reuses both operands from L2.
-  int pm, pn;
-  {
-    const int cid = static_cast<int>(blockIdx.x >> 1);
-    const int in_group = kGroupM * p.num_n;
-    const int first_m = (cid / in_group) * kGroupM;
-    const int gsz = min(p.num_m - first_m, kGroupM);
-    pm = first_m + (cid % in_group) % gsz;
-    pn = (cid % in_group) / gsz;
+  const int ns = p.ns;
+  // The cluster's K-steps in the linear (tile, K-step) order: a whole tile in
+  // the full waves, a contiguous share of the remaining tiles' steps for a
+  // stream-K unit.  Running step j of the cluster is linear step G0 + j.
+  int64_t G0, G1;
+  int unit = -1;
+  const int cid = static_cast<int>(blockIdx.x >> 1);
+  if (cid < p.dp_tiles) {
+    G0 = static_cast<int64_t>(cid) * ns;
+    G1 = G0 + ns;
+  } else {
+    unit = cid - p.dp_tiles;
+    const int64_t base = static_cast<int64_t>(p.dp_tiles) * ns;
+    G0 = base + sk_begin(p.sk_steps, p.sk_units, unit);
+    G1 = base + sk_begin(p.sk_steps, p.sk_units, unit + 1);
   }
-  // this CTA's rows of accumulator t: mbase + 256 t .. + 127
-  const int64_t mbase = static_cast<int64_t>(pm) * (2 * BM * NACC) + rank * BM;
-  const int64_t n0 = static_cast<int64_t>(pn) * BN;                    // pair's first output column
-  const int64_t nb0 = n0 + rank * 128;                                  // this CTA's operand columns
-  const int nsteps = p.nkb + p.nls;
+  const int t_first = static_cast<int>(G0 / ns);
+  const int t_last = static_cast<int>((G1 - 1) / ns);
+  const int nseg = t_last - t_first + 1;
+  const int nsteps = static_cast<int>(G1 - G0);
+
+  // One segment = the cluster's K-steps [k_lo, k_hi) of tile t; j0 is the
+  // running index of its first step.  This CTA's rows of accumulator a are
+  // mbase + 256 a .. + 127, its operand columns nb0 .. + 127.
+  struct Seg {
+    int k_lo, k_hi, j0;
+    int mbase, n0, nb0;      // M, N and K are below 2^31
+  };
+  auto segment = [&](int t) {
+    Seg sg;
+    const int64_t tb = static_cast<int64_t>(t) * ns;
+    sg.k_lo = static_cast<int>((G0 > tb ? G0 : tb) - tb);
+    sg.k_hi = static_cast<int>((G1 < tb + ns ? G1 : tb + ns) - tb);
+    sg.j0 = static_cast<int>(tb + sg.k_lo - G0);
+    int pm, pn;
+    tile_coords(p, t, pm, pn);
+    sg.mbase = pm * (2 * BM * NACC) + static_cast<int>(rank) * BM;
+    sg.n0 = pn * BN;
+    sg.nb0 = sg.n0 + static_cast<int>(rank) * 128;
+    return sg;
+  };
+  // Follows running steps forward (never back) across tile boundaries.
+  struct Cursor {
+    int t;
+    int64_t tb;
+    int mbase, nb0;
+  };
+  auto cursor_start = [&]() {
+    const Seg sg = segment(t_first);
+    return Cursor{t_first, static_cast<int64_t>(t_first) * ns, sg.mbase, sg.nb0};
+  };
+  // tile-local K-step of running step j (j < nsteps), moving the cursor to its tile
+  auto cursor_at = [&](Cursor &c, int j) {
+    const int64_t G = G0 + j;
+    if (G >= c.tb + ns) {
+      do {
+        ++c.t;
+        c.tb += ns;
+      } while (G >= c.tb + ns);
+      const Seg sg = segment(c.t);
+      c.mbase = sg.mbase;
+      c.nb0 = sg.nb0;
+    }
+    return static_cast<int>(G - c.tb);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_STAGES; ++s) {
@@ -196,10 +291,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm->peer_decoded[s], 1);
     }
     mbar_init(&sm->acc_full, 1);
+    mbar_init(&sm->tmem_empty, 2 * NUM_DEC_WARPS);
     sm->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_act);
     tma_prefetch_desc(&tm_lact);
+    tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc_pair(&sm->tmem_base, C::TMEM_COLS);
@@ -215,37 +312,49 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ activation TMA (each CTA)
     if (lane == 0) {
       int issued = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i % A_STAGES;
-        const uint32_t ph = (i / A_STAGES) & 1;
-        if (i >= A_STAGES && !wait_or_abort<false>(&sm->aempty[s], ph ^ 1, p, sm)) break;
-        uint8_t *st = a_ring + s * A_BYTES;
-        // atom column (t, kh) of the stage at (t * KH + kh) * HALF
-        if (i < p.nkb) {
-          mbar_arrive_expect_tx(&sm->afull[s], A_BYTES);
-          for (int t = 0; t < NACC; ++t)
-            for (int kh = 0; kh < C::KH; ++kh)
-              tma_load_2d(st + (t * C::KH + kh) * HALF, &tm_act, &sm->afull[s], i * BK + 64 * kh,
-                          static_cast<int>(mbase + 256 * t));
+      bool stop = false;
+      Cursor pf = cursor_start();            // the step A_STAGES ahead, for the L2 prefetch
+      for (int t = t_first; t <= t_last && !stop; ++t) {
+        const Seg sg = segment(t);
+        for (int k = sg.k_lo; k < sg.k_hi; ++k) {
+          const int i = sg.j0 + (k - sg.k_lo);
+          const int s = i % A_STAGES;
+          const uint32_t ph = (i / A_STAGES) & 1;
+          if (i >= A_STAGES && !wait_or_abort<false>(&sm->aempty[s], ph ^ 1, p, sm)) {
+            stop = true;
+            break;
+          }
+          uint8_t *st = a_ring + s * A_BYTES;
+          // atom column (t, kh) of the stage at (t * KH + kh) * HALF
+          if (k < p.nkb) {
+            mbar_arrive_expect_tx(&sm->afull[s], A_BYTES);
+            for (int a = 0; a < NACC; ++a)
+              for (int kh = 0; kh < C::KH; ++kh)
+                tma_load_2d(st + (a * C::KH + kh) * HALF, &tm_act, &sm->afull[s], k * BK + 64 * kh,
+                            static_cast<int>(sg.mbase + 256 * a));
+          } else {
+            const int ls = k - p.nkb;
+            const int rem = p.r - ls * BK;
+            const int halves = rem > 64 ? C::KH : 1;
+            mbar_arrive_expect_tx(&sm->afull[s], NACC * halves * HALF);
+            for (int a = 0; a < NACC; ++a)
+              for (int kh = 0; kh < halves; ++kh)
+                tma_load_2d(st + (a * C::KH + kh) * HALF, &tm_lact, &sm->afull[s], ls * BK + 64 * kh,
+                            static_cast<int>(sg.mbase + 256 * a));
+          }
           // the tile A_STAGES steps further on goes to L2 now: its load waits for a free
           // slot, and for the operands read from DRAM the wait would otherwise add the
           // DRAM latency to the step
           const int ipf = i + A_STAGES;
-          if (ipf < p.nkb)
-            for (int t = 0; t < NACC; ++t)
-              for (int kh = 0; kh < C::KH; ++kh)
-                tma_prefetch_2d(&tm_act, ipf * BK + 64 * kh, static_cast<int>(mbase + 256 * t));
-        } else {
-          const int ls = i - p.nkb;
-          const int rem = p.r - ls * BK;
-          const int halves = rem > 64 ? C::KH : 1;
-          mbar_arrive_expect_tx(&sm->afull[s], NACC * halves * HALF);
-          for (int t = 0; t < NACC; ++t)
-            for (int kh = 0; kh < halves; ++kh)
-              tma_load_2d(st + (t * C::KH + kh) * HALF, &tm_lact, &sm->afull[s], ls * BK + 64 * kh,
-                          static_cast<int>(mbase + 256 * t));
+          if (ipf < nsteps) {
+            const int kpf = cursor_at(pf, ipf);
+            if (kpf < p.nkb)
+              for (int a = 0; a < NACC; ++a)
+                for (int kh = 0; kh < C::KH; ++kh)
+                  tma_prefetch_2d(&tm_act, kpf * BK + 64 * kh, static_cast<int>(pf.mbase + 256 * a));
+          }
+          issued = i + 1;
         }
-        issued = i + 1;
       }
       for (int j = (issued > A_STAGES ? issued - A_STAGES : 0); j < issued; ++j)
         mbar_wait(&sm->afull[j % A_STAGES], (j / A_STAGES) & 1, kDrainLimit);
@@ -254,39 +363,61 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------- pair MMA issuer (even CTA)
       constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, 0, DGRAD ? 1 : 0);
-      for (int i = 0; i < nsteps; ++i) {
-        const int sa = i % A_STAGES, sd = i % D_STAGES;
-        const uint32_t pa = (i / A_STAGES) & 1, pd = (i / D_STAGES) & 1;
-        // the three inputs of the step probed together (their latencies overlap);
-        // the bounded waits only when one of them is not there yet
-        const bool ready = mbar_test(smem_addr(&sm->afull[sa]), pa) & mbar_test(smem_addr(&sm->decoded[sd]), pd) &
-                           mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd);
-        if (!ready) {
-          if (!mbar_test(smem_addr(&sm->afull[sa]), pa) && !wait_or_abort<false>(&sm->afull[sa], pa, p, sm)) break;
-          if (!mbar_test(smem_addr(&sm->decoded[sd]), pd) && !wait_or_abort<false>(&sm->decoded[sd], pd, p, sm)) break;
-          if (!wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) break;
+      int commits = 0;
+      bool stop = false;
+      for (int t = t_first, seg = 0; t <= t_last && !stop; ++t, ++seg) {
+        const Seg sg = segment(t);
+        // a later tile overwrites the accumulators: both CTAs must have read them
+        if (seg > 0 && !wait_or_abort<true>(&sm->tmem_empty, (seg - 1) & 1, p, sm)) {
+          stop = true;
+          break;
         }
-        tc_fence_after();
-        const uint32_t a_base = smem_addr(a_ring + sa * A_BYTES);
-        const uint32_t d_base = smem_addr(d_ring + sd * D_BYTES);
-        int nk = BK / 16;
-        if (i >= p.nkb) {
-          const int rem = p.r - (i - p.nkb) * BK;
-          nk = rem >= BK ? BK / 16 : (rem + 15) / 16;
-        }
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-          const uint64_t bdesc = DGRAD ? sdesc_sw128(d_base + kk * 2048, BK * 128, 1024)
-                                       : sdesc_sw128(d_base + koff, 16, 1024);
-          for (int t = 0; t < NACC; ++t) {
-            const uint64_t adesc = sdesc_sw128(a_base + t * C::KH * HALF + koff, 16, 1024);
-            tc_mma_bf16_pair(tmem + 256 * t, adesc, bdesc, IDESC, (i | kk) != 0 ? 1u : 0u);
+        for (int k = sg.k_lo; k < sg.k_hi; ++k) {
+          const int i = sg.j0 + (k - sg.k_lo);
+          const int sa = i % A_STAGES, sd = i % D_STAGES;
+          const uint32_t pa = (i / A_STAGES) & 1, pd = (i / D_STAGES) & 1;
+          // the three inputs of the step probed together (their latencies overlap);
+          // the bounded waits only when one of them is not there yet
+          const bool ready = mbar_test(smem_addr(&sm->afull[sa]), pa) & mbar_test(smem_addr(&sm->decoded[sd]), pd) &
+                             mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd);
+          if (!ready) {
+            if ((!mbar_test(smem_addr(&sm->afull[sa]), pa) && !wait_or_abort<false>(&sm->afull[sa], pa, p, sm)) ||
+                (!mbar_test(smem_addr(&sm->decoded[sd]), pd) && !wait_or_abort<false>(&sm->decoded[sd], pd, p, sm)) ||
+                !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
+              stop = true;
+              break;
+            }
           }
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(a_ring + sa * A_BYTES);
+          const uint32_t d_base = smem_addr(d_ring + sd * D_BYTES);
+          int nk = BK / 16;
+          if (k >= p.nkb) {
+            const int rem = p.r - (k - p.nkb) * BK;
+            nk = rem >= BK ? BK / 16 : (rem + 15) / 16;
+          }
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
+            const uint64_t bdesc = DGRAD ? sdesc_sw128(d_base + kk * 2048, BK * 128, 1024)
+                                         : sdesc_sw128(d_base + koff, 16, 1024);
+            for (int a = 0; a < NACC; ++a) {
+              const uint64_t adesc = sdesc_sw128(a_base + a * C::KH * HALF + koff, 16, 1024);
+              tc_mma_bf16_pair(tmem + 256 * a, adesc, bdesc, IDESC, (k != sg.k_lo || kk != 0) ? 1u : 0u);
+            }
+          }
+          tc_commit_pair_mc(&sm->aempty[sa], 0x3);
+          tc_commit_pair_mc(&sm->dfree[sd], 0x3);
         }
-        tc_commit_pair_mc(&sm->aempty[sa], 0x3);
-        tc_commit_pair_mc(&sm->dfree[sd], 0x3);
+        if (stop) break;
+        tc_commit_pair_mc(&sm->acc_full, 0x3);
+        ++commits;
       }
-      tc_commit_pair_mc(&sm->acc_full, 0x3);
+      if (stop) {
+        // given up: one more commit, and wait until it (every MMA issued) has
+        // completed, so that the accumulators are idle before teardown
+        tc_commit_pair_mc(&sm->acc_full, 0x3);
+        mbar_wait(&sm->acc_full, commits & 1, kDrainLimit);
+      }
     } else if (rank != 0 && lane < kFwdLanes) {
       // ---------------------------------------------------------- odd CTA: forward readiness
       // The even CTA's MMA reads this CTA's activation tile and operand half:
@@ -308,8 +439,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ decoders (each CTA)
-    // NACC groups of decode warps take alternate K-steps; within a group,
-    // thread u owns block jb of operand row `row` (forward: weight row,
+    // NACC groups of decode warps take alternate running steps; within a
+    // group, thread u owns block jb of operand row `row` (forward: weight row,
     // 128 per stage; dgrad: reduction row, BK per stage).
     const int dwarp = warp - 2;
     const int grp = dwarp / C::GROUP_WARPS;
@@ -318,18 +449,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row = u % DROWS;
     const int jb = u / DROWS;
     const int64_t kblocks = p.wK / kBlock;
-    auto fetch = [&](int i, BlockLoad &b) {
+    // Loads for K-step k of the current tile (operand columns nb0 ..) into
+    // registers; zero past the tile's weight steps.  The prefetch stays within
+    // a segment, so nothing is held across a segment's epilogue.
+    auto fetch = [&](int k, bool live, int nb0, BlockLoad &b) {
       b.lo = b.hi = make_uint4(0, 0, 0, 0);
       b.q = 0;
       b.S = 0.0f;
-      if (i >= p.nkb) return;
+      if (!live || k >= p.nkb) return;
       int64_t n, kb;
       if (DGRAD) {
-        n = static_cast<int64_t>(i) * BK + row;
+        n = static_cast<int64_t>(k) * BK + row;
         kb = nb0 / kBlock + jb;
       } else {
         n = nb0 + row;
-        kb = static_cast<int64_t>(i) * C::KH + jb;
+        kb = static_cast<int64_t>(k) * C::KH + jb;
       }
       if (n < p.wN && kb < kblocks) {
         const int64_t idx = n * kblocks + kb;
@@ -342,120 +476,281 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     // DENSE: the operand row's 64 weights of this thread's run, 8 x 16 bytes
     // (zero past the matrix), loaded one of the group's K-steps ahead.
-    auto fetch_dense = [&](int i, DenseLoad &d) {
+    auto fetch_dense = [&](int k, bool live, int nb0, DenseLoad &d) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) d.v[c] = make_uint4(0, 0, 0, 0);
-      if (i >= p.nkb) return;
-      int64_t n, k;
+      if (!live || k >= p.nkb) return;
+      int64_t n, kk;
       if (DGRAD) {
-        n = static_cast<int64_t>(i) * BK + row;
-        k = nb0 + 64 * jb;
+        n = static_cast<int64_t>(k) * BK + row;
+        kk = nb0 + 64 * jb;
       } else {
         n = nb0 + row;
-        k = static_cast<int64_t>(i) * BK + 64 * jb;
+        kk = static_cast<int64_t>(k) * BK + 64 * jb;
       }
-      if (n < p.wN && k < p.wK) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.wdense + n * p.wK + k);
+      if (n < p.wN && kk < p.wK) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.wdense + n * p.wK + kk);
 #pragma unroll
         for (int c = 0; c < 8; ++c) d.v[c] = __ldg(src + c);
       }
     };
     const float mu = DENSE ? 0.0f : dq_offset(tab);
-    BlockLoad bq[DENSE ? 1 : PREFETCH];       // this group's next PREFETCH K-steps
-    DenseLoad dnext;
-    if (DENSE) {
-      fetch_dense(grp, dnext);
-    } else {
-#pragma unroll
-      for (int j = 0; j < PREFETCH; ++j) fetch(grp + j * NACC, bq[j]);
-    }
     const uint32_t swz = row & 7;             // 128B swizzle of the operand
-    for (int i = grp; i < nsteps; i += NACC) {
-      const int sd = i % D_STAGES;
-      BlockLoad cur{};
-      DenseLoad dcur;
-      if (DENSE) {
-        dcur = dnext;
-        fetch_dense(i + NACC, dnext);
-      } else {
-        cur = bq[0];
-#pragma unroll
-        for (int j = 0; j + 1 < (DENSE ? 1 : PREFETCH); ++j) bq[j] = bq[j + 1];
-        fetch(i + PREFETCH * NACC, bq[(DENSE ? 1 : PREFETCH) - 1]);
-      }
-      if (i >= D_STAGES &&
-          !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
-        break;
-      const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
-      if (DENSE && i < p.nkb) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), dcur.v[c].x, dcur.v[c].y, dcur.v[c].z,
-                       dcur.v[c].w);
-      } else if (i < p.nkb) {
-        const float ap = block_constant(cur.q, cur.S, tab.qx, mu);
-        uint32_t LO[4], HI[4];
-        nf4_block_table(ap, tab, LO, HI);
-        const uint32_t words[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          uint32_t o[4];
-          nf4_lut8(words[w], LO, HI, o);
-          st_shared_v4(drow + ((static_cast<uint32_t>(w) ^ swz) << 4), o[0], o[1], o[2], o[3]);
-        }
-      } else {
-        // adapter weight slice in the same operand layout; zero past r / past the matrix
-        const int64_t base_r = static_cast<int64_t>(i - p.nkb) * BK + 64 * jb;
-        for (int c = 0; c < 8; ++c) {
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (DGRAD) {
-            const int64_t rr = static_cast<int64_t>(i - p.nkb) * BK + row;
-            const int64_t kk = nb0 + 64 * jb + 8 * c;
-            if (rr < p.r && kk < p.wK) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + rr * p.wK + kk));
-          } else {
-            const int64_t n = nb0 + row;
-            const int64_t rr = base_r + 8 * c;
-            if (n < p.wN && rr < p.r) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + n * p.r + rr));
-          }
-          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), v.x, v.y, v.z, v.w);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm->decoded[sd]);
-    }
-
-    // ------------------------------------------------------------ epilogue (each CTA, its rows)
-    const bool acc_ok = mbar_wait(&sm->acc_full, 0, kDrainLimit);
-    tc_fence_after();
     volatile int *abort_flag = &sm->abort_flag;
-    if (__all_sync(0xffffffffu, acc_ok && *abort_flag == 0)) {
-      // NACC 1: the two warps of a lane quarter split the 256 columns;
+    volatile int *sk_role = &sm->sk_role;
+    volatile int *sk_ok = &sm->sk_ok;
+    bool dead = false;                        // warp-uniform: this warp gave up waiting
+    for (int t = t_first, seg = 0; t <= t_last; ++t, ++seg) {
+      const Seg sg = segment(t);
+      const int i_end = sg.j0 + (sg.k_hi - sg.k_lo);
+      const int i_first = sg.j0 + (((grp - sg.j0) % NACC) + NACC) % NACC;
+      // this group's steps i = i_first, i_first + NACC, ... < i_end; K-step k = k_lo + i - j0
+      BlockLoad bq[DENSE ? 1 : PREFETCH];     // the group's next PREFETCH K-steps
+      DenseLoad dnext;
+      if (DENSE) {
+        fetch_dense(sg.k_lo + i_first - sg.j0, i_first < i_end, sg.nb0, dnext);
+      } else {
+#pragma unroll
+        for (int j = 0; j < PREFETCH; ++j)
+          fetch(sg.k_lo + i_first + j * NACC - sg.j0, i_first + j * NACC < i_end, sg.nb0, bq[j]);
+      }
+      for (int i = i_first; i < i_end && !dead; i += NACC) {
+        const int k = sg.k_lo + (i - sg.j0);
+        const int sd = i % D_STAGES;
+        BlockLoad cur{};
+        DenseLoad dcur;
+        if (DENSE) {
+          dcur = dnext;
+          fetch_dense(k + NACC, i + NACC < i_end, sg.nb0, dnext);
+        } else {
+          cur = bq[0];
+#pragma unroll
+          for (int j = 0; j + 1 < (DENSE ? 1 : PREFETCH); ++j) bq[j] = bq[j + 1];
+          fetch(k + PREFETCH * NACC, i + PREFETCH * NACC < i_end, sg.nb0, bq[(DENSE ? 1 : PREFETCH) - 1]);
+        }
+        if (i >= D_STAGES &&
+            !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm))) {
+          dead = true;
+          break;
+        }
+        const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
+        if (DENSE && k < p.nkb) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), dcur.v[c].x, dcur.v[c].y, dcur.v[c].z,
+                         dcur.v[c].w);
+        } else if (k < p.nkb) {
+          const float ap = block_constant(cur.q, cur.S, tab.qx, mu);
+          uint32_t LO[4], HI[4];
+          nf4_block_table(ap, tab, LO, HI);
+          const uint32_t words[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            uint32_t o[4];
+            nf4_lut8(words[w], LO, HI, o);
+            st_shared_v4(drow + ((static_cast<uint32_t>(w) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+          }
+        } else {
+          // adapter weight slice in the same operand layout; zero past r / past the matrix
+          const int64_t base_r = static_cast<int64_t>(k - p.nkb) * BK + 64 * jb;
+          for (int c = 0; c < 8; ++c) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (DGRAD) {
+              const int64_t rr = static_cast<int64_t>(k - p.nkb) * BK + row;
+              const int64_t kk = sg.nb0 + 64 * jb + 8 * c;
+              if (rr < p.r && kk < p.wK) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + rr * p.wK + kk));
+            } else {
+              const int64_t n = sg.nb0 + row;
+              const int64_t rr = base_r + 8 * c;
+              if (n < p.wN && rr < p.r) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + n * p.r + rr));
+            }
+            st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), v.x, v.y, v.z, v.w);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->decoded[sd]);
+      }
+
+      // ---------------------------------------------------------- segment epilogue (each CTA, its rows)
+      // Every decode warp passes here once per segment, also after giving up,
+      // so that the named barriers below always meet.
+      // epilogue geometry: warp quarter q reads TMEM lanes 32 q .. + 31;
+      // NACC 1: the two warps of a quarter split the 256 columns;
       // NACC 2: decode group g drains accumulator g (256 columns).
       const int quarter = warp & 3;
       const int acc = NACC == 1 ? 0 : (dwarp >> 2);
       const int col_begin = NACC == 1 ? (dwarp >> 2) * 128 : 0;
       const int nchunk = NACC == 1 ? 4 : 8;
-      const int64_t orow_i = mbase + 256 * acc + quarter * 32 + lane;
-      uint16_t *orow = p.out + orow_i * p.ldo;
-      for (int cc = 0; cc < nchunk; ++cc) {
-        const int col0 = col_begin + cc * 32;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + 256 * acc + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
-        tmem_ld_wait();
-        if (orow_i < p.M) {
-          const int64_t c0 = n0 + col0;
+      const int arow = quarter * 32 + lane;     // row of this CTA's accumulator
+      // A piece is laid out by thread: float4 group g (columns 4g .. 4g + 3) of
+      // lane l of warp quarter q of accumulator a at float4 index
+      // ((a * 4 + q) * 64 + g) * 32 + l, so that a warp writes and reads 512
+      // contiguous bytes per instruction.
+      constexpr int64_t kPart = static_cast<int64_t>(NACC) * 128 * 256;   // fp32 of one rank's piece
+      auto piece_at = [&](int un, int which) {
+        return reinterpret_cast<float4 *>(p.sk_part + (static_cast<int64_t>(un * 2 + which) * 2 + rank) * kPart) +
+               (acc * 4 + quarter) * 64 * 32 + lane;
+      };
+      // the final epilogue of the cluster's last tile stages its bf16 rows in the
+      // (then idle) activation ring: 64-column boxes of this warp's 32 rows
+      const uint32_t stage = smem_addr(a_ring) + dwarp * (NACC == 1 ? 8192 : 16384);
+      bool ok = false;
+      if (!dead) {
+        ok = mbar_wait(&sm->acc_full, seg & 1, kDrainLimit);
+        if (!ok) latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+      }
+      tc_fence_after();
+      ok = __all_sync(0xffffffffu, ok) && *abort_flag == 0;
+      // A tile shared by P stream-K units: the CTA that finishes its piece last
+      // adds the others' fp32 pieces to its own in piece order (the same sum
+      // whoever arrives last) and writes the tile; the others write their piece.
+      int P = 1, fu = 0;
+      int64_t tb_sk = 0;
+      if (t >= p.dp_tiles) {
+        tb_sk = static_cast<int64_t>(t - p.dp_tiles) * ns;
+        fu = sk_unit_of(p, tb_sk);
+        P = sk_unit_of(p, tb_sk + ns - 1) - fu + 1;
+      }
+      int role = 0;                           // 0 whole tile, 1 piece writer, 2 finisher, -1 nothing
+      if (P > 1) {
+        const int ti = (t - p.dp_tiles) * 2 + static_cast<int>(rank);
+        if (threadIdx.x == 64) *sk_role = ok ? atomicAdd(p.sk_count + ti, 1) : -1;
+        named_bar_sync(1, 32 * NUM_DEC_WARPS);
+        const int arrived = *sk_role;
+        role = arrived < 0 ? -1 : (arrived == P - 1 ? 2 : 1);
+        if (role == 1) {
+          float4 *dst = piece_at(unit, seg == 0 ? 0 : 1);
+          if (ok) {
+            for (int cc = 0; cc < nchunk; ++cc) {
+              const int col0 = col_begin + cc * 32;
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(tmem + 256 * acc + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                __stcg(dst + (col0 / 4 + j) * 32, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                              __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+            }
+          }
+          named_bar_sync(1, 32 * NUM_DEC_WARPS);
+          if (threadIdx.x == 64) red_release_gpu_add(p.sk_ready + ti, 1);
+        } else if (role == 2) {
+          if (threadIdx.x == 64) {
+            // the other pieces' CTAs have counted themselves in: they are running and
+            // write their pieces now, so this wait is short and cannot depend on a
+            // cluster that has not started
+            int good = 1;
+            if (ld_acquire_gpu(p.sk_ready + ti) < P - 1) {
+              const long long t0 = clock64();
+              while (ld_acquire_gpu(p.sk_ready + ti) < P - 1) {
+                if (static_cast<uint64_t>(clock64() - t0) > p.wait_limit) {
+                  latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+                  good = 0;
+                  break;
+                }
+              }
+            }
+            *sk_ok = good;
+          }
+          named_bar_sync(1, 32 * NUM_DEC_WARPS);
+          if (!*sk_ok) role = -1;
+        } else {
+          // every path passes two barriers, so that the role word is read by all
+          // before the next shared tile's arrival overwrites it
+          named_bar_sync(1, 32 * NUM_DEC_WARPS);
+        }
+      }
+      if (ok && (role == 0 || role == 2)) {
+        const int own = unit - fu;
+        const bool staged = seg + 1 == nseg;
+        const int64_t orow0 = static_cast<int64_t>(sg.mbase) + 256 * acc + quarter * 32;
+        for (int cc = 0; cc < nchunk; ++cc) {
+          const int col0 = col_begin + cc * 32;
+          uint32_t v[32];
+          if (role == 0) {
+            tmem_ld_32x32b_x32(tmem + 256 * acc + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
+            tmem_ld_wait();
+          } else {
+            // the pieces in order: this CTA's own from TMEM, the others' from the workspace
+            float sum[32];
+            for (int pc = 0; pc < P; ++pc) {
+              if (pc == own) {
+                tmem_ld_32x32b_x32(tmem + 256 * acc + (static_cast<uint32_t>(quarter * 32) << 16) + col0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sum[j] = pc == 0 ? __uint_as_float(v[j]) : sum[j] + __uint_as_float(v[j]);
+              } else {
+                const int un = fu + pc;
+                const float4 *src = piece_at(un, sk_begin(p.sk_steps, p.sk_units, un) >= tb_sk ? 0 : 1) + (col0 / 4) * 32;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  float4 f[4];
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) f[j] = __ldcg(src + (4 * h + j) * 32);
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const int e = 16 * h + 4 * j;
+                    sum[e] = pc == 0 ? f[j].x : sum[e] + f[j].x;
+                    sum[e + 1] = pc == 0 ? f[j].y : sum[e + 1] + f[j].y;
+                    sum[e + 2] = pc == 0 ? f[j].z : sum[e + 2] + f[j].z;
+                    sum[e + 3] = pc == 0 ? f[j].w : sum[e + 3] + f[j].w;
+                  }
+                }
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(sum[j]);
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          if (c0 + 32 <= p.n_out && (p.ldo & 7) == 0) {
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+          if (staged) {
+            // 128B-swizzled rows of a 32 x 64 box; one TMA store per box
+            const uint32_t box = stage + (cc >> 1) * 4096;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t c = static_cast<uint32_t>((cc & 1) * 4 + j);
+              st_shared_v4(box + lane * 128 + ((c ^ static_cast<uint32_t>(lane & 7)) << 4), pk[4 * j], pk[4 * j + 1],
+                           pk[4 * j + 2], pk[4 * j + 3]);
+            }
+            if (cc & 1) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              const int64_t x = static_cast<int64_t>(sg.n0) + col_begin + (cc >> 1) * 64;
+              if (lane == 0 && orow0 < p.M && x < p.n_out) {
+                tma_store_2d(&tm_out, box, static_cast<int>(x), static_cast<int>(orow0));
+                bulk_commit();
+              }
+            }
           } else {
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < p.n_out) orow[c0 + j] = static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1)));
+            const int64_t orow_i = orow0 + lane;
+            if (orow_i < p.M) {
+              uint16_t *orow = p.out + orow_i * p.ldo;
+              const int64_t c0 = sg.n0 + col0;
+              if (c0 + 32 <= p.n_out && (p.ldo & 7) == 0) {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              } else {
+                for (int j = 0; j < 32; ++j)
+                  if (c0 + j < p.n_out) orow[c0 + j] = static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1)));
+              }
+            }
           }
+        }
+        // the stores have read the staged rows before the CTA's shared memory is released
+        if (staged && lane == 0) bulk_wait_read<0>();
+      }
+      // the next segment's MMAs overwrite the accumulators once both CTAs have read them
+      if (seg + 1 < nseg) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(&sm->tmem_empty);
+          else
+            mbar_arrive_cluster(mapa_shared(smem_addr(&sm->tmem_empty), 0));
         }
       }
     }
@@ -470,16 +765,45 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+constexpr size_t kSkCounterBytes = 2 * 2 * kSkMaxUnits * sizeof(int);   // count and ready, per tile and rank
+
+// Clusters of this kernel that fit on the device at once (cached per device).
+template <typename Kern>
+int cluster_slots(Kern kern, cudaLaunchConfig_t cfg) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int v = cache[dev].load();
+  if (v == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    v = n > 0 ? n : -1;
+    cache[dev].store(v);
+  }
+  return v > 0 ? v : 0;
+}
+
 }  // namespace
 
+size_t pair_sk_workspace_bytes(int64_t M) {
+  const int64_t nacc = M > 2 * BM ? 2 : 1;
+  return kSkCounterBytes + static_cast<size_t>(kSkMaxUnits) * 2 * 2 * nacc * 128 * 256 * sizeof(float);
+}
+
 qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
-  CUtensorMap tm_act, tm_lact;
+  CUtensorMap tm_act, tm_lact, tm_out;
   const int64_t kred = a.dgrad ? a.wN : a.wK;
   const int64_t n_out = a.dgrad ? a.wK : a.wN;
   bool ok = make_tmap_2d(&tm_act, a.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kred, a.M, kred * 2, 64, BM,
                          CU_TENSOR_MAP_SWIZZLE_128B);
   ok = ok && make_tmap_2d(&tm_lact, a.lora_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.r, a.M,
                           static_cast<uint64_t>(a.r) * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  // the output, written from shared memory in 32-row x 64-column boxes
+  ok = ok && make_tmap_2d(&tm_out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, n_out, a.M,
+                          static_cast<uint64_t>(n_out) * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return QLORA_ERR_CUDA;
 
   Params p{};
@@ -504,11 +828,14 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   const int bk = nacc == 2 ? Cfg<2>::BK : Cfg<1>::BK;
   p.nkb = static_cast<int>(ceil_div(kred, bk));
   p.nls = static_cast<int>(ceil_div(a.r, bk));
+  p.ns = p.nkb + p.nls;
   p.num_m = static_cast<int>(ceil_div(a.M, 2 * BM * nacc));
   p.num_n = static_cast<int>(ceil_div(n_out, BN));
+  const int tiles = p.num_m * p.num_n;
+  p.dp_tiles = tiles;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * p.num_m * p.num_n));
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * tiles));
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
@@ -523,8 +850,30 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // Whole waves take one tile per cluster; the tiles of a last, partial wave
+    // have their K-steps split evenly over the cluster slots (stream-K), so
+    // that no slot idles while the others finish the tail.
+    const int mode = stream_k_mode();
+    const int slots = a.sk_ws && mode != QLORA_STREAM_K_OFF ? std::min(cluster_slots(kern, cfg), kSkMaxUnits) : 0;
+    const int tail = slots > 0 ? tiles % slots : 0;
+    const int64_t sk_steps = static_cast<int64_t>(tail) * p.ns;
+    const int units = static_cast<int>(std::min<int64_t>(slots, std::max<int64_t>(1, sk_steps / kSkMinSteps)));
+    const bool split = tail > 0 && (mode == QLORA_STREAM_K_ALWAYS ||
+                                    ceil_div(sk_steps, units) + kSkCostSteps < p.ns + kTileCostSteps);
+    if (split) {
+      p.dp_tiles = tiles - tail;
+      p.sk_steps = sk_steps;
+      p.sk_units = units;
+      p.sk_count = static_cast<int *>(a.sk_ws);
+      p.sk_ready = p.sk_count + 2 * kSkMaxUnits;
+      p.sk_part = reinterpret_cast<float *>(static_cast<char *>(a.sk_ws) + kSkCounterBytes);
+      cfg.gridDim = dim3(static_cast<unsigned>(2 * (p.dp_tiles + p.sk_units)));
+      e = cudaMemsetAsync(a.sk_ws, 0, kSkCounterBytes, st);
+      if (e != cudaSuccess) return e;
+    }
     prof_mark(kind, true, st);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, kern, tm_act, tm_lact, p, tab);
+    e = cudaLaunchKernelEx(&cfg, kern, tm_act, tm_lact, tm_out, p, tab);
     prof_mark(kind, false, st);
     return e;
   };

@@ -51,7 +51,7 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_weight *w, cons
                                                  const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y,
                                                  float *H_out, void *stream) {
   if (!w) return QLORA_ERR_INVALID_ARG;
-  const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, M, w->rows, w->cols, r);
+  const size_t need = qlora_workspace_min_bytes(QLORA_OP_FWD, M, w->rows, w->cols, r);
   if (need > qlora::kStaticScratchBytes) return QLORA_ERR_WORKSPACE;   // sizes beyond the static scratch
   void *scratch = qlora::static_scratch_ptr();
   if (!scratch) return QLORA_ERR_CUDA;

@@ -158,9 +158,18 @@ qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *
 #define QLORA_OP_FWD_DENSE 2
 #define QLORA_OP_BWD_DENSE 3
 
-/* Workspace bytes the linear calls need for the given sizes (0 never means
- * "no workspace" for the linear; it is at least 256). */
+/* Workspace bytes for the linear calls at the given sizes, with every kernel
+ * path enabled (0 never means "no workspace" for the linear; it is at least
+ * 256).  When the fused GEMMs run on CTA pairs (M > 128, or a dense weight)
+ * the last part of this workspace holds the stream-K tail of those GEMMs: the
+ * fp32 pieces of output tiles that several clusters share when the tiles do
+ * not fill whole waves of the device (up to 80 MB for M > 256).  That part is
+ * optional: a workspace of qlora_workspace_min_bytes() bytes or more is
+ * accepted, and below qlora_workspace_bytes() the GEMMs run without the tail
+ * split (same results to rounding, slower when the last wave is partial).
+ * Returns 0 for an unknown op or sizes below 1. */
 size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
+size_t qlora_workspace_min_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
 
 /* qlora_linear_fwd -- Y = X W'^T + s (X A^T) B^T   (W' = dequantized base).
  * ("QLoRA" Abstract; "Where the memory goes".)
@@ -169,7 +178,8 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
  *   r      : 8 <= r <= 256, r % 8 == 0;  s : the adapter scale alpha / r (finite).
  *   Y      : device bf16 [M, N] (output).
  *   H_out  : optional device fp32 [M, r]; receives H = X A^T for the backward.
- *   ws     : device workspace of ws_bytes >= qlora_workspace_bytes(FWD, ...).
+ *   ws     : device workspace, 16-byte aligned, of ws_bytes >= qlora_workspace_min_bytes(FWD, ...)
+ *            (qlora_workspace_bytes(FWD, ...) for the stream-K tail); QLORA_ERR_WORKSPACE below.
  * N % 8 == 0.  M >= 1.  M <= 16 runs the memory-bound dequant-GEMV path; larger M runs the
  * tensor-core fused dequant-GEMM with the adapter term as an extra K segment of
  * the same accumulation.  fp32 accumulation; Y rounded once to bf16. */
@@ -245,9 +255,10 @@ qlora_status qlora_linear_bwd_materialized(qlora_materialize_fn materialize, voi
  *   QLORA_STATIC_SCRATCH_BYTES array inside the library, held on every GPU that
  *   loads the library until the process exits; the call allocates and frees
  *   nothing.
- *   Returns QLORA_ERR_WORKSPACE when qlora_workspace_bytes(QLORA_OP_FWD, M, N,
- *   K, r) exceeds QLORA_STATIC_SCRATCH_BYTES (e.g. M = 8192, r = 64 fits;
- *   M = 8192, r = 256 does not).
+ *   Returns QLORA_ERR_WORKSPACE when qlora_workspace_min_bytes(QLORA_OP_FWD,
+ *   M, N, K, r) exceeds QLORA_STATIC_SCRATCH_BYTES (e.g. M = 8192, r = 64 fits;
+ *   M = 8192, r = 256 does not); the fused GEMM runs without its stream-K tail
+ *   when the full workspace does not fit.
  *   The first call on a device looks up the array's device address; make that
  *   first call before any stream capture.  Every call shares the one array
  *   (it keeps the previous call's contents; nothing needs clearing), so calls
@@ -332,6 +343,21 @@ const char *qlora_status_string(qlora_status st);
 /* Upper bound, in GPU clock cycles, on every pipeline wait inside the
  * library's kernels (default 2e9, about one second).  Returns the old value. */
 uint64_t qlora_set_wait_limit(uint64_t cycles);
+
+/* When the fused GEMM's pair tiles leave a last, partial wave of cluster slots,
+ * the K-steps of those tiles can be split evenly over all slots (stream-K; the
+ * clusters sharing a tile add their fp32 pieces in a fixed order, so results
+ * repeat bit for bit).  Each split costs its clusters about 33 K-steps of
+ * drain, piece traffic and refill (measured on B200), so AUTO splits only when
+ * a cluster's share plus that cost is shorter than a whole tile plus its own
+ * fill and drain (about 8 K-steps); ALWAYS splits whenever the last wave is
+ * partial; OFF never splits.  The split needs the workspace's optional tail
+ * (qlora_workspace_bytes).  Returns the previous mode, or -1 (mode unchanged)
+ * for an unknown one.  Process-wide; takes effect at the next launch. */
+#define QLORA_STREAM_K_OFF 0
+#define QLORA_STREAM_K_AUTO 1
+#define QLORA_STREAM_K_ALWAYS 2
+int qlora_set_stream_k(int mode);
 
 /* Self-test of the bounded wait: launches one block that waits on a barrier
  * nothing ever signals, with a bound of `cycles`.  The wait must give up and

@@ -61,6 +61,42 @@ def test_workspace_sizes_positive_and_monotone():
     assert q.workspace_bytes(7, 1, 1, 1, 1) == 0
 
 
+def test_stream_k_mode_round_trip():
+    lib = q.load()
+    assert lib.qlora_set_stream_k(q.STREAM_K_ALWAYS) == q.STREAM_K_AUTO       # the default
+    assert lib.qlora_set_stream_k(q.STREAM_K_OFF) == q.STREAM_K_ALWAYS
+    assert lib.qlora_set_stream_k(3) == -1 and lib.qlora_set_stream_k(-1) == -1
+    assert q.set_stream_k(q.STREAM_K_AUTO) == q.STREAM_K_OFF
+    with pytest.raises(ValueError):
+        q.set_stream_k(7)
+
+
+def test_stream_k_region_is_an_optional_tail():
+    """The fused GEMMs' stream-K pieces are the last, optional part of the
+    workspace: present for the CTA-pair kernel (M > 128, or a dense weight),
+    at most 2 x 2 x 80 fp32 tile pieces of 128 x 256 x NACC per CTA, absent for the
+    few-token and one-CTA paths."""
+    lib = q.load()
+    piece = 128 * 256 * 4
+    for op in range(4):
+        for M, nacc in ((4096, 2), (300, 2), (200, 1)):
+            full = lib.qlora_workspace_bytes(op, M, 4096, 4096, 64)
+            low = lib.qlora_workspace_min_bytes(op, M, 4096, 4096, 64)
+            assert 256 <= low < full
+            assert full - low >= 80 * 2 * 2 * nacc * piece
+            assert full - low <= 80 * 2 * 2 * nacc * piece + 4096
+    for op in (q.QLORA_OP_FWD, q.QLORA_OP_BWD):
+        for M in (1, 16, 128):     # few-token or one-CTA kernels: no tail
+            assert lib.qlora_workspace_min_bytes(op, M, 4096, 4096, 64) == lib.qlora_workspace_bytes(op, M, 4096, 4096, 64)
+    for op in (q.QLORA_OP_FWD_DENSE, q.QLORA_OP_BWD_DENSE):
+        assert lib.qlora_workspace_min_bytes(op, 16, 4096, 4096, 64) < lib.qlora_workspace_bytes(op, 16, 4096, 4096, 64)
+    assert lib.qlora_workspace_min_bytes(9, 1, 1, 1, 1) == 0
+    # below the minimum the calls refuse, with nothing launched
+    for op, call in ((q.QLORA_OP_FWD, _fwd), (q.QLORA_OP_BWD, _bwd)):
+        ws_min = lib.qlora_workspace_min_bytes(op, 4096, 4096, 4096, 64)
+        assert call(_w(4096, 4096), M=4096, r=64, wsb=ws_min - 1) == 7
+
+
 # ---------------------------------------------------------------- host-side argument errors
 
 FAKE = 0x10000          # 16-byte aligned, never dereferenced: validation fails first
