@@ -146,6 +146,10 @@ struct Smem {
 constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + static_cast<int>(sizeof(Smem));
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(A_STAGES * A_BYTES >= NUM_DEC_WARPS * 16384, "epilogue staging fits the activation ring");
+static_assert(Cfg<1>::D_STAGES > 1 && Cfg<2>::D_STAGES > 2 &&
+                  Cfg<1>::D_BYTES >= NUM_DEC_WARPS / (Cfg<1>::D_STAGES - 1) * 4096 &&
+                  Cfg<2>::D_BYTES >= NUM_DEC_WARPS / (Cfg<2>::D_STAGES - 2) * 4096,
+              "a 4 KB staging box per decode warp fits the operand slots left after the early steps");
 
 // Tile t of the grouped raster: consecutive tiles walk kGroupM M-pairs before
 // moving to the next N tile, so a wave reuses both operands from L2.
@@ -215,69 +219,65 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();                              // 0 = even (MMA-issuing) CTA
   const int ns = p.ns;
-  // The cluster's K-steps in the linear (tile, K-step) order: a whole tile in
-  // the full waves, a contiguous share of the remaining tiles' steps for a
-  // stream-K unit.  Running step j of the cluster is linear step G0 + j.
-  int64_t G0, G1;
-  int unit = -1;
+  // The cluster's work, as consecutive segments: whole tiles cid, cid + C,
+  // cid + 2C, ... (C = nclus clusters; round i takes tiles iC .. iC + C - 1, in
+  // raster order), then, for a stream-K unit, its contiguous share [G0, G1) of the
+  // shared tiles' K-steps (tail-linear order: shared tile ts, step k at ts ns + k).
+  // Running step j of the cluster counts all its K-steps in that order.
+  const int nclus = static_cast<int>(gridDim.x >> 1);
   const int cid = static_cast<int>(blockIdx.x >> 1);
-  if (cid < p.dp_tiles) {
-    G0 = static_cast<int64_t>(cid) * ns;
-    G1 = G0 + ns;
-  } else {
-    unit = cid - p.dp_tiles;
-    const int64_t base = static_cast<int64_t>(p.dp_tiles) * ns;
-    G0 = base + sk_begin(p.sk_steps, p.sk_units, unit);
-    G1 = base + sk_begin(p.sk_steps, p.sk_units, unit + 1);
+  const int n_dp = cid < p.dp_tiles ? (p.dp_tiles - cid + nclus - 1) / nclus : 0;
+  const int unit = cid < p.sk_units ? cid : -1;
+  int64_t G0 = 0, G1 = 0;
+  int sk_t0 = 0, n_sk = 0;
+  if (unit >= 0) {
+    G0 = sk_begin(p.sk_steps, p.sk_units, unit);
+    G1 = sk_begin(p.sk_steps, p.sk_units, unit + 1);
+    sk_t0 = static_cast<int>(G0 / ns);
+    n_sk = static_cast<int>((G1 - 1) / ns) - sk_t0 + 1;
   }
-  const int t_first = static_cast<int>(G0 / ns);
-  const int t_last = static_cast<int>((G1 - 1) / ns);
-  const int nseg = t_last - t_first + 1;
-  const int nsteps = static_cast<int>(G1 - G0);
+  const int nseg = n_dp + n_sk;
+  const int nsteps = n_dp * ns + static_cast<int>(G1 - G0);
 
-  // One segment = the cluster's K-steps [k_lo, k_hi) of tile t; j0 is the
-  // running index of its first step.  This CTA's rows of accumulator a are
-  // mbase + 256 a .. + 127, its operand columns nb0 .. + 127.
+  // Segment s: K-steps [k_lo, k_hi) of tile t; j0 is the running index of its
+  // first step.  This CTA's rows of accumulator a are mbase + 256 a .. + 127,
+  // its operand columns nb0 .. + 127.
   struct Seg {
-    int k_lo, k_hi, j0;
+    int t, k_lo, k_hi, j0;
     int mbase, n0, nb0;      // M, N and K are below 2^31
   };
-  auto segment = [&](int t) {
+  auto segment = [&](int s) {
     Seg sg;
-    const int64_t tb = static_cast<int64_t>(t) * ns;
-    sg.k_lo = static_cast<int>((G0 > tb ? G0 : tb) - tb);
-    sg.k_hi = static_cast<int>((G1 < tb + ns ? G1 : tb + ns) - tb);
-    sg.j0 = static_cast<int>(tb + sg.k_lo - G0);
+    if (s < n_dp) {
+      sg.t = cid + s * nclus;
+      sg.k_lo = 0;
+      sg.k_hi = ns;
+      sg.j0 = s * ns;
+    } else {
+      const int ts = sk_t0 + (s - n_dp);
+      const int64_t tb = static_cast<int64_t>(ts) * ns;
+      sg.t = p.dp_tiles + ts;
+      sg.k_lo = static_cast<int>((G0 > tb ? G0 : tb) - tb);
+      sg.k_hi = static_cast<int>((G1 < tb + ns ? G1 : tb + ns) - tb);
+      sg.j0 = n_dp * ns + static_cast<int>(tb + sg.k_lo - G0);
+    }
     int pm, pn;
-    tile_coords(p, t, pm, pn);
+    tile_coords(p, sg.t, pm, pn);
     sg.mbase = pm * (2 * BM * NACC) + static_cast<int>(rank) * BM;
     sg.n0 = pn * BN;
     sg.nb0 = sg.n0 + static_cast<int>(rank) * 128;
     return sg;
   };
-  // Follows running steps forward (never back) across tile boundaries.
+  auto seg_end = [](const Seg &sg) { return sg.j0 + (sg.k_hi - sg.k_lo); };
+  // Follows running steps forward (never back) across segments.
   struct Cursor {
-    int t;
-    int64_t tb;
-    int mbase, nb0;
+    int s;
+    Seg sg;
   };
-  auto cursor_start = [&]() {
-    const Seg sg = segment(t_first);
-    return Cursor{t_first, static_cast<int64_t>(t_first) * ns, sg.mbase, sg.nb0};
-  };
-  // tile-local K-step of running step j (j < nsteps), moving the cursor to its tile
+  // tile-local K-step of running step j (j < nsteps), moving the cursor to its segment
   auto cursor_at = [&](Cursor &c, int j) {
-    const int64_t G = G0 + j;
-    if (G >= c.tb + ns) {
-      do {
-        ++c.t;
-        c.tb += ns;
-      } while (G >= c.tb + ns);
-      const Seg sg = segment(c.t);
-      c.mbase = sg.mbase;
-      c.nb0 = sg.nb0;
-    }
-    return static_cast<int>(G - c.tb);
+    while (j >= seg_end(c.sg)) c.sg = segment(++c.s);
+    return c.sg.k_lo + (j - c.sg.j0);
   };
 
   if (threadIdx.x == 0) {
@@ -313,9 +313,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int issued = 0;
       bool stop = false;
-      Cursor pf = cursor_start();            // the step A_STAGES ahead, for the L2 prefetch
-      for (int t = t_first; t <= t_last && !stop; ++t) {
-        const Seg sg = segment(t);
+      Cursor pf{0, segment(0)};              // the step A_STAGES ahead, for the L2 prefetch
+      for (int s = 0; s < nseg && !stop; ++s) {
+        const Seg sg = segment(s);
         for (int k = sg.k_lo; k < sg.k_hi; ++k) {
           const int i = sg.j0 + (k - sg.k_lo);
           const int s = i % A_STAGES;
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (kpf < p.nkb)
               for (int a = 0; a < NACC; ++a)
                 for (int kh = 0; kh < C::KH; ++kh)
-                  tma_prefetch_2d(&tm_act, kpf * BK + 64 * kh, static_cast<int>(pf.mbase + 256 * a));
+                  tma_prefetch_2d(&tm_act, kpf * BK + 64 * kh, static_cast<int>(pf.sg.mbase + 256 * a));
           }
           issued = i + 1;
         }
@@ -365,8 +365,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, 0, DGRAD ? 1 : 0);
       int commits = 0;
       bool stop = false;
-      for (int t = t_first, seg = 0; t <= t_last && !stop; ++t, ++seg) {
-        const Seg sg = segment(t);
+      for (int seg = 0; seg < nseg && !stop; ++seg) {
+        const Seg sg = segment(seg);
         // a later tile overwrites the accumulators: both CTAs must have read them
         if (seg > 0 && !wait_or_abort<true>(&sm->tmem_empty, (seg - 1) & 1, p, sm)) {
           stop = true;
@@ -500,76 +500,106 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *sk_role = &sm->sk_role;
     volatile int *sk_ok = &sm->sk_ok;
     bool dead = false;                        // warp-uniform: this warp gave up waiting
-    for (int t = t_first, seg = 0; t <= t_last; ++t, ++seg) {
-      const Seg sg = segment(t);
-      const int i_end = sg.j0 + (sg.k_hi - sg.k_lo);
-      const int i_first = sg.j0 + (((grp - sg.j0) % NACC) + NACC) % NACC;
-      // this group's steps i = i_first, i_first + NACC, ... < i_end; K-step k = k_lo + i - j0
-      BlockLoad bq[DENSE ? 1 : PREFETCH];     // the group's next PREFETCH K-steps
-      DenseLoad dnext;
-      if (DENSE) {
-        fetch_dense(sg.k_lo + i_first - sg.j0, i_first < i_end, sg.nb0, dnext);
+    // Writes the operand of running step i (K-step k of the tile whose operand
+    // columns start at nb0) once its ring slot is free; false if the wait gave up.
+    auto emit = [&](int i, int k, int nb0, const BlockLoad &cur, const DenseLoad &dcur) {
+      const int sd = i % D_STAGES;
+      if (i >= D_STAGES &&
+          !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
+        return false;
+      const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
+      if (DENSE && k < p.nkb) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), dcur.v[c].x, dcur.v[c].y, dcur.v[c].z,
+                       dcur.v[c].w);
+      } else if (k < p.nkb) {
+        const float ap = block_constant(cur.q, cur.S, tab.qx, mu);
+        uint32_t LO[4], HI[4];
+        nf4_block_table(ap, tab, LO, HI);
+        const uint32_t words[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          uint32_t o[4];
+          nf4_lut8(words[w], LO, HI, o);
+          st_shared_v4(drow + ((static_cast<uint32_t>(w) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+        }
       } else {
-#pragma unroll
-        for (int j = 0; j < PREFETCH; ++j)
-          fetch(sg.k_lo + i_first + j * NACC - sg.j0, i_first + j * NACC < i_end, sg.nb0, bq[j]);
+        // adapter weight slice in the same operand layout; zero past r / past the matrix
+        const int64_t base_r = static_cast<int64_t>(k - p.nkb) * BK + 64 * jb;
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (DGRAD) {
+            const int64_t rr = static_cast<int64_t>(k - p.nkb) * BK + row;
+            const int64_t kk = static_cast<int64_t>(nb0) + 64 * jb + 8 * c;
+            if (rr < p.r && kk < p.wK) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + rr * p.wK + kk));
+          } else {
+            const int64_t n = static_cast<int64_t>(nb0) + row;
+            const int64_t rr = base_r + 8 * c;
+            if (n < p.wN && rr < p.r) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + n * p.r + rr));
+          }
+          st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), v.x, v.y, v.z, v.w);
+        }
       }
-      for (int i = i_first; i < i_end && !dead; i += NACC) {
-        const int k = sg.k_lo + (i - sg.j0);
-        const int sd = i % D_STAGES;
-        BlockLoad cur{};
-        DenseLoad dcur;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm->decoded[sd]);
+      return true;
+    };
+    bool ahead = false;                       // this group's first step of the segment was written early
+    for (int seg = 0; seg < nseg; ++seg) {
+      const Seg sg = segment(seg);
+      const int t = sg.t;
+      const int i_end = seg_end(sg);
+      const int i_first = sg.j0 + (((grp - sg.j0) % NACC) + NACC) % NACC + (ahead ? NACC : 0);
+      // this group's steps i = i_first, i_first + NACC, ... < i_end; K-step k = k_lo + i - j0
+      {
+        BlockLoad bq[DENSE ? 1 : PREFETCH];   // the group's next PREFETCH K-steps
+        DenseLoad dnext;
         if (DENSE) {
-          dcur = dnext;
-          fetch_dense(k + NACC, i + NACC < i_end, sg.nb0, dnext);
+          fetch_dense(sg.k_lo + i_first - sg.j0, i_first < i_end, sg.nb0, dnext);
         } else {
-          cur = bq[0];
 #pragma unroll
-          for (int j = 0; j + 1 < (DENSE ? 1 : PREFETCH); ++j) bq[j] = bq[j + 1];
-          fetch(k + PREFETCH * NACC, i + PREFETCH * NACC < i_end, sg.nb0, bq[(DENSE ? 1 : PREFETCH) - 1]);
+          for (int j = 0; j < PREFETCH; ++j)
+            fetch(sg.k_lo + i_first + j * NACC - sg.j0, i_first + j * NACC < i_end, sg.nb0, bq[j]);
         }
-        if (i >= D_STAGES &&
-            !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm))) {
-          dead = true;
-          break;
-        }
-        const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
-        if (DENSE && k < p.nkb) {
+        for (int i = i_first; i < i_end && !dead; i += NACC) {
+          const int k = sg.k_lo + (i - sg.j0);
+          BlockLoad cur{};
+          DenseLoad dcur;
+          if (DENSE) {
+            dcur = dnext;
+            fetch_dense(k + NACC, i + NACC < i_end, sg.nb0, dnext);
+          } else {
+            cur = bq[0];
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), dcur.v[c].x, dcur.v[c].y, dcur.v[c].z,
-                         dcur.v[c].w);
-        } else if (k < p.nkb) {
-          const float ap = block_constant(cur.q, cur.S, tab.qx, mu);
-          uint32_t LO[4], HI[4];
-          nf4_block_table(ap, tab, LO, HI);
-          const uint32_t words[8] = {cur.lo.x, cur.lo.y, cur.lo.z, cur.lo.w, cur.hi.x, cur.hi.y, cur.hi.z, cur.hi.w};
-#pragma unroll
-          for (int w = 0; w < 8; ++w) {
-            uint32_t o[4];
-            nf4_lut8(words[w], LO, HI, o);
-            st_shared_v4(drow + ((static_cast<uint32_t>(w) ^ swz) << 4), o[0], o[1], o[2], o[3]);
+            for (int j = 0; j + 1 < (DENSE ? 1 : PREFETCH); ++j) bq[j] = bq[j + 1];
+            fetch(k + PREFETCH * NACC, i + PREFETCH * NACC < i_end, sg.nb0, bq[(DENSE ? 1 : PREFETCH) - 1]);
           }
-        } else {
-          // adapter weight slice in the same operand layout; zero past r / past the matrix
-          const int64_t base_r = static_cast<int64_t>(k - p.nkb) * BK + 64 * jb;
-          for (int c = 0; c < 8; ++c) {
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (DGRAD) {
-              const int64_t rr = static_cast<int64_t>(k - p.nkb) * BK + row;
-              const int64_t kk = sg.nb0 + 64 * jb + 8 * c;
-              if (rr < p.r && kk < p.wK) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + rr * p.wK + kk));
-            } else {
-              const int64_t n = sg.nb0 + row;
-              const int64_t rr = base_r + 8 * c;
-              if (n < p.wN && rr < p.r) v = __ldg(reinterpret_cast<const uint4 *>(p.lora_w + n * p.r + rr));
-            }
-            st_shared_v4(drow + ((static_cast<uint32_t>(c) ^ swz) << 4), v.x, v.y, v.z, v.w);
-          }
+          if (!emit(i, k, sg.nb0, cur, dcur)) dead = true;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->decoded[sd]);
+      }
+      // The next tile's first step of this group goes into its slot now, while
+      // the tensor cores finish this tile: the next tile's MMAs can start as
+      // soon as the accumulators are read.  (The slots of the following
+      // D_STAGES - NACC steps hold the epilogue's staging meanwhile.)
+      ahead = false;
+      if (seg + 1 < nseg && !dead) {
+        const Seg nx = segment(seg + 1);
+        const int ia = nx.j0 + (((grp - nx.j0) % NACC) + NACC) % NACC;
+        if (ia < seg_end(nx)) {
+          const int ka = nx.k_lo + (ia - nx.j0);
+          BlockLoad b{};
+          DenseLoad d;
+          if (DENSE)
+            fetch_dense(ka, true, nx.nb0, d);
+          else
+            fetch(ka, true, nx.nb0, b);
+          if (emit(ia, ka, nx.nb0, b, d))
+            ahead = true;
+          else
+            dead = true;
+        }
       }
 
       // ---------------------------------------------------------- segment epilogue (each CTA, its rows)
@@ -592,9 +622,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         return reinterpret_cast<float4 *>(p.sk_part + (static_cast<int64_t>(un * 2 + which) * 2 + rank) * kPart) +
                (acc * 4 + quarter) * 64 * 32 + lane;
       };
-      // the final epilogue of the cluster's last tile stages its bf16 rows in the
-      // (then idle) activation ring: 64-column boxes of this warp's 32 rows
-      const uint32_t stage = smem_addr(a_ring) + dwarp * (NACC == 1 ? 8192 : 16384);
+      // The bf16 rows go out through shared memory in 32 x 64 boxes, one TMA
+      // store each: after the cluster's last tile all of a warp's boxes fit in
+      // the (then idle) activation ring; before that the ring holds the next
+      // tile's activations, and each warp takes one 4 KB box in the operand
+      // slots of the D_STAGES - NACC steps after the early ones, reused box by box.
+      const bool last = seg + 1 == nseg;
+      constexpr int kStageSlots = D_STAGES - NACC;
+      constexpr int kWarpsPerSlot = NUM_DEC_WARPS / kStageSlots;
+      const uint32_t stage =
+          last ? smem_addr(a_ring) + dwarp * (NACC == 1 ? 8192 : 16384)
+               : smem_addr(d_ring + ((i_end + NACC + dwarp / kWarpsPerSlot) % D_STAGES) * D_BYTES) +
+                     (dwarp % kWarpsPerSlot) * 4096;
       bool ok = false;
       if (!dead) {
         ok = mbar_wait(&sm->acc_full, seg & 1, kDrainLimit);
@@ -620,7 +659,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int arrived = *sk_role;
         role = arrived < 0 ? -1 : (arrived == P - 1 ? 2 : 1);
         if (role == 1) {
-          float4 *dst = piece_at(unit, seg == 0 ? 0 : 1);
+          float4 *dst = piece_at(unit, seg == n_dp ? 0 : 1);
           if (ok) {
             for (int cc = 0; cc < nchunk; ++cc) {
               const int col0 = col_begin + cc * 32;
@@ -663,7 +702,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok && (role == 0 || role == 2)) {
         const int own = unit - fu;
-        const bool staged = seg + 1 == nseg;
         const int64_t orow0 = static_cast<int64_t>(sg.mbase) + 256 * acc + quarter * 32;
         for (int cc = 0; cc < nchunk; ++cc) {
           const int col0 = col_begin + cc * 32;
@@ -705,9 +743,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          if (staged) {
+          {
             // 128B-swizzled rows of a 32 x 64 box; one TMA store per box
-            const uint32_t box = stage + (cc >> 1) * 4096;
+            const uint32_t box = last ? stage + (cc >> 1) * 4096 : stage;
+            if (!last && cc > 0 && (cc & 1) == 0) {
+              if (lane == 0) bulk_wait_read<0>();   // the previous box has been read out
+              __syncwarp();
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t c = static_cast<uint32_t>((cc & 1) * 4 + j);
@@ -723,27 +765,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 bulk_commit();
               }
             }
-          } else {
-            const int64_t orow_i = orow0 + lane;
-            if (orow_i < p.M) {
-              uint16_t *orow = p.out + orow_i * p.ldo;
-              const int64_t c0 = sg.n0 + col0;
-              if (c0 + 32 <= p.n_out && (p.ldo & 7) == 0) {
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-              } else {
-                for (int j = 0; j < 32; ++j)
-                  if (c0 + j < p.n_out) orow[c0 + j] = static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1)));
-              }
-            }
           }
         }
-        // the stores have read the staged rows before the CTA's shared memory is released
-        if (staged && lane == 0) bulk_wait_read<0>();
+        // the stores have read the staged rows before the shared memory is reused or released
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
       }
-      // the next segment's MMAs overwrite the accumulators once both CTAs have read them
-      if (seg + 1 < nseg) {
+      if (!last) {
+        // every warp's boxes are out of the operand slots before they are decoded into
+        named_bar_sync(1, 32 * NUM_DEC_WARPS);
+        // the next segment's MMAs overwrite the accumulators once both CTAs have read them
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -835,7 +866,7 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   p.dp_tiles = tiles;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * tiles));
+  cfg.gridDim = dim3(2);        // set per launch below (the occupancy query reads the rest)
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
@@ -851,12 +882,14 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   auto go = [&](auto kern) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    // Whole waves take one tile per cluster; the tiles of a last, partial wave
-    // have their K-steps split evenly over the cluster slots (stream-K), so
-    // that no slot idles while the others finish the tail.
+    // Persistent clusters: as many as fit on the device at once (one per tile
+    // when that is not known), each taking tiles cid, cid + C, ...  The tiles
+    // of a last, partial round can instead have their K-steps split evenly over
+    // all clusters (stream-K), so that no cluster idles while others finish.
+    const int slots = std::min(cluster_slots(kern, cfg), kSkMaxUnits);
+    int clusters = slots > 0 ? std::min(tiles, slots) : tiles;
     const int mode = stream_k_mode();
-    const int slots = a.sk_ws && mode != QLORA_STREAM_K_OFF ? std::min(cluster_slots(kern, cfg), kSkMaxUnits) : 0;
-    const int tail = slots > 0 ? tiles % slots : 0;
+    const int tail = slots > 0 && a.sk_ws && mode != QLORA_STREAM_K_OFF ? tiles % slots : 0;
     const int64_t sk_steps = static_cast<int64_t>(tail) * p.ns;
     const int units = static_cast<int>(std::min<int64_t>(slots, std::max<int64_t>(1, sk_steps / kSkMinSteps)));
     const bool split = tail > 0 && (mode == QLORA_STREAM_K_ALWAYS ||
@@ -868,10 +901,11 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
       p.sk_count = static_cast<int *>(a.sk_ws);
       p.sk_ready = p.sk_count + 2 * kSkMaxUnits;
       p.sk_part = reinterpret_cast<float *>(static_cast<char *>(a.sk_ws) + kSkCounterBytes);
-      cfg.gridDim = dim3(static_cast<unsigned>(2 * (p.dp_tiles + p.sk_units)));
+      clusters = p.dp_tiles > 0 ? slots : units;
       e = cudaMemsetAsync(a.sk_ws, 0, kSkCounterBytes, st);
       if (e != cudaSuccess) return e;
     }
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
     prof_mark(kind, true, st);
     e = cudaLaunchKernelEx(&cfg, kern, tm_act, tm_lact, tm_out, p, tab);
     prof_mark(kind, false, st);
