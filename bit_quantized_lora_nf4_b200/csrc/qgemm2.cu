@@ -146,10 +146,6 @@ struct Smem {
 constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + static_cast<int>(sizeof(Smem));
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(A_STAGES * A_BYTES >= NUM_DEC_WARPS * 16384, "epilogue staging fits the activation ring");
-static_assert(Cfg<1>::D_STAGES > 1 && Cfg<2>::D_STAGES > 2 &&
-                  Cfg<1>::D_BYTES >= NUM_DEC_WARPS / (Cfg<1>::D_STAGES - 1) * 4096 &&
-                  Cfg<2>::D_BYTES >= NUM_DEC_WARPS / (Cfg<2>::D_STAGES - 2) * 4096,
-              "a 4 KB staging box per decode warp fits the operand slots left after the early steps");
 
 // Tile t of the grouped raster: consecutive tiles walk kGroupM M-pairs before
 // moving to the next N tile, so a wave reuses both operands from L2.
@@ -629,7 +625,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       // slots of the D_STAGES - NACC steps after the early ones, reused box by box.
       const bool last = seg + 1 == nseg;
       constexpr int kStageSlots = D_STAGES - NACC;
-      constexpr int kWarpsPerSlot = NUM_DEC_WARPS / kStageSlots;
+      constexpr int kWarpsPerSlot = (NUM_DEC_WARPS + kStageSlots - 1) / kStageSlots;
+      static_assert(kStageSlots >= 1 && kWarpsPerSlot * 4096 <= D_BYTES, "staging boxes fit the free operand slots");
       const uint32_t stage =
           last ? smem_addr(a_ring) + dwarp * (NACC == 1 ? 8192 : 16384)
                : smem_addr(d_ring + ((i_end + NACC + dwarp / kWarpsPerSlot) % D_STAGES) * D_BYTES) +
