@@ -214,6 +214,11 @@ __global__ void __launch_bounds__(TTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  // The next kernel on the stream may be scheduled once every CTA of this grid
+  // has passed here (so it never takes a slot one of these still needs); no
+  // global memory is touched before the previous kernel's writes are visible.
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -416,13 +421,15 @@ cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st) {
     cfg.blockDim = dim3(TTHREADS);
     cfg.dynamicSmemBytes = TSMEM;
     cfg.stream = st;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;   // the splits of one tile: one cluster
     at[0].val.clusterDim.x = 1;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = fused ? static_cast<unsigned>(a.splits) : 1u;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the previous kernel's tail
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p);
   };
   prof_mark(kProfLora, true, st);

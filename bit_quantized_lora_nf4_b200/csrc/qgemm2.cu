@@ -303,6 +303,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync_all();        // peer barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  // The next kernel on the stream may be scheduled once every CTA of this grid
+  // has passed here (so it never takes a slot one of these still needs); no
+  // global memory is touched before the previous kernel's writes are visible.
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ activation TMA (each CTA)
@@ -867,13 +872,15 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;             // the occupancy query sees the cluster shape only
   const Nf4Table tab = a.tab;
   const int kind = a.dgrad ? kProfGemmDgrad : kProfGemmFwd;
   auto go = [&](auto kern) {
@@ -904,7 +911,9 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
     }
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
     prof_mark(kind, true, st);
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, tm_act, tm_lact, tm_out, p, tab);
+    cfg.numAttrs = 1;
     prof_mark(kind, false, st);
     return e;
   };
