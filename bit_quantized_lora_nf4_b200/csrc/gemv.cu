@@ -545,6 +545,10 @@ __global__ void __maxnreg__(QLORA_GEMV_MAXNREG) gemv_kernel(const __grid_constan
                                                           const GemvParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The next kernel on the stream may be scheduled once every CTA has passed
+  // here; nothing is read before the previous kernel's writes are visible.
+  griddep_launch_dependents();
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool h_cta = static_cast<int>(blockIdx.x) < p.JT * p.HS;
   const int gw = (static_cast<int>(blockIdx.x) - p.JT * p.HS) * GV_WARPS + warp;   // weight warp index
@@ -690,11 +694,13 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
   cfg.blockDim = dim3(GV_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // launch during the previous kernel's tail
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kern, tm, p) != cudaSuccess) return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
