@@ -23,6 +23,9 @@
 //   3. Every warp finishes tiles t = w, w + W, ...: adds the tile's pieces in
 //      piece order (a fixed order, so results are deterministic), adds
 //      (s H) B^T with two more mma chains, stores bf16 Y.
+#include <atomic>
+#include <random>
+
 #include "decode.cuh"
 #include "internal.h"
 
@@ -87,34 +90,51 @@ __device__ __forceinline__ float ldg_once_f32(const float *p) {
 }
 
 
-// Grid-wide barrier of a cooperative launch.  The driver gives every such
-// launch a barrier word (its address is in %envreg1:%envreg2, high:low; the
-// word follows a 4-byte size field).  Each CTA adds 1, CTA 0 adds
-// 2^31 - (CTAs - 1): one full round adds 2^31, so the top bit flips once per
-// barrier and the low bits return to where they were.  A CTA waits, for at
-// most `limit` cycles, until the top bit differs from the value it saw when it
-// arrived; on timeout it latches the status and goes on.
-__device__ __forceinline__ void grid_barrier(int *status, uint64_t limit) {
+// Grid-wide barrier of the cooperative launch (every CTA resident), on a 64-bit
+// word of the workspace: the high half holds the launch's epoch (unique per
+// launch in this process, from a random start), the low half the arrivals of
+// that launch so far.  CTA 0 stamps the word with its epoch and a zero count
+// when the kernel starts (grid_barrier_open); every CTA counts itself in with an
+// atomic add only once it sees that epoch, so whatever the word held before
+// (an earlier launch's tag, or never written) is neither counted nor needs
+// clearing.  Round `round` (1, 2, ...) is complete once round x CTAs have
+// arrived.  Each CTA's writes before the barrier are published by its thread
+// 0 (after the CTA barrier) with a GPU-scope fence before it counts itself in.
+// Waits are bounded; on timeout the status is latched and the CTA goes on.
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const unsigned long long *p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void grid_barrier_open(unsigned long long *word, uint32_t epoch) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(word, static_cast<unsigned long long>(epoch) << 32);
+}
+__device__ __forceinline__ void grid_barrier(unsigned long long *word, uint32_t epoch, uint32_t round, int *status,
+                                             uint64_t limit) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t lo, hi;
-    asm volatile("mov.u32 %0, %%envreg2;" : "=r"(lo));
-    asm volatile("mov.u32 %0, %%envreg1;" : "=r"(hi));
-    unsigned int *word = reinterpret_cast<unsigned int *>(((static_cast<uint64_t>(hi) << 32) | lo) + 4);
-    const unsigned int n = gridDim.x * gridDim.y * gridDim.z;
-    const unsigned int add = (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) ? 0x80000000u - (n - 1) : 1u;
-    unsigned int old;
-    asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(word), "r"(add) : "memory");
+    const uint32_t n = gridDim.x * gridDim.y * gridDim.z;
+    __threadfence();
     const long long t0 = clock64();
-    while (true) {
-      unsigned int cur;
-      asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(word) : "memory");
-      if ((cur ^ old) & 0x80000000u) break;
+    bool ok = true;
+    while ((ld_acquire_gpu_u64(word) >> 32) != epoch) {   // the launch's stamp is in place
       if (static_cast<uint64_t>(clock64() - t0) > limit) {
-        latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
+        ok = false;
         break;
       }
     }
+    if (ok) {
+      atomicAdd(word, 1ull);
+      while (true) {
+        const uint64_t w = ld_acquire_gpu_u64(word);
+        if ((w >> 32) == epoch && static_cast<uint32_t>(w) >= round * n) break;
+        if (static_cast<uint64_t>(clock64() - t0) > limit) {
+          ok = false;
+          break;
+        }
+      }
+    }
+    if (!ok) latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
   }
   __syncthreads();
 }
@@ -140,6 +160,8 @@ struct GemvParams {
   uint16_t *sh_lo;          //              and the remainder
   float *pieces;            // [T][P][M][16] tile sums, one per weight warp that touches the tile
   float *hpart;             // [JT][HS][8 NT][16] partial H of the H CTAs (HS > 1)
+  unsigned long long *bar;  // grid barrier word (see grid_barrier)
+  uint32_t epoch;           // this launch's tag on it
   int M, r, r16;
   int JT, HS;               // H CTAs: blockIdx.x < JT * HS, adapter tile blockIdx.x / HS, K split blockIdx.x % HS
   int G;                    // weight warps (CTA blockIdx.x - JT HS holds weight warps 8 (that) .. +7)
@@ -549,6 +571,7 @@ __global__ void __maxnreg__(QLORA_GEMV_MAXNREG) gemv_kernel(const __grid_constan
   // here; nothing is read before the previous kernel's writes are visible.
   griddep_launch_dependents();
   griddep_wait();
+  grid_barrier_open(p.bar, p.epoch);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool h_cta = static_cast<int>(blockIdx.x) < p.JT * p.HS;
   const int gw = (static_cast<int>(blockIdx.x) - p.JT * p.HS) * GV_WARPS + warp;   // weight warp index
@@ -588,10 +611,10 @@ __global__ void __maxnreg__(QLORA_GEMV_MAXNREG) gemv_kernel(const __grid_constan
     if (weight) weight_role<NT, XS>(&tm_codes, p, x, cs, gw, a, b);
   }
 
-  grid_barrier(p.status, p.wait_limit);   // pieces (and s H or its partial sums) complete and visible
+  grid_barrier(p.bar, p.epoch, 1, p.status, p.wait_limit);   // pieces (and s H or its partial sums) complete and visible
   if (p.HS > 1) {
     h_finish<NT>(p);
-    grid_barrier(p.status, p.wait_limit);
+    grid_barrier(p.bar, p.epoch, 2, p.status, p.wait_limit);
   }
   finish_role<NT>(p);
 }
@@ -614,7 +637,7 @@ struct GemvLayout {
   int NT, r16, JT, HS, P;
   int64_t T, S, U, G_max;
   bool fits32;
-  size_t off_pieces, off_hpart, off_hi, off_lo, total;
+  size_t off_pieces, off_hpart, off_hi, off_lo, off_bar, total;
 };
 
 GemvLayout gemv_layout(int64_t M, int64_t N, int64_t K, int r) {
@@ -643,8 +666,16 @@ GemvLayout gemv_layout(int64_t M, int64_t N, int64_t K, int r) {
   off += align256(sh);
   L.off_lo = off;
   off += align256(sh);
+  L.off_bar = off;
+  off += 256;
   L.total = off;
   return L;
+}
+
+// A tag for each launch's barrier word: consecutive from a random start.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> next{static_cast<uint32_t>(std::random_device{}())};
+  return next.fetch_add(1);
 }
 
 template <int NT>
@@ -686,7 +717,7 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
   GemvParams p{a.X, a.absmax_q, a.group_scale, a.A, a.B, a.s, a.Y, a.H_out,
                reinterpret_cast<uint16_t *>(ws + L.off_hi), reinterpret_cast<uint16_t *>(ws + L.off_lo),
                reinterpret_cast<float *>(ws + L.off_pieces), reinterpret_cast<float *>(ws + L.off_hpart),
-               static_cast<int>(a.M), a.r, L.r16, L.JT, L.HS, static_cast<int>(G), static_cast<int>(L.S),
+               reinterpret_cast<unsigned long long *>(ws + L.off_bar), next_epoch(), static_cast<int>(a.M), a.r, L.r16, L.JT, L.HS, static_cast<int>(G), static_cast<int>(L.S),
                static_cast<int>(L.U), static_cast<int>(L.T), L.P, xs ? xs_row_bytes(KB) : 0, a.wN, a.wK, status,
                wait_limit(), a.tab};
   cudaLaunchConfig_t cfg{};

@@ -90,3 +90,28 @@ def test_gemv_matches_tensor_core_path(lib):
     Y16, _ = q.linear_fwd(w, X[:16].contiguous(), A, B, d["s"])
     torch.cuda.synchronize()
     assert rel(f64(Y16), f64(Y17[:16])) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_any_workspace_contents(lib, M):
+    """The grid barrier's word lives in the caller's workspace and is tagged per
+    launch: whatever an unused workspace holds (random bytes, all ones, zeros),
+    the result is the same bits, call after call."""
+    case = qi.LinearCase(f"ws_{M}", M, 1032, 2112, 24, 16.0, 61 + M)
+    d = qi.make_linear(case, with_dy=False)
+    w = q.quantize_nf4(d["W"].cuda())
+    X, A, B = d["X"].cuda(), d["A"].cuda(), d["B"].cuda()
+    need = q.workspace_bytes(q.QLORA_OP_FWD, M, case.N, case.K, case.r)
+    g = torch.Generator(device="cpu").manual_seed(5)
+    fills = [torch.randint(0, 256, (need,), dtype=torch.uint8, generator=g).cuda(),
+             torch.full((need,), 255, dtype=torch.uint8, device="cuda"),
+             torch.zeros(need, dtype=torch.uint8, device="cuda")]
+    outs = []
+    for ws in fills:
+        for _ in range(2):
+            Y, _ = q.linear_fwd(w, X, A, B, case.s, save_h=False, workspace=ws)
+            outs.append(Y.clone())
+    torch.cuda.synchronize()
+    assert q.device_status() == 0
+    for Y in outs[1:]:
+        assert torch.equal(Y, outs[0])
