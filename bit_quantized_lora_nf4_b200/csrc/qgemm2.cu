@@ -133,9 +133,10 @@ struct Params {
 struct Smem {
   uint64_t afull[A_STAGES];        // activation tile landed (TMA)
   uint64_t aempty[A_STAGES];       // the pair's MMAs reading it completed (multicast commit)
-  uint64_t dfree[MAX_D_STAGES];        // the pair's MMAs reading the operand half completed (multicast commit)
+  uint64_t dfree[MAX_D_STAGES];        // the pair's MMAs reading the operand half completed (multicast commit;
+                                       // aempty serves both rings when they share their depth)
   uint64_t decoded[MAX_D_STAGES];      // this CTA's decode group wrote the operand half
-  uint64_t peer_decoded[MAX_D_STAGES]; // even CTA only: the odd CTA's A tile and operand half are ready
+  uint64_t peer_decoded[MAX_D_STAGES]; // even CTA only: the step's inputs are ready (see kMerged)
   uint64_t acc_full;               // the pair's accumulation completed (multicast commit)
   uint64_t tmem_empty;             // even CTA: both CTAs read the accumulators (next tile may start)
   uint32_t tmem_base;
@@ -207,6 +208,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   using C = Cfg<NACC>;
   constexpr int BK = C::BK;
   constexpr int D_STAGES = C::D_STAGES;
+  // When both rings have the same depth, the even CTA's inputs of a step all
+  // arrive on one barrier, peer_decoded[s]: its activation TMA (bytes), its
+  // decode group's warps and the odd CTA's forwarder, so the MMA issuer tests
+  // one barrier per step instead of three (each test costs the issuer time in
+  // which the tensor pipe can run dry).  Otherwise peer_decoded carries the
+  // forwarder alone and afull / decoded are tested too.
+  constexpr bool kMerged = A_STAGES == D_STAGES;
   constexpr int D_BYTES = C::D_BYTES;
   uint8_t *d_ring = smem + A_STAGES * A_BYTES;
   Smem *sm = reinterpret_cast<Smem *>(d_ring + D_RING);
@@ -214,6 +222,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();                              // 0 = even (MMA-issuing) CTA
+  const bool merged_even = kMerged && rank == 0;
   const int ns = p.ns;
   // The cluster's work, as consecutive segments: whole tiles cid, cid + C,
   // cid + 2C, ... (C = nclus clusters; round i takes tiles iC .. iC + C - 1, in
@@ -284,7 +293,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < D_STAGES; ++s) {
       mbar_init(&sm->dfree[s], 1);
       mbar_init(&sm->decoded[s], C::GROUP_WARPS);
-      mbar_init(&sm->peer_decoded[s], 1);
+      mbar_init(&sm->peer_decoded[s], kMerged ? C::GROUP_WARPS + 2 : 1);
     }
     mbar_init(&sm->acc_full, 1);
     mbar_init(&sm->tmem_empty, 2 * NUM_DEC_WARPS);
@@ -325,22 +334,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             stop = true;
             break;
           }
+          uint64_t *full = merged_even ? &sm->peer_decoded[s] : &sm->afull[s];
           uint8_t *st = a_ring + s * A_BYTES;
           // atom column (t, kh) of the stage at (t * KH + kh) * HALF
           if (k < p.nkb) {
-            mbar_arrive_expect_tx(&sm->afull[s], A_BYTES);
+            mbar_arrive_expect_tx(full, A_BYTES);
             for (int a = 0; a < NACC; ++a)
               for (int kh = 0; kh < C::KH; ++kh)
-                tma_load_2d(st + (a * C::KH + kh) * HALF, &tm_act, &sm->afull[s], k * BK + 64 * kh,
+                tma_load_2d(st + (a * C::KH + kh) * HALF, &tm_act, full, k * BK + 64 * kh,
                             static_cast<int>(sg.mbase + 256 * a));
           } else {
             const int ls = k - p.nkb;
             const int rem = p.r - ls * BK;
             const int halves = rem > 64 ? C::KH : 1;
-            mbar_arrive_expect_tx(&sm->afull[s], NACC * halves * HALF);
+            mbar_arrive_expect_tx(full, NACC * halves * HALF);
             for (int a = 0; a < NACC; ++a)
               for (int kh = 0; kh < halves; ++kh)
-                tma_load_2d(st + (a * C::KH + kh) * HALF, &tm_lact, &sm->afull[s], ls * BK + 64 * kh,
+                tma_load_2d(st + (a * C::KH + kh) * HALF, &tm_lact, full, ls * BK + 64 * kh,
                             static_cast<int>(sg.mbase + 256 * a));
           }
           // the tile A_STAGES steps further on goes to L2 now: its load waits for a free
@@ -358,7 +368,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       for (int j = (issued > A_STAGES ? issued - A_STAGES : 0); j < issued; ++j)
-        mbar_wait(&sm->afull[j % A_STAGES], (j / A_STAGES) & 1, kDrainLimit);
+        mbar_wait(merged_even ? &sm->peer_decoded[j % A_STAGES] : &sm->afull[j % A_STAGES], (j / A_STAGES) & 1,
+                  kDrainLimit);
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
@@ -379,9 +390,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t pa = (i / A_STAGES) & 1, pd = (i / D_STAGES) & 1;
           // the three inputs of the step probed together (their latencies overlap);
           // the bounded waits only when one of them is not there yet
-          const bool ready = mbar_test(smem_addr(&sm->afull[sa]), pa) & mbar_test(smem_addr(&sm->decoded[sd]), pd) &
-                             mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd);
-          if (!ready) {
+          if (kMerged) {
+            if (!mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd) &&
+                !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
+              stop = true;
+              break;
+            }
+          } else if (!(mbar_test(smem_addr(&sm->afull[sa]), pa) & mbar_test(smem_addr(&sm->decoded[sd]), pd) &
+                       mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd))) {
             if ((!mbar_test(smem_addr(&sm->afull[sa]), pa) && !wait_or_abort<false>(&sm->afull[sa], pa, p, sm)) ||
                 (!mbar_test(smem_addr(&sm->decoded[sd]), pd) && !wait_or_abort<false>(&sm->decoded[sd], pd, p, sm)) ||
                 !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
@@ -397,17 +413,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int rem = p.r - (k - p.nkb) * BK;
             nk = rem >= BK ? BK / 16 : (rem + 15) / 16;
           }
+          // descriptors of the stage's first slice; a slice's start address adds
+          // its byte offset / 16 to the low field (no carry: shared memory < 256 KB)
+          const uint64_t adesc0 = sdesc_sw128(a_base, 16, 1024);
+          const uint64_t bdesc0 = DGRAD ? sdesc_sw128(d_base, BK * 128, 1024) : sdesc_sw128(d_base, 16, 1024);
           for (int kk = 0; kk < nk; ++kk) {
             const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-            const uint64_t bdesc = DGRAD ? sdesc_sw128(d_base + kk * 2048, BK * 128, 1024)
-                                         : sdesc_sw128(d_base + koff, 16, 1024);
+            const uint64_t bdesc = bdesc0 + ((DGRAD ? kk * 2048u : koff) >> 4);
             for (int a = 0; a < NACC; ++a) {
-              const uint64_t adesc = sdesc_sw128(a_base + a * C::KH * HALF + koff, 16, 1024);
+              const uint64_t adesc = adesc0 + ((a * C::KH * HALF + koff) >> 4);
               tc_mma_bf16_pair(tmem + 256 * a, adesc, bdesc, IDESC, (k != sg.k_lo || kk != 0) ? 1u : 0u);
             }
           }
+          // both rings' slot of the step is free once its MMAs complete: one commit
+          // when they share their depth
           tc_commit_pair_mc(&sm->aempty[sa], 0x3);
-          tc_commit_pair_mc(&sm->dfree[sd], 0x3);
+          if (!kMerged) tc_commit_pair_mc(&sm->dfree[sd], 0x3);
         }
         if (stop) break;
         tc_commit_pair_mc(&sm->acc_full, 0x3);
@@ -505,8 +526,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // columns start at nb0) once its ring slot is free; false if the wait gave up.
     auto emit = [&](int i, int k, int nb0, const BlockLoad &cur, const DenseLoad &dcur) {
       const int sd = i % D_STAGES;
-      if (i >= D_STAGES &&
-          !__all_sync(0xffffffffu, wait_or_abort<false>(&sm->dfree[sd], ((i / D_STAGES) & 1) ^ 1, p, sm)))
+      if (i >= D_STAGES && !__all_sync(0xffffffffu, wait_or_abort<false>(kMerged ? &sm->aempty[sd] : &sm->dfree[sd],
+                                                                         ((i / D_STAGES) & 1) ^ 1, p, sm)))
         return false;
       const uint32_t drow = smem_addr(d_ring + sd * D_BYTES) + jb * (DROWS * 128) + row * 128;
       if (DENSE && k < p.nkb) {
@@ -544,7 +565,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm->decoded[sd]);
+      if (lane == 0) mbar_arrive(merged_even ? &sm->peer_decoded[sd] : &sm->decoded[sd]);
       return true;
     };
     bool ahead = false;                       // this group's first step of the segment was written early
