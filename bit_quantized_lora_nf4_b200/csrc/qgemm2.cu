@@ -9,7 +9,7 @@
 // tensor-core work per SM as the one-CTA kernel: the decode (ALU) cost per MMA
 // flop halves.
 //
-// Per CTA (320 threads, K-step 128 = two NF4 blocks per weight row), with
+// Per CTA (352 threads, K-step 128 = two NF4 blocks per weight row), with
 // separate rings so that neither load latency nor decode sits on the MMA's
 // critical path:
 //   warp 0      TMA: activation tiles (128 rows x 128, two 128B-swizzled
@@ -26,6 +26,8 @@
 //               operand halves (K-major for the forward, MN-major for dgrad;
 //               the byte address is the same formula in both).  After the last
 //               step the decode warps drain this CTA's TMEM.
+//   warp 10     even CTA, two accumulators: the second MMA issuer (accumulator
+//               1; warp 1's lane issues accumulator 0).
 // The MMA issuer probes its three inputs (activation tile, own operand half,
 // the odd CTA's forwarded readiness) together without blocking and falls back
 // to bounded waits only for one that is not complete; the odd CTA's forwarder
@@ -69,7 +71,10 @@ constexpr int HALF = 16384;                 // one 128-row x 64-column swizzled 
 constexpr int D_RING = QLORA_PAIR_D_RING_KB * 1024;   // decoded-operand stages
 constexpr int PREFETCH = QLORA_PAIR_PREFETCH;
 constexpr int NUM_DEC_WARPS = 8;
-constexpr int THREADS = 32 * (2 + NUM_DEC_WARPS);
+// warp 0 TMA, warp 1 MMA issuer (accumulator 0) / forwarder, warps 2-9 decode,
+// warp 10 the second MMA issuer (accumulator 1) when a CTA holds two
+constexpr int ISSUER2_WARP = 2 + NUM_DEC_WARPS;
+constexpr int THREADS = 32 * (3 + NUM_DEC_WARPS);
 
 // NACC = accumulators per CTA: the pair tile covers 256 * NACC rows.  With
 // NACC = 2 every decoded operand half feeds two MMAs (rows 0-255 and 256-511
@@ -288,14 +293,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_STAGES; ++s) {
       mbar_init(&sm->afull[s], 1);
-      mbar_init(&sm->aempty[s], 1);
+      mbar_init(&sm->aempty[s], NACC);   // one commit per issuer
     }
     for (int s = 0; s < D_STAGES; ++s) {
       mbar_init(&sm->dfree[s], 1);
       mbar_init(&sm->decoded[s], C::GROUP_WARPS);
       mbar_init(&sm->peer_decoded[s], kMerged ? C::GROUP_WARPS + 2 : 1);
     }
-    mbar_init(&sm->acc_full, 1);
+    mbar_init(&sm->acc_full, NACC);
     mbar_init(&sm->tmem_empty, 2 * NUM_DEC_WARPS);
     sm->abort_flag = 0;
     fence_mbar_init();
@@ -317,6 +322,80 @@ __global__ void __launch_bounds__(THREADS, 1)
   // global memory is touched before the previous kernel's writes are visible.
   griddep_launch_dependents();
   griddep_wait();
+
+  // Pair MMA issuer (even CTA): accumulators [acc_lo, acc_hi) of every step.
+  // With two accumulators a second thread (warp ISSUER2_WARP) issues the other
+  // one, so one issuer's barrier tests and commits overlap the other's MMAs
+  // and the tensor pipe is not left idle between steps; each commits its own
+  // MMAs (the slot and accumulator barriers count one arrival per issuer).
+  auto run_issuer = [&](int acc_lo, int acc_hi) {
+    constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, 0, DGRAD ? 1 : 0);
+    int commits = 0;
+    bool stop = false;
+    for (int seg = 0; seg < nseg && !stop; ++seg) {
+      const Seg sg = segment(seg);
+      // a later tile overwrites the accumulators: both CTAs must have read them
+      if (seg > 0 && !wait_or_abort<true>(&sm->tmem_empty, (seg - 1) & 1, p, sm)) {
+        stop = true;
+        break;
+      }
+      for (int k = sg.k_lo; k < sg.k_hi; ++k) {
+        const int i = sg.j0 + (k - sg.k_lo);
+        const int sa = i % A_STAGES, sd = i % D_STAGES;
+        const uint32_t pa = (i / A_STAGES) & 1, pd = (i / D_STAGES) & 1;
+        // the three inputs of the step probed together (their latencies overlap);
+        // the bounded waits only when one of them is not there yet
+        if (kMerged) {
+          if (!mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd) &&
+              !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
+            stop = true;
+            break;
+          }
+        } else if (!(mbar_test(smem_addr(&sm->afull[sa]), pa) & mbar_test(smem_addr(&sm->decoded[sd]), pd) &
+                     mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd))) {
+          if ((!mbar_test(smem_addr(&sm->afull[sa]), pa) && !wait_or_abort<false>(&sm->afull[sa], pa, p, sm)) ||
+              (!mbar_test(smem_addr(&sm->decoded[sd]), pd) && !wait_or_abort<false>(&sm->decoded[sd], pd, p, sm)) ||
+              !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
+            stop = true;
+            break;
+          }
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_addr(a_ring + sa * A_BYTES);
+        const uint32_t d_base = smem_addr(d_ring + sd * D_BYTES);
+        int nk = BK / 16;
+        if (k >= p.nkb) {
+          const int rem = p.r - (k - p.nkb) * BK;
+          nk = rem >= BK ? BK / 16 : (rem + 15) / 16;
+        }
+        // descriptors of the stage's first slice; a slice's start address adds
+        // its byte offset / 16 to the low field (no carry: shared memory < 256 KB)
+        const uint64_t adesc0 = sdesc_sw128(a_base, 16, 1024);
+        const uint64_t bdesc0 = DGRAD ? sdesc_sw128(d_base, BK * 128, 1024) : sdesc_sw128(d_base, 16, 1024);
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
+          const uint64_t bdesc = bdesc0 + ((DGRAD ? kk * 2048u : koff) >> 4);
+          for (int a = acc_lo; a < acc_hi; ++a) {
+            const uint64_t adesc = adesc0 + ((a * C::KH * HALF + koff) >> 4);
+            tc_mma_bf16_pair(tmem + 256 * a, adesc, bdesc, IDESC, (k != sg.k_lo || kk != 0) ? 1u : 0u);
+          }
+        }
+        // both rings' slot of the step is free once its MMAs complete: one commit
+        // per issuer when they share their depth
+        tc_commit_pair_mc(&sm->aempty[sa], 0x3);
+        if (!kMerged) tc_commit_pair_mc(&sm->dfree[sd], 0x3);
+      }
+      if (stop) break;
+      tc_commit_pair_mc(&sm->acc_full, 0x3);
+      ++commits;
+    }
+    if (stop) {
+      // given up: one more commit, and wait until it (every MMA issued) has
+      // completed, so that the accumulators are idle before teardown
+      tc_commit_pair_mc(&sm->acc_full, 0x3);
+      mbar_wait(&sm->acc_full, commits & 1, kDrainLimit);
+    }
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ activation TMA (each CTA)
@@ -374,72 +453,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------- pair MMA issuer (even CTA)
-      constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, 0, DGRAD ? 1 : 0);
-      int commits = 0;
-      bool stop = false;
-      for (int seg = 0; seg < nseg && !stop; ++seg) {
-        const Seg sg = segment(seg);
-        // a later tile overwrites the accumulators: both CTAs must have read them
-        if (seg > 0 && !wait_or_abort<true>(&sm->tmem_empty, (seg - 1) & 1, p, sm)) {
-          stop = true;
-          break;
-        }
-        for (int k = sg.k_lo; k < sg.k_hi; ++k) {
-          const int i = sg.j0 + (k - sg.k_lo);
-          const int sa = i % A_STAGES, sd = i % D_STAGES;
-          const uint32_t pa = (i / A_STAGES) & 1, pd = (i / D_STAGES) & 1;
-          // the three inputs of the step probed together (their latencies overlap);
-          // the bounded waits only when one of them is not there yet
-          if (kMerged) {
-            if (!mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd) &&
-                !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
-              stop = true;
-              break;
-            }
-          } else if (!(mbar_test(smem_addr(&sm->afull[sa]), pa) & mbar_test(smem_addr(&sm->decoded[sd]), pd) &
-                       mbar_test_cluster(smem_addr(&sm->peer_decoded[sd]), pd))) {
-            if ((!mbar_test(smem_addr(&sm->afull[sa]), pa) && !wait_or_abort<false>(&sm->afull[sa], pa, p, sm)) ||
-                (!mbar_test(smem_addr(&sm->decoded[sd]), pd) && !wait_or_abort<false>(&sm->decoded[sd], pd, p, sm)) ||
-                !wait_or_abort<true>(&sm->peer_decoded[sd], pd, p, sm)) {
-              stop = true;
-              break;
-            }
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_addr(a_ring + sa * A_BYTES);
-          const uint32_t d_base = smem_addr(d_ring + sd * D_BYTES);
-          int nk = BK / 16;
-          if (k >= p.nkb) {
-            const int rem = p.r - (k - p.nkb) * BK;
-            nk = rem >= BK ? BK / 16 : (rem + 15) / 16;
-          }
-          // descriptors of the stage's first slice; a slice's start address adds
-          // its byte offset / 16 to the low field (no carry: shared memory < 256 KB)
-          const uint64_t adesc0 = sdesc_sw128(a_base, 16, 1024);
-          const uint64_t bdesc0 = DGRAD ? sdesc_sw128(d_base, BK * 128, 1024) : sdesc_sw128(d_base, 16, 1024);
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-            const uint64_t bdesc = bdesc0 + ((DGRAD ? kk * 2048u : koff) >> 4);
-            for (int a = 0; a < NACC; ++a) {
-              const uint64_t adesc = adesc0 + ((a * C::KH * HALF + koff) >> 4);
-              tc_mma_bf16_pair(tmem + 256 * a, adesc, bdesc, IDESC, (k != sg.k_lo || kk != 0) ? 1u : 0u);
-            }
-          }
-          // both rings' slot of the step is free once its MMAs complete: one commit
-          // when they share their depth
-          tc_commit_pair_mc(&sm->aempty[sa], 0x3);
-          if (!kMerged) tc_commit_pair_mc(&sm->dfree[sd], 0x3);
-        }
-        if (stop) break;
-        tc_commit_pair_mc(&sm->acc_full, 0x3);
-        ++commits;
-      }
-      if (stop) {
-        // given up: one more commit, and wait until it (every MMA issued) has
-        // completed, so that the accumulators are idle before teardown
-        tc_commit_pair_mc(&sm->acc_full, 0x3);
-        mbar_wait(&sm->acc_full, commits & 1, kDrainLimit);
-      }
+      run_issuer(0, NACC == 2 ? 1 : NACC);
     } else if (rank != 0 && lane < kFwdLanes) {
       // ---------------------------------------------------------- odd CTA: forward readiness
       // The even CTA's MMA reads this CTA's activation tile and operand half:
@@ -459,6 +473,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive_cluster(mapa_shared(smem_addr(&sm->peer_decoded[sd]), 0));
       }
     }
+  } else if (warp == ISSUER2_WARP) {
+    if (NACC == 2 && lane == 0 && rank == 0) run_issuer(1, 2);
   } else {
     // ------------------------------------------------------------ decoders (each CTA)
     // NACC groups of decode warps take alternate running steps; within a
