@@ -3,42 +3,44 @@
 // Same computation as qgemm.cu ("Where the memory goes": the 4-bit base is
 // dequantized on the fly for each forward and backward pass; the adapter term
 // is the last K segment of the same accumulation), on a 256 x 256 output tile
-// per cluster of two CTAs.  The pair's MMA (M = 256, N = 256, K = 16) takes
-// its A rows from both CTAs (128 each) and its B columns from both CTAs (128
-// each), so every CTA decodes only half of the 256-row weight tile for the same
-// tensor-core work per SM as the one-CTA kernel: the decode (ALU) cost per MMA
-// flop halves.
+// per accumulator and cluster of two CTAs.  The pair's MMA (M = 256, N = 256,
+// K = 16) takes its A rows from both CTAs (128 each) and its B columns from
+// both CTAs (128 each), so every CTA decodes only half of the 256-row weight
+// tile for the same tensor-core work per SM as the one-CTA kernel; with two
+// accumulators per CTA (M > 256: a 512-row pair tile, K-step 64) each decoded
+// operand half feeds two MMAs, halving the decode cost per flop again.
 //
-// Per CTA (352 threads, K-step 128 = two NF4 blocks per weight row), with
+// Persistent: one cluster per co-resident slot walks its tiles (cid, cid + C,
+// ...) as segments, then, when the last round of tiles is split (stream-K),
+// its share of the shared tiles' K-steps.  Per CTA (352 threads), with
 // separate rings so that neither load latency nor decode sits on the MMA's
 // critical path:
-//   warp 0      TMA: activation tiles (128 rows x 128, two 128B-swizzled
-//               64-column boxes) into a 4-deep ring.
+//   warp 0      TMA: activation tiles (two 128B-swizzled 64-column boxes per
+//               accumulator) into a 4-deep ring, and an L2 prefetch of the
+//               tile four steps ahead.
 //   warp 1      TMEM allocation for the pair; in the even CTA one lane issues
-//               the pair MMA and commits to both CTAs' barriers (multicast);
-//               in the odd CTA two lanes, taking the K-steps in turn, forward
-//               "decoded" to the even CTA.
+//               the MMAs of accumulator 0 (of all, with one accumulator); in
+//               the odd CTA two lanes, taking the K-steps in turn, forward the
+//               readiness of its activation tile and operand half.
 //   warps 2-9   decode: thread (row = t % 128, j = t / 128) owns block j of its
 //               row.  Its 32 bytes of codes and its 8-bit constant are loaded
 //               from global memory into registers two of its K-steps ahead; it
 //               builds the block's 16-entry table, looks the codes up with byte
 //               permutes and writes 128 swizzled bytes into a 64 KB ring of
 //               operand halves (K-major for the forward, MN-major for dgrad;
-//               the byte address is the same formula in both).  After the last
-//               step the decode warps drain this CTA's TMEM.
-//   warp 10     even CTA, two accumulators: the second MMA issuer (accumulator
-//               1; warp 1's lane issues accumulator 0).
-// The MMA issuer probes its three inputs (activation tile, own operand half,
-// the odd CTA's forwarded readiness) together without blocking and falls back
-// to bounded waits only for one that is not complete; the odd CTA's forwarder
-// does the same with its two.  Measured per K-step on the LLaMA-7B projections
-// the issuer spends ~1150 clocks issuing MMAs and 70-350 clocks on its inputs,
-// almost all of it on the forwarded signal (one forwarding lane could not keep
-// ahead: its cluster-scope arrive takes ~1100 clocks; two lanes can); the
-// shallower operand ring and code
-// prefetch (fewer loads in flight) took 2-6 % off the step time, and an L2
-// prefetch of the activation tile A_STAGES steps ahead 4-5 % off the launches
-// whose large activation operand comes from DRAM.
+//               the byte address is the same formula in both).  At a tile's end
+//               each group first writes its step of the next tile, then drains
+//               its accumulator (TMEM -> bf16 boxes in shared memory -> TMA
+//               stores, or fp32 pieces for a shared tile).
+//   warp 10     even CTA, two accumulators: the MMA issuer of accumulator 1,
+//               so that one issuer's barrier test and commit overlap the
+//               other's MMAs.
+// In the even CTA a step's inputs (its activation bytes, its decode group, the
+// odd CTA's forwarded readiness) all arrive on one barrier per stage, and one
+// commit per issuer frees both rings' slots.  Measured per K-step on the
+// LLaMA-7B projections, MMA issue takes ~1070 clocks (paced by the tensor
+// pipe) against ~150 of barrier testing and ~57 of commits per issuer, and
+// late inputs are rare (3-10 % of steps).
 // Waits are bounded; on expiry a CTA latches QLORA_ERR_DEVICE_TIMEOUT, lets
 // its outstanding loads and the pair's MMAs land, frees TMEM and exits.
 #include <algorithm>
