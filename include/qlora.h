@@ -24,7 +24,8 @@
  *   - Every pointer argument named as "device" is CUDA device memory owned by
  *     the caller.  The library never allocates or frees device memory; the
  *     linear calls take a caller-provided workspace whose size is returned by
- *     qlora_workspace_bytes().
+ *     qlora_workspace_bytes() (at least qlora_workspace_min_bytes(); its
+ *     contents on entry do not matter).
  *   - bf16 tensors are passed as uint16_t bit patterns.  All tensors are dense
  *     row-major and every device pointer must be 16-byte aligned.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
@@ -200,7 +201,8 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int6
  * call stays stream-ordered and capturable) beside the dgrad GEMM.
  *   H_saved : optional device fp32 [M, r] from qlora_linear_fwd; NULL makes the
  *             call recompute X A^T.
- * Same shape rules as the forward; M >= 1. */
+ * Same shape rules as the forward; M >= 1.  Workspace as for the forward, with
+ * QLORA_OP_BWD. */
 qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY,
                               int64_t M, const uint16_t *A, const uint16_t *B, int r, float s,
                               const float *H_saved, uint16_t *dX, float *dA, float *dB,
@@ -216,7 +218,8 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, cons
  * decoded; the pair kernel serves every M).  With W' = qlora_dequantize(w) the
  * results equal the packed calls' bit for bit whenever those take the pair
  * kernel (M > 128).  Workspace: qlora_workspace_bytes(QLORA_OP_FWD_DENSE /
- * QLORA_OP_BWD_DENSE, M, N, K, r).  Shape rules as for the packed calls. */
+ * QLORA_OP_BWD_DENSE, M, N, K, r), at least qlora_workspace_min_bytes of the
+ * same op.  Shape rules as for the packed calls. */
 qlora_status qlora_linear_fwd_dense(const uint16_t *W, int64_t N, int64_t K, const uint16_t *X, int64_t M,
                                     const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *Y, float *H_out,
                                     void *ws, size_t ws_bytes, void *stream);
