@@ -49,6 +49,11 @@ FORMAT_NF4, FORMAT_FP4, FORMAT_INT4 = 0, 1, 2
 # Readings of the 8-bit block constants (QLORA_DQ_*): unsigned with no offset,
 # or signed around the tensor-wide mean constant (stored after the group scales).
 DQ_PLAIN, DQ_SIGNED = 0, 1
+# size of the library-owned scratch array of qlora_linear_fwd_noalloc (include/qlora.h)
+QLORA_STATIC_SCRATCH_BYTES = 8 << 20
+# element types the quantizer accepts (QLORA_DTYPE_F32 / QLORA_DTYPE_BF16)
+DTYPE_F32, DTYPE_BF16 = 0, 1
+_WEIGHT_DTYPES = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
 
 # Kernel kinds of the timing hook (qlora_profile_read).
 (PROF_ALL, PROF_GEMM_FWD, PROF_GEMM_DGRAD, PROF_LORA, PROF_QUANT, PROF_DEQUANT, PROF_GEMV, PROF_LQ_PRODUCT,
@@ -88,7 +93,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_codes_bytes": (sz, [i64, i64]),
         "qlora_absmax_bytes": (sz, [i64, i64]),
         "qlora_group_scale_bytes": (sz, [i64, i64]),
-        "qlora_quantize_nf4": (i32, [vp, wp, vp]),
+        "qlora_quantize_nf4": (i32, [vp, i32, wp, vp]),
         "qlora_dequantize": (i32, [wp, vp, vp]),
         "qlora_workspace_bytes": (sz, [i32, i64, i64, i64, i32]),
         "qlora_workspace_min_bytes": (sz, [i32, i64, i64, i64, i32]),
@@ -106,7 +111,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "qlora_linear_fwd_noalloc": (i32, [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp]),
         "qlora_group_scale_bytes_dq": (sz, [i64, i64, i32]),
         "qlora_quantize_workspace_bytes": (sz, [i64, i64, i32]),
-        "qlora_quantize_nf4_ws": (i32, [vp, wp, vp, sz, vp]),
+        "qlora_quantize_nf4_ws": (i32, [vp, i32, wp, vp, sz, vp]),
         "qlora_lq_workspace_bytes": (sz, [i64, i64, i32, i32, i32]),
         "qlora_lq_decompose": (i32, [vp, wp, vp, vp, i32, vp, i32, i32, i32, vp, vp, sz, vp]),
         "qlora_lq_quantize_residual": (i32, [vp, vp, vp, i32, wp, vp, sz, vp]),
@@ -227,13 +232,13 @@ def profile_read(kind: int):
 
 def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, format: int = FORMAT_NF4,
                  dq: int = DQ_PLAIN, workspace: torch.Tensor | None = None) -> NF4Weight:
-    """Quantize a contiguous fp32 CUDA tensor [rows, cols] (flat row-major) to a
-    4-bit table (NF4 unless `format` says otherwise) with block constants as
-    `dq` reads them (`out.format` / `out.dq` when `out` is given).  DQ_SIGNED
-    uses a workspace of qlora_quantize_workspace_bytes (allocated here when not
-    given)."""
+    """Quantize a contiguous fp32 or bf16 CUDA tensor [rows, cols] (flat
+    row-major) to a 4-bit table (NF4 unless `format` says otherwise) with block
+    constants as `dq` reads them (`out.format` / `out.dq` when `out` is given).
+    DQ_SIGNED uses a workspace of qlora_quantize_workspace_bytes (allocated here
+    when not given)."""
     lib = load()
-    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous()
+    assert W.is_cuda and W.dtype in _WEIGHT_DTYPES and W.is_contiguous()
     rows, cols = (W.shape[0], W[0].numel()) if W.dim() >= 2 else (1, W.numel())
     w = out if out is not None else NF4Weight.empty(rows, cols, W.device, format, dq)
     s = w.c_struct()
@@ -241,7 +246,8 @@ def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, format: int = FO
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.qlora_quantize_nf4_ws(_ptr(W), ctypes.byref(s), _ptr(workspace), nbytes, _stream()),
+    _check(lib.qlora_quantize_nf4_ws(_ptr(W), _WEIGHT_DTYPES[W.dtype], ctypes.byref(s), _ptr(workspace), nbytes,
+                                     _stream()),
            "qlora_quantize_nf4_ws")
     return w
 

@@ -46,8 +46,9 @@ class QLoRALinear(torch.nn.Module):
 
     @classmethod
     def from_float(cls, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float, format: int = 0):
-        """Quantize an fp32 weight [N, K] (on its device) and wrap it with adapters."""
-        return cls(quantize_nf4(W.float().contiguous(), format=format), A, B, alpha)
+        """Quantize an fp32 or bf16 weight [N, K] (on its device) and wrap it with adapters."""
+        Wq = W.contiguous() if W.dtype in (torch.float32, torch.bfloat16) else W.float().contiguous()
+        return cls(quantize_nf4(Wq, format=format), A, B, alpha)
 
     def _ws(self, op: int, M: int) -> torch.Tensor:
         key = (op, M)

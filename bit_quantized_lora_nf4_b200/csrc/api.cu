@@ -534,9 +534,9 @@ size_t qlora_workspace_min_bytes(int op, int64_t M, int64_t N, int64_t K, int r)
   return make_plan(base, M, N, K, r, !dense).min_total;
 }
 
-qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
-                                   void *stream) {
-  if (!W) return QLORA_ERR_INVALID_ARG;
+qlora_status qlora_quantize_nf4_ws(const void *W, int dtype, const qlora_nf4_weight *out, void *ws,
+                                   size_t ws_bytes, void *stream) {
+  if (!W || (dtype != QLORA_DTYPE_F32 && dtype != QLORA_DTYPE_BF16)) return QLORA_ERR_INVALID_ARG;
   QL_TRY(check_weight(out));
   if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
   const int64_t numel = out->rows * out->cols;
@@ -547,13 +547,13 @@ qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, 
   }
   int *status = device_status_ptr();
   if (!status) return QLORA_ERR_CUDA;
-  QL_CUDA(launch_quantize(W, numel, out->codes, out->absmax_q, out->group_scale, weight_table(out),
+  QL_CUDA(launch_quantize(W, dtype, numel, out->codes, out->absmax_q, out->group_scale, weight_table(out),
                           out->dq == QLORA_DQ_SIGNED ? ws : nullptr, status, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
 }
 
-qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream) {
-  return qlora_quantize_nf4_ws(W, out, nullptr, 0, stream);
+qlora_status qlora_quantize_nf4(const void *W, int dtype, const qlora_nf4_weight *out, void *stream) {
+  return qlora_quantize_nf4_ws(W, dtype, out, nullptr, 0, stream);
 }
 
 qlora_status qlora_dequantize(const qlora_nf4_weight *w, uint16_t *W_out, void *stream) {

@@ -49,8 +49,9 @@ bool make_tmap_2d(CUtensorMap *tm, const void *base, CUtensorMapDataType dtype, 
 // Quantizer.  tab.qx != 0 selects signed block constants; those need `ws`
 // (quantize_workspace_bytes(numel) bytes) and write mu to tab.offset.
 size_t quantize_workspace_bytes(int64_t numel);
-cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
-                            const Nf4Table &tab, void *ws, int *status, cudaStream_t st);
+// W holds QLORA_DTYPE_F32 or QLORA_DTYPE_BF16 elements.
+cudaError_t launch_quantize(const void *W, int dtype, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
+                            float *group_scale, const Nf4Table &tab, void *ws, int *status, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
                               int64_t numel, const Nf4Table &tab, uint16_t *out, cudaStream_t st);
 

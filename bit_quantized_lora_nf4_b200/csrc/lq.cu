@@ -912,7 +912,7 @@ qlora_status qlora_lq_quantize_residual(const float *W, const float *L1, const f
   float *E = wsp<float>(ws, p.E);
   run.residual(L1, L2, LqQuant{nullptr, nullptr, nullptr, tab}, E, nullptr);
   if (run.err == cudaSuccess)
-    run.err = launch_quantize(E, p.N * p.K, Q->codes, Q->absmax_q, Q->group_scale, tab,
+    run.err = launch_quantize(E, QLORA_DTYPE_F32, p.N * p.K, Q->codes, Q->absmax_q, Q->group_scale, tab,
                               Q->dq == QLORA_DQ_SIGNED ? wsp<void>(ws, p.qws) : nullptr, status, st);
   return run.err == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -964,7 +964,7 @@ qlora_status qlora_lq_decompose(const float *W, const qlora_nf4_weight *Q, float
   for (int t = 0; t < iters && run.err == cudaSuccess; ++t) {
     run.residual(L1, L2, none, E, nullptr);               // E = W - L1 L2
     if (run.err == cudaSuccess)
-      run.err = launch_quantize(E, p.N * p.K, Q->codes, Q->absmax_q, Q->group_scale, tab,
+      run.err = launch_quantize(E, QLORA_DTYPE_F32, p.N * p.K, Q->codes, Q->absmax_q, Q->group_scale, tab,
                                 Q->dq == QLORA_DQ_SIGNED ? wsp<void>(ws, p.qws) : nullptr, status, st);
     run.residual(L1, L2, quant, nullptr, part);           // before the rank-r step
     run.sum(part, p.res_ctas, norm2, err + 2 * t);

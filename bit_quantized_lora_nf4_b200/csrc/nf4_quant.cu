@@ -9,7 +9,8 @@
 // expanded to 16-bit in every pass.
 //
 // Arithmetic contract (IEEE fp32 round-to-nearest, no FMA contraction, no
-// flush-to-zero; this file is compiled with -fmad=false):
+// flush-to-zero; this file is compiled with -fmad=false), w the weight as fp32
+// (a bf16 weight widened exactly):
 //   a_b = max |w| over the 64-element block (exact)
 //   n   = fl32(w / a_b)            (0 when a_b == 0)
 //   code = #{ i : n > thresh[i] }  == nearest level, ties to the lower index
@@ -119,11 +120,29 @@ __device__ float exact_mean(const unsigned long long *acc, int64_t n) {
   return __double2float_rn(__ddiv_rn(s, static_cast<double>(n)));
 }
 
+// Weights arrive as fp32 or bf16; a bf16 weight is widened to fp32 (exact) and
+// every later step is the fp32 arithmetic above.
+__device__ __forceinline__ float load_weight(const float *W, int64_t e) { return W[e]; }
+__device__ __forceinline__ float load_weight(const uint16_t *W, int64_t e) {
+  return __uint_as_float(static_cast<uint32_t>(W[e]) << 16);
+}
+// Four consecutive weights starting at a 4-element boundary (16 or 8 bytes), streamed once.
+__device__ __forceinline__ float4 load_weight4(const float *W, int64_t i4) {
+  return __ldcs(reinterpret_cast<const float4 *>(W) + i4);
+}
+__device__ __forceinline__ float4 load_weight4(const uint16_t *W, int64_t i4) {
+  const uint2 v = __ldcs(reinterpret_cast<const uint2 *>(W) + i4);
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                     __uint_as_float(v.y & 0xFFFF0000u));
+}
+
 // One CTA per group of 256 blocks (16384 weights).  Full, aligned groups take
 // the vectorised path: each half-warp streams one block per iteration with
-// 16-byte loads, reduces its absmax with shuffles and writes 8 bytes of codes
-// per half-warp row.  A partial final group takes the per-block scalar path.
-__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float *__restrict__ W, int64_t numel,
+// 16-byte (fp32) or 8-byte (bf16) loads, reduces its absmax with shuffles and
+// writes 8 bytes of codes per half-warp row.  A partial final group takes the
+// per-block scalar path.
+template <typename TW>
+__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *__restrict__ W, int64_t numel,
                                                                      uint8_t *__restrict__ codes,
                                                                      uint8_t *__restrict__ absmax_q,
                                                                      float *__restrict__ group_scale, Nf4Table tab,
@@ -145,11 +164,10 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float
   bool bad = false;
 
   if (base + kGroupElems <= numel && (reinterpret_cast<uintptr_t>(W) & 15u) == 0) {
-    const float4 *W4 = reinterpret_cast<const float4 *>(W + base);
     uint16_t *C2 = reinterpret_cast<uint16_t *>(codes + base / 2);
     float4 v[16];
 #pragma unroll
-    for (int it = 0; it < 16; ++it) v[it] = __ldcs(W4 + it * kQuantThreads + t);
+    for (int it = 0; it < 16; ++it) v[it] = load_weight4(W, base / 4 + it * kQuantThreads + t);
 #pragma unroll
     for (int it = 0; it < 16; ++it) {
       const float4 x = v[it];
@@ -171,13 +189,13 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const float
       const int64_t e0 = blk * kBlock;
       const int64_t e1 = (e0 + kBlock < numel) ? e0 + kBlock : numel;
       for (int64_t e = e0; e < e1; ++e) {
-        const float w = W[e];
+        const float w = load_weight(W, e);
         bad |= !isfinite(w);
         a = fmaxf(a, fabsf(w));
       }
       for (int64_t e = e0; e < e1; e += 2) {
-        const uint32_t lo = encode_nf4(block_norm(W[e], a), s_thr);
-        const uint32_t hi = (e + 1 < e1) ? encode_nf4(block_norm(W[e + 1], a), s_thr) : 0u;
+        const uint32_t lo = encode_nf4(block_norm(load_weight(W, e), a), s_thr);
+        const uint32_t hi = (e + 1 < e1) ? encode_nf4(block_norm(load_weight(W, e + 1), a), s_thr) : 0u;
         codes[e / 2] = static_cast<uint8_t>(lo | (hi << 4));
       }
     }
@@ -390,8 +408,8 @@ size_t quantize_workspace_bytes(int64_t numel) {
   return static_cast<size_t>((128 + 4 * nblocks + 255) / 256 * 256);
 }
 
-cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q, float *group_scale,
-                            const Nf4Table &tab, void *ws, int *status, cudaStream_t st) {
+cudaError_t launch_quantize(const void *W, int dtype, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
+                            float *group_scale, const Nf4Table &tab, void *ws, int *status, cudaStream_t st) {
   const int64_t ngroups = (numel + kGroupElems - 1) / kGroupElems;
   const int64_t nblocks = (numel + kBlock - 1) / kBlock;
   const bool sgn = tab.qx != 0;
@@ -402,8 +420,12 @@ cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8
     cudaError_t e = cudaMemsetAsync(acc, 0, kSumDigits * sizeof(unsigned long long), st);
     if (e != cudaSuccess) return e;
   }
-  nf4_quantize_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(W, numel, codes, absmax_q,
-                                                                                 group_scale, tab, abs_ws, acc, status);
+  if (dtype == QLORA_DTYPE_BF16)
+    nf4_quantize_kernel<uint16_t><<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(
+        static_cast<const uint16_t *>(W), numel, codes, absmax_q, group_scale, tab, abs_ws, acc, status);
+  else
+    nf4_quantize_kernel<float><<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(
+        static_cast<const float *>(W), numel, codes, absmax_q, group_scale, tab, abs_ws, acc, status);
   if (sgn)
     nf4_dq_signed_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(
         abs_ws, acc, nblocks, absmax_q, group_scale, const_cast<float *>(tab.offset));

@@ -36,6 +36,9 @@
  *     the quantizer, a pipeline wait that exceeded its bound) are latched in a
  *     device status word; read and clear it with qlora_device_status().
  *   - Outputs are overwritten, never accumulated into.
+ *   - The library caches per-device state on first use (the device addresses
+ *     of its status word and scratch array, its side streams and events); do
+ *     not reset a device (cudaDeviceReset) after calling the library on it.
  *
  * Fixed format: block = 64 consecutive elements of the flat row-major weight,
  * group = 256 consecutive blocks.  codes: element 2j in the low nibble of byte
@@ -118,19 +121,27 @@ size_t qlora_absmax_bytes(int64_t rows, int64_t cols);
 size_t qlora_group_scale_bytes(int64_t rows, int64_t cols);
 size_t qlora_group_scale_bytes_dq(int64_t rows, int64_t cols, int dq);
 
-/* qlora_quantize_nf4 -- quantize fp32 weights once, up front (in out->format;
+/* Element types of the weight handed to the quantizer. */
+#define QLORA_DTYPE_F32 0    /* IEEE binary32                                   */
+#define QLORA_DTYPE_BF16 1   /* bfloat16 bit patterns (uint16_t)                */
+
+/* qlora_quantize_nf4 -- quantize the weights once, up front (in out->format;
  * NF4 unless the caller chose another table; block constants as out->dq).
- * ("Where the memory goes": the base never changes, so it is quantized once.)
- *   W   : device fp32 [out->rows * out->cols], flat row-major.
- *   out : rows/cols set by the caller; codes/absmax_q/group_scale receive the
- *         result.  Any rows*cols >= 1 is accepted (last block/group partial).
+ * ("Where the memory goes": the base never changes, so it is quantized once,
+ * from the 16-bit or 32-bit form it was trained in.)
+ *   W     : device [out->rows * out->cols] elements of `dtype`, flat row-major.
+ *   dtype : QLORA_DTYPE_F32 or QLORA_DTYPE_BF16 (QLORA_ERR_INVALID_ARG for any
+ *           other value).  A bf16 weight is widened to fp32, which is exact,
+ *           so it gives the same result as its fp32 copy.
+ *   out   : rows/cols set by the caller; codes/absmax_q/group_scale receive the
+ *           result.  Any rows*cols >= 1 is accepted (last block/group partial).
  * Per block b: a_b = max|w| (exact fp32); n = fl32(w / a_b) (n = 0 if a_b = 0);
  * code = index of the nearest level of the table, ties to the lower index.
  * The block constants a_b are then stored as QLORA_DQ_* describes.
  * QLORA_DQ_SIGNED needs a workspace: this call returns QLORA_ERR_WORKSPACE for
  * it; use qlora_quantize_nf4_ws.
  * A non-finite weight latches QLORA_ERR_NONFINITE (outputs then undefined). */
-qlora_status qlora_quantize_nf4(const float *W, const qlora_nf4_weight *out, void *stream);
+qlora_status qlora_quantize_nf4(const void *W, int dtype, const qlora_nf4_weight *out, void *stream);
 
 /* Workspace bytes qlora_quantize_nf4_ws needs (0 for QLORA_DQ_PLAIN; for
  * QLORA_DQ_SIGNED 128 + 4 bytes per block, rounded up to 256). */
@@ -143,8 +154,8 @@ size_t qlora_quantize_workspace_bytes(int64_t rows, int64_t cols, int dq);
  * against mu, and the exact sum (ten 64-bit words of 32-bit digits, cleared
  * by the call).  rows*cols < 2^38 for QLORA_DQ_SIGNED
  * (QLORA_ERR_UNSUPPORTED_SHAPE beyond). */
-qlora_status qlora_quantize_nf4_ws(const float *W, const qlora_nf4_weight *out, void *ws, size_t ws_bytes,
-                                   void *stream);
+qlora_status qlora_quantize_nf4_ws(const void *W, int dtype, const qlora_nf4_weight *out, void *ws,
+                                   size_t ws_bytes, void *stream);
 
 /* qlora_dequantize -- W' = bf16(fl32(v_code * a'_b)) into a device bf16 buffer
  * of rows*cols elements, row-major, a'_b the dequantized block constant of
@@ -250,22 +261,27 @@ qlora_status qlora_linear_bwd_materialized(qlora_materialize_fn materialize, voi
 
 /* qlora_linear_fwd_noalloc -- the same forward as qlora_linear_fwd, for
  * callers that cannot allocate device memory (code running where cudaMalloc
- * is unavailable or forbidden: inside host callbacks or allocator hooks,
- * runtimes with a memory map fixed at start-up, plugin hosts that own every
- * allocation).  The pages have no counterpart of this call; it is a
- * deployment convenience.
+ * is unavailable or forbidden: custom allocator hooks, runtimes with a memory
+ * map fixed at start-up, plugin hosts that own every allocation).  The pages
+ * have no counterpart of this call; it is a deployment convenience.
  *   Arguments as qlora_linear_fwd, minus the workspace.  The scratch is a
  *   QLORA_STATIC_SCRATCH_BYTES array inside the library, held on every GPU that
  *   loads the library until the process exits; the call allocates and frees
  *   nothing.
- *   Returns QLORA_ERR_WORKSPACE when qlora_workspace_min_bytes(QLORA_OP_FWD,
- *   M, N, K, r) exceeds QLORA_STATIC_SCRATCH_BYTES (e.g. M = 8192, r = 64 fits;
- *   M = 8192, r = 256 does not); the fused GEMM runs without its stream-K tail
- *   when the full workspace does not fit.
+ *   Returns QLORA_ERR_WORKSPACE (nothing enqueued) when
+ *   qlora_workspace_min_bytes(QLORA_OP_FWD, M, N, K, r) exceeds
+ *   QLORA_STATIC_SCRATCH_BYTES.  That minimum grows with M r and does not
+ *   depend on N or K: at r = 64 it is about 2.4 KB per token, so M <= 3449 fits
+ *   (M = 2048, r = 64 fits; M = 4096, r = 64 does not); at r = 256, M <= 862.
+ *   The fused GEMM always runs without its stream-K tail here (that optional
+ *   workspace region is about 80 MB for M > 128), so a partial last wave of
+ *   tiles is not split.
  *   The first call on a device looks up the array's device address; make that
  *   first call before any stream capture.  Every call shares the one array
  *   (it keeps the previous call's contents; nothing needs clearing), so calls
- *   that overlap on the GPU race: serialize them on one stream. */
+ *   that overlap on the GPU race: serialize them on one stream.  Like every
+ *   entry point here, it must not be called from a stream host callback
+ *   (cudaLaunchHostFunc), where CUDA calls are not allowed. */
 qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_weight *w, const uint16_t *X, int64_t M,
                                       const uint16_t *A, const uint16_t *B, int r, float s,
                                       uint16_t *Y, float *H_out, void *stream);

@@ -139,9 +139,14 @@ def test_linear_argument_errors():
 def test_quantize_dequantize_argument_errors():
     lib = q.load()
     w = _w()
-    assert lib.qlora_quantize_nf4(None, ctypes.byref(w), None) == 1
-    assert lib.qlora_quantize_nf4(MIS, ctypes.byref(w), None) == 3
-    assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(_w(rows=0)), None) == 1
+    for dt in (q.DTYPE_F32, q.DTYPE_BF16):
+        assert lib.qlora_quantize_nf4(None, dt, ctypes.byref(w), None) == 1
+        assert lib.qlora_quantize_nf4(MIS, dt, ctypes.byref(w), None) == 3
+        assert lib.qlora_quantize_nf4(FAKE, dt, ctypes.byref(_w(rows=0)), None) == 1
+    # element types other than fp32 / bf16 are refused before anything is enqueued
+    for dt in (-1, 2, 7):
+        assert lib.qlora_quantize_nf4(FAKE, dt, ctypes.byref(w), None) == 1
+        assert lib.qlora_quantize_nf4_ws(FAKE, dt, ctypes.byref(w), FAKE, 1 << 20, None) == 1
     assert lib.qlora_dequantize(ctypes.byref(w), None, None) == 1
     assert lib.qlora_dequantize(ctypes.byref(_w(scale=MIS)), FAKE, None) == 3
     assert lib.qlora_nf4_codebook(None) == 1
@@ -163,13 +168,13 @@ def test_signed_block_constant_sizes_and_errors():
         assert ws % 256 == 0 and ws >= 128 + 4 * nf4.num_blocks(n)
     assert lib.qlora_group_scale_bytes_dq(4, 4, 2) == 0
     w = q.Nf4WeightC(256, 256, FAKE, FAKE, FAKE, q.FORMAT_NF4, q.DQ_SIGNED)
-    assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(w), None) == 7          # needs the workspace call
-    assert lib.qlora_quantize_nf4_ws(FAKE, ctypes.byref(w), FAKE, 16, None) == 7
-    assert lib.qlora_quantize_nf4_ws(FAKE, ctypes.byref(w), MIS, 1 << 20, None) == 3
+    assert lib.qlora_quantize_nf4(FAKE, q.DTYPE_F32, ctypes.byref(w), None) == 7          # needs the workspace call
+    assert lib.qlora_quantize_nf4_ws(FAKE, q.DTYPE_BF16, ctypes.byref(w), FAKE, 16, None) == 7
+    assert lib.qlora_quantize_nf4_ws(FAKE, q.DTYPE_F32, ctypes.byref(w), MIS, 1 << 20, None) == 3
     big = q.Nf4WeightC(1 << 20, 1 << 18, FAKE, FAKE, FAKE, q.FORMAT_NF4, q.DQ_SIGNED)
-    assert lib.qlora_quantize_nf4_ws(FAKE, ctypes.byref(big), FAKE, 1 << 62, None) == 2
+    assert lib.qlora_quantize_nf4_ws(FAKE, q.DTYPE_F32, ctypes.byref(big), FAKE, 1 << 62, None) == 2
     bad = q.Nf4WeightC(256, 256, FAKE, FAKE, FAKE, q.FORMAT_NF4, 2)
-    assert lib.qlora_quantize_nf4(FAKE, ctypes.byref(bad), None) == 1
+    assert lib.qlora_quantize_nf4(FAKE, q.DTYPE_F32, ctypes.byref(bad), None) == 1
     assert lib.qlora_dequantize(ctypes.byref(bad), FAKE, None) == 1
     assert _fwd(bad) == 1
 
@@ -228,3 +233,22 @@ def test_dense_linear_sizes_and_argument_errors():
     assert calls == []          # argument errors are found before the weight is materialized
     bad = q.MATERIALIZE_FN(lambda ctx, w_out, n, k, stream: 4)
     assert m(bad, None, FAKE, 256, 256, FAKE, 64, FAKE, FAKE, 16, 1.0, FAKE, None, FAKE, big, None) == 4
+
+
+def test_noalloc_scratch_size_and_documented_limits():
+    """The binding's copy of QLORA_STATIC_SCRATCH_BYTES matches the header, and
+    the size limits the header states for qlora_linear_fwd_noalloc hold for the
+    library's own workspace sizing (host-only calls)."""
+    hdr = open(HEADER).read()
+    m = re.search(r"#define QLORA_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m and int(m.group(1)) << int(m.group(2)) == q.QLORA_STATIC_SCRATCH_BYTES
+    lib = q.load()
+    lim = q.QLORA_STATIC_SCRATCH_BYTES
+    for N, K in ((4096, 4096), (11008, 4096), (4096, 11008), (8192, 22016)):
+        assert lib.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 2048, N, K, 64) <= lim
+        assert lib.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3449, N, K, 64) <= lim
+        assert lib.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3450, N, K, 64) > lim
+        assert lib.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 862, N, K, 256) <= lim
+        assert lib.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 863, N, K, 256) > lim
+        # the stream-K tail never fits beside the forward
+        assert lib.qlora_workspace_bytes(q.QLORA_OP_FWD, 256, N, K, 64) > lim
