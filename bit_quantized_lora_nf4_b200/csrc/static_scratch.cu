@@ -2,11 +2,12 @@
 // allocate device memory.
 //
 // Some callers have no way to hand the library a workspace: code that runs
-// where cudaMalloc is forbidden or unavailable (inside a host callback, a
-// custom allocator's own hooks, a real-time or embedded runtime that fixes its
-// memory map at start-up, or a plugin host that owns every allocation).  This
-// entry point takes only the inputs and outputs and runs the ordinary forward
-// with its scratch taken from one array that lives in the library itself.
+// where cudaMalloc is forbidden or unavailable (a custom allocator's own hooks,
+// a real-time or embedded runtime that fixes its memory map at start-up, or a
+// plugin host that owns every allocation).  This entry point takes only the
+// inputs and outputs and runs the ordinary forward with its scratch taken from
+// one array that lives in the library itself.  It launches kernels, so like
+// any CUDA call it cannot be made from a stream host callback.
 //
 // The array is a file-scope __device__ variable of kStaticScratchBytes bytes:
 // every GPU on which the library's device code is loaded holds it until the
@@ -17,7 +18,14 @@
 // before any stream capture.  All calls share the array and it keeps the
 // previous call's contents; the forward overwrites every scratch element it
 // reads, so nothing needs clearing.  Calls that overlap on the GPU (two
-// streams, or two host threads) race on the array.
+// streams, or two host threads) race on the array.  The address is cached for
+// the life of the process, so the device must not be reset after the first
+// call (a reset reloads the module, and the array may move).
+//
+// The array covers the forward's minimum workspace only: the minimum grows
+// with M r (about 2.4 KB per token at r = 64, so M <= 3449 there), and the
+// fused GEMM's optional stream-K region (about 80 MB for M > 128) never fits,
+// so the GEMM always runs without the stream-K split of a partial last wave.
 #include <mutex>
 
 #include "internal.h"

@@ -58,3 +58,27 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch(lib):
     Y = torch.empty((8192, 4096), dtype=torch.bfloat16, device="cuda")
     assert lib_.qlora_workspace_bytes(q.QLORA_OP_FWD, 8192, 4096, 4096, 256) > (8 << 20)
     assert _noalloc(w, X, A, B, 0.25, Y, None) == 7          # QLORA_ERR_WORKSPACE, nothing launched
+
+
+def test_noalloc_documented_size_limits(lib):
+    """The limits the header states: at r = 64, M = 2048 fits the static
+    scratch and M = 4096 does not (the minimum forward workspace grows with
+    M r, not with N or K).  The fitting case runs and matches the workspace
+    entry point; the other is refused before anything is enqueued."""
+    lib_ = q.load()
+    limit = q.QLORA_STATIC_SCRATCH_BYTES
+    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 2048, 4096, 4096, 64) <= limit
+    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3449, 4096, 4096, 64) <= limit
+    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3450, 4096, 4096, 64) > limit
+    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 4096, 4096, 4096, 64) > limit
+    # fits: runs, and equals the ordinary entry point within the parity tolerance
+    _check_case(qi.LinearCase("noalloc_fits", 2048, 4096, 4096, 64, 16.0, 73))
+    # does not fit: QLORA_ERR_WORKSPACE, outputs untouched
+    w = q.NF4Weight.empty(4096, 4096)
+    X = torch.zeros((4096, 4096), dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros((64, 4096), dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros((4096, 64), dtype=torch.bfloat16, device="cuda")
+    Y = torch.full((4096, 4096), 7.0, dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(w, X, A, B, 0.25, Y, None) == 7
+    torch.cuda.synchronize()
+    assert bool((Y == 7.0).all())
