@@ -1,8 +1,9 @@
 """A decoder layer with all seven projections on the library (NF4 + LoRA):
 
-- at a reduced width, output, input gradient and every adapter gradient
+- at two reduced widths, output, input gradient and every adapter gradient
   against the fp64 reference layer (oracle/layer.py) built on the oracle's
-  dequantized weights;
+  dequantized weights: 128 tokens (one-CTA GEMM) and 512 tokens (the CTA-pair
+  GEMM that serves the full-size layer);
 - at the LLaMA-7B shape with 4 x 2048 tokens (the decoder-layer
   configuration), one forward + backward: finite results, clean device
   status and bit-identical results on a second run.
@@ -38,13 +39,20 @@ def _bf16(t):
     return t.to(torch.bfloat16)
 
 
-def test_reduced_width_layer_against_the_fp64_reference(lib):
-    cfg = ql.LayerConfig(d=512, heads=4, hidden=1408, r=16)
+# (width, heads, SwiGLU hidden, adapter rank, batch, sequence): 2 x 64 tokens take the
+# one-CTA GEMM (M <= 128); 2 x 256 tokens take the CTA-pair kernel with both of its
+# TMEM accumulators in use (M > 256), the kernel that serves the full-size layer.
+REDUCED = [(512, 4, 1408, 16, 2, 64), (1024, 8, 2816, 64, 2, 256)]
+
+
+@pytest.mark.parametrize("d,heads,hidden,r,batch,seq", REDUCED, ids=["m128_one_cta", "m512_cta_pair"])
+def test_reduced_width_layer_against_the_fp64_reference(lib, d, heads, hidden, r, batch, seq):
+    cfg = ql.LayerConfig(d=d, heads=heads, hidden=hidden, r=r)
     params = ql.make_params(cfg, seed=7)
     layer = ql.QLoRADecoderLayer(cfg, params, "cuda")
     g = torch.Generator().manual_seed(8)
-    x = _bf16(torch.randn(2, 64, cfg.d, generator=g))
-    gout = _bf16(torch.randn(2, 64, cfg.d, generator=g))
+    x = _bf16(torch.randn(batch, seq, cfg.d, generator=g))
+    gout = _bf16(torch.randn(batch, seq, cfg.d, generator=g))
     xd = x.cuda().requires_grad_(True)
     out = layer(xd)
     (out.float() * gout.cuda().float()).sum().backward()
