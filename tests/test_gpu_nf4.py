@@ -146,7 +146,13 @@ def test_bf16_weights_bit_exact(lib, shape, dq):
     w32 = q.quantize_nf4(W32.cuda().contiguous(), dq=dq)
     torch.cuda.synchronize()
     assert q.device_status() == 0
-    assert_weight_bits(w, oq)
+    if dq == q.DQ_PLAIN:
+        assert_weight_bits(w, oq)
+    else:   # signed constants: the group scales, then mu, in one array
+        assert np.array_equal(w.codes.cpu().numpy(), oq["codes"])
+        assert np.array_equal(w.absmax_q.cpu().numpy(), oq["absmax_q"])
+        assert np.array_equal(w.scales.cpu().numpy().view(np.uint32), oq["group_scale"].view(np.uint32))
+        assert w.offset.cpu().numpy().view(np.uint32)[0] == np.float32(oq["offset"]).view(np.uint32)
     assert torch.equal(w.codes, w32.codes) and torch.equal(w.absmax_q, w32.absmax_q)
     assert torch.equal(w.group_scale, w32.group_scale)
     got = q.dequantize(w).view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
