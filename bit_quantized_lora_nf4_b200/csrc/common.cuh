@@ -135,6 +135,10 @@ __device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uin
                "r"(bytes)
                : "memory");
 }
+// Bring `bytes` bytes at `gsrc` into L2 (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gsrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N bulk groups of this thread still read shared memory.
 template <int N>

@@ -5,24 +5,34 @@
 // handful of tokens the packed weight stream (0.516 B per weight) is the whole
 // cost: the codes stream into shared memory by TMA and are decoded straight
 // into tensor-core register fragments.  The decode (a per-block 16-entry bf16
-// table and byte permutes) runs on the integer pipe, which puts this path's
-// ceiling below the HBM roofline.
+// table and byte permutes) runs on the integer pipe.
 //
-// One cooperative launch (every CTA resident), three phases:
-//   1. H CTAs (one per 16 adapter rows) compute s H = s X A^T on mma.sync with
-//      a fixed-order reduction over their warps and store it as a bf16 hi/lo
-//      pair (and H in fp32 when asked).  Weight CTAs stream the weight: it is
-//      cut into positions (16-row tile, 256-wide K step) and weight warp g of
-//      G takes positions [g U / G, (g+1) U / G), so every SM gets the same
-//      decode work to within one position.  Per position a thread decodes one
-//      64-weight block of two rows into m16n8k16 A fragments (tokens are the
-//      8-column B operand; two column tiles when M > 8).  A warp stores its
-//      fp32 sum for every tile it touches as that tile's piece number
-//      g - g0(t), g0(t) being the first warp on the tile.
-//   2. One grid-wide barrier (bounded wait).
-//   3. Every warp finishes tiles t = w, w + W, ...: adds the tile's pieces in
-//      piece order (a fixed order, so results are deterministic), adds
-//      (s H) B^T with two more mma chains, stores bf16 Y.
+// One cooperative launch (every CTA resident, so the bounded waits below on
+// other CTAs' flags always end).  The weight is cut into units (16-row tile,
+// 256-wide K step), numbered tile-major; CTA c takes the contiguous range
+// [start(c), start(c+1)) (a closed-form split by cost, see cta_start) and its
+// GV_WARPS warps split that range contiguously again.
+//   1. H = X A^T is cut into JT S parts (16 adapter rows x one 256-wide K
+//      step); CTA c computes parts c, c + G, ... first (their two 16-byte
+//      loads of A per thread are the first loads it issues), publishes each
+//      under a flag; CTA jt < JT then adds the S parts of adapter tile jt in
+//      K order and publishes that tile of H under its own flag.  Those CTAs'
+//      weight ranges are shorter by that cost.
+//   2. Every warp streams its units (per-warp TMA code ring, constants fetched
+//      one unit ahead) and decodes each 64-weight block of two rows into
+//      m16n8k16 A fragments (tokens are the 8-column B operand; two column
+//      tiles when M > 8).  For every tile it touches it stores its fp32 sum
+//      as a piece in the CTA's slot (tile - first tile of the CTA) + warp.
+//   3. The CTA stamps its flag once all its pieces are stored, gathers s H
+//      from the JT tiles of H into shared memory, and finishes
+//      the tiles whose last unit it holds: the pieces of every CTA on the
+//      tile, in CTA order and warp order within a CTA (a fixed order, so
+//      results do not depend on timing), waiting only for the flags of the
+//      earlier CTAs on that tile; then (s H) B^T and bf16 Y.
+// Nothing waits before it has published what others wait for, so the waits
+// form no cycle.  Flags carry a 64-bit tag unique to the launch (consecutive
+// from a random start), so no word needs clearing between launches.
+#include <algorithm>
 #include <atomic>
 #include <random>
 
@@ -40,19 +50,30 @@ constexpr int GV_THREADS = 32 * GV_WARPS;
 #endif
 constexpr int GV_CTAS_PER_SM = QLORA_GEMV_CTAS_PER_SM;
 
-// One position's codes arrive by TMA as a 16-row x 128-byte box (256 codes of
-// each of the tile's rows), 128-byte swizzled, into a per-warp ring.
+// One unit's codes arrive by TMA as a 16-row x 128-byte box (256 codes of each
+// of the tile's rows), 128-byte swizzled, into a per-warp ring.
 constexpr int GV_STAGE_BYTES = 16 * 128;
 #ifndef QLORA_GEMV_STAGES
-#define QLORA_GEMV_STAGES 2
+#define QLORA_GEMV_STAGES 4
 #endif
 constexpr int GV_STAGES = QLORA_GEMV_STAGES;
 constexpr int GV_RING_BYTES = GV_WARPS * GV_STAGES * GV_STAGE_BYTES;
-constexpr int GV_RED_OFFSET = GV_RING_BYTES + 1024;          // after the ring and its barriers
-constexpr int GV_RED_BYTES = GV_WARPS * 2 * 4 * 32 * 4;      // H CTAs: per-warp C fragments (two token tiles)
-constexpr int GV_XS_OFFSET = GV_RED_OFFSET + GV_RED_BYTES;
-constexpr int GV_SMEM_BASE = GV_XS_OFFSET + 1024;             // + alignment slack of the dynamic segment
-constexpr int GV_XS_MAX = 64 * 1024;                          // activations kept in shared memory up to this size
+constexpr int GV_BAR_OFFSET = GV_RING_BYTES;               // ring barriers, then the activation barrier
+constexpr int GV_MAX_CTAS = 511;                            // CTA starts kept in shared memory
+constexpr int GV_START_OFFSET = GV_RING_BYTES + 512;        // int starts[GV_MAX_CTAS + 1]
+constexpr int GV_AUX_OFFSET = GV_RING_BYTES + 512 + 2048 + 512;   // H reduction, then s H (hi, lo); 1024-aligned
+// Units a warp brings into L2 before the previous kernel's results are waited for.
+#ifndef QLORA_GEMV_PREFETCH_UNITS
+#define QLORA_GEMV_PREFETCH_UNITS 64
+#endif
+constexpr int GV_PREFETCH_UNITS = QLORA_GEMV_PREFETCH_UNITS;
+// Weight units a CTA gives up for a part of H and for adding a tile of H (tuned on B200).
+#ifndef QLORA_GEMV_PC
+#define QLORA_GEMV_PC 1
+#endif
+#ifndef QLORA_GEMV_HC
+#define QLORA_GEMV_HC 3
+#endif
 
 // Activations in shared memory: token row m at m * xs_row (rows copied whole by
 // one bulk copy each, so every CTA asks L2 for whole rows, not 16-byte pieces),
@@ -89,97 +110,94 @@ __device__ __forceinline__ float ldg_once_f32(const float *p) {
   return v;
 }
 
-
-// Grid-wide barrier of the cooperative launch (every CTA resident), on a 64-bit
-// word of the workspace: the high half holds the launch's epoch (unique per
-// launch in this process, from a random start), the low half the arrivals of
-// that launch so far.  CTA 0 stamps the word with its epoch and a zero count
-// when the kernel starts (grid_barrier_open); every CTA counts itself in with an
-// atomic add only once it sees that epoch, so whatever the word held before
-// (an earlier launch's tag, or never written) is neither counted nor needs
-// clearing.  Round `round` (1, 2, ...) is complete once round x CTAs have
-// arrived.  Each CTA's writes before the barrier are published by its thread
-// 0 (after the CTA barrier) with a GPU-scope fence before it counts itself in.
-// Waits are bounded; on timeout the status is latched and the CTA goes on.
+// Flags between the CTAs of one launch: 64-bit words stamped with the launch's tag.
 __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const unsigned long long *p) {
   uint64_t v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void grid_barrier_open(unsigned long long *word, uint32_t epoch) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(word, static_cast<unsigned long long>(epoch) << 32);
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long *p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ void grid_barrier(unsigned long long *word, uint32_t epoch, uint32_t round, int *status,
-                                             uint64_t limit) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t n = gridDim.x * gridDim.y * gridDim.z;
-    __threadfence();
-    const long long t0 = clock64();
-    bool ok = true;
-    while ((ld_acquire_gpu_u64(word) >> 32) != epoch) {   // the launch's stamp is in place
-      if (static_cast<uint64_t>(clock64() - t0) > limit) {
-        ok = false;
-        break;
-      }
-    }
-    if (ok) {
-      atomicAdd(word, 1ull);
-      while (true) {
-        const uint64_t w = ld_acquire_gpu_u64(word);
-        if ((w >> 32) == epoch && static_cast<uint32_t>(w) >= round * n) break;
-        if (static_cast<uint64_t>(clock64() - t0) > limit) {
-          ok = false;
-          break;
-        }
-      }
-    }
-    if (!ok) latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
-  }
-  __syncthreads();
-}
-
-// First position of weight warp g's range, and the warp whose range holds position u.
-__device__ __forceinline__ int range_start(int g, int U, int G) {
-  return static_cast<int>(static_cast<int64_t>(g) * U / G);
-}
-__device__ __forceinline__ int range_owner(int u, int U, int G) {
-  return static_cast<int>((static_cast<int64_t>(u + 1) * G - 1) / U);
+// Wait (bounded) until *f carries `tag`; false when the bound ran out.
+__device__ __forceinline__ bool wait_flag(const unsigned long long *f, uint64_t tag, uint64_t limit) {
+  const long long t0 = clock64();
+  while (ld_acquire_gpu_u64(f) != tag)
+    if (static_cast<uint64_t>(clock64() - t0) > limit) return false;
+  return true;
 }
 
 struct GemvParams {
   const uint16_t *X;
   const uint8_t *absmax_q;
   const float *group_scale;
-  const uint16_t *A;        // [r, K]
-  const uint16_t *B;        // [N, r]
+  const uint16_t *A;            // [r, K]
+  const uint16_t *B;            // [N, r]
   float s;
-  uint16_t *Y;              // [M, N]
-  float *H_out;             // optional [M, r]
-  uint16_t *sh_hi;          // [8 NT, r16] s H, high bf16 part
-  uint16_t *sh_lo;          //              and the remainder
-  float *pieces;            // [T][P][M][16] tile sums, one per weight warp that touches the tile
-  float *hpart;             // [JT][HS][8 NT][16] partial H of the H CTAs (HS > 1)
-  unsigned long long *bar;  // grid barrier word (see grid_barrier)
-  uint32_t epoch;           // this launch's tag on it
+  uint16_t *Y;                  // [M, N]
+  float *H_out;                 // optional [M, r]
+  float *pieces;                // [G][SLOTS][M][16] tile sums, one per warp and tile it touches
+  float *hpart;                 // [JT S][8 NT][16] parts of H^T (adapter tile i / S, K step i % S)
+  float *hsum;                  // [JT][8 NT][16] tiles of H^T
+  unsigned long long *hpflag;   // [JT S] a part of H is stored
+  unsigned long long *hflag;    // [JT] a tile of H is stored
+  unsigned long long *wflag;    // [G][GV_WARPS] a warp's pieces are stored
+  unsigned long long tag;       // this launch's flag value
   int M, r, r16;
-  int JT, HS;               // H CTAs: blockIdx.x < JT * HS, adapter tile blockIdx.x / HS, K split blockIdx.x % HS
-  int G;                    // weight warps (CTA blockIdx.x - JT HS holds weight warps 8 (that) .. +7)
-  int S, U, T, P;           // K steps per tile, positions, tiles, piece slots per tile
-  int xs_row;               // row pitch of the activations in shared memory (0: global memory)
+  int JT, HP;                   // adapter tiles, parts of H (JT S)
+  int pc, hc;                   // weight units a CTA gives up for an H part / for adding a tile of H
+  int G;                        // CTAs
+  int S, U, T;                  // K steps per tile, units (T S), tiles
+  int SLOTS;                    // piece slots per CTA
+  int xs_row;                   // row pitch of the activations in shared memory (0: global memory)
+  int cs_rows;                  // block constants of up to cs_rows rows per CTA in shared memory (0: none)
   int64_t N, K;
   int *status;
   uint64_t wait_limit;
   Nf4Table tab;
 };
 
-// Quantized constants of one position for rows n0 = 16 t + g and n0 + 8, block 4 step + c.
+// First unit of CTA c (0 <= c <= G): an even split of U + P pc + JT hc units
+// of work (P = min(HP, G) CTAs with an H part, JT CTAs adding a tile of H),
+// each such CTA's share shortened by pc or hc.  Non-decreasing in c (the host
+// keeps pc + hc <= U / G); start(0) = 0, start(G) = U.
+__host__ __device__ __forceinline__ int cta_start(int c, int U, int G, int P, int pc, int JT, int hc) {
+  const int64_t total = static_cast<int64_t>(U) + static_cast<int64_t>(P) * pc + static_cast<int64_t>(JT) * hc;
+  return static_cast<int>(static_cast<int64_t>(c) * total / G - static_cast<int64_t>(c < P ? c : P) * pc -
+                          static_cast<int64_t>(c < JT ? c : JT) * hc);
+}
+__device__ __forceinline__ int cta_start(const GemvParams &p, int c) {
+  return cta_start(c, p.U, p.G, min(p.HP, p.G), p.pc, p.JT, p.hc);
+}
+// Every CTA's first unit, computed once per CTA into shared memory (G + 1 ints).
+__device__ __forceinline__ void fill_starts(const GemvParams &p, int *starts) {
+  for (int c = threadIdx.x; c <= p.G; c += GV_THREADS) starts[c] = cta_start(p, c);
+}
+// The CTA whose range holds unit u: the largest c with start(c) <= u.
+__device__ __forceinline__ int cta_owner(const int *starts, int G, int u) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (starts[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+// Warp w of a CTA with range [a, a + L) starts at a + floor(w L / GV_WARPS); the
+// warp whose range holds unit u (a <= u < a + L) is the largest such w.  (U <
+// 2^27, so these products fit 32 bits.)
+__device__ __forceinline__ int warp_start(int a, int L, int w) { return a + ((w * L) >> 3); }
+__device__ __forceinline__ int warp_owner(int a, int L, int u) {
+  return static_cast<int>(static_cast<uint32_t>((u - a + 1) * GV_WARPS - 1) / static_cast<uint32_t>(L));
+}
+
+// Quantized constants of one unit for rows n0 = 16 t + g and n0 + 8, block 4 step + c.
 struct PosConst {
   uint32_t q0, q1;   // 8-bit block constants; bit 8 set for rows past N / blocks past K
   float S0, S1;      // 32-bit group constants
 };
 
-// a' of one position's block, and 0 for the padding positions (bit 8 of q set).
+// a' of one unit's block, and 0 for the padding units (bit 8 of q set).
 __device__ __forceinline__ float pos_constant(uint32_t q, float S, uint32_t qx, float mu) {
   return (q & 0x100u) ? 0.0f : block_constant(q, S, qx, mu);
 }
@@ -206,65 +224,47 @@ struct XSource {
   }
 };
 
-// s H (and H) from the C fragment of one adapter tile.
-template <int NT>
-__device__ __forceinline__ void write_sh(const GemvParams &p, int j0, int t, int e, int lane, float h) {
+// Phase 1: part i of H^T (adapter rows j0 = 16 (i / S) .. +15, K step i % S).
+// Warp w covers K columns 256 step + 32 w .. +31; thread (g, c) the eight
+// columns from +8 c of A rows j0 + g and j0 + g + 8, loaded (16 bytes each)
+// before anything else, in the K order the weight uses.
+struct HLoad {
+  uint4 a, b;
+};
+__device__ __forceinline__ HLoad h_load(const GemvParams &p, int i) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
-  // C fragment: H^T[j][tok], j = j0 + g + 8 (e >> 1), tok = 8 t + 2 c + (e & 1)
-  const int j = j0 + g + 8 * (e >> 1);
-  const int tok = 8 * t + 2 * c + (e & 1);
-  if (p.H_out && tok < p.M && j < p.r) p.H_out[static_cast<int64_t>(tok) * p.r + j] = h;
-  const float sh = __fmul_rn(p.s, h);
-  const __nv_bfloat16 hi = __float2bfloat16_rn(sh);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(sh, __bfloat162float(hi)));
-  p.sh_hi[tok * p.r16 + j] = *reinterpret_cast<const uint16_t *>(&hi);
-  p.sh_lo[tok * p.r16 + j] = *reinterpret_cast<const uint16_t *>(&lo);
+  const int j0 = (i / p.S) * 16, step = i - (i / p.S) * p.S;
+  const int64_t k = static_cast<int64_t>(step) * 256 + warp * 32 + c * 8;   // a multiple of 8; K % 64 == 0
+  const int ja = j0 + g, jb = j0 + g + 8;
+  HLoad h;
+  h.a = (k < p.K && ja < p.r) ? __ldg(reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(ja) * p.K + k))
+                              : make_uint4(0, 0, 0, 0);
+  h.b = (k < p.K && jb < p.r) ? __ldg(reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(jb) * p.K + k))
+                              : make_uint4(0, 0, 0, 0);
+  return h;
 }
 
-// Phase 1, H CTA (adapter tile jt = blockIdx.x / HS: rows j0 .. j0+15; K part
-// hs = blockIdx.x % HS).  H warp q = 8 hs + warp takes K steps q, q + 8 HS, ...;
-// in a step thread (g, c) covers columns 256 step + 64 c .. +63 of A rows j0 + g
-// and j0 + g + 8, in the same K order as the weight.  The 8 warps are added in
-// a fixed order; with one K part the CTA writes s H, otherwise its partial sum.
+// The part's products (two m16n8k16 steps per warp), the 8 warps added in a
+// fixed order, stored and published under the part's flag.
 template <int NT, bool XS>
-__device__ __forceinline__ void h_role(const GemvParams &p, const XSource<NT, XS> &x, float *red) {
+__device__ __forceinline__ void h_part(const GemvParams &p, const XSource<NT, XS> &x, const HLoad &h, int i,
+                                       float *red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int jt = blockIdx.x / p.HS, hs = blockIdx.x - jt * p.HS;
-  const int j0 = jt * 16;
+  const int step = i - (i / p.S) * p.S;
+  const int64_t k = static_cast<int64_t>(step) * 256 + warp * 32 + c * 8;
   const int KB = static_cast<int>(p.K / kBlock);
+  const int kb = static_cast<int>(min(k, p.K - 8) / kBlock), w8 = static_cast<int>((min(k, p.K - 8) % kBlock) / 8);
+  (void)KB;
   float acc[NT][4];
 #pragma unroll
-  for (int t = 0; t < NT; ++t)
+  for (int t = 0; t < NT; ++t) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
-  const int ja = j0 + g, jb = j0 + g + 8;
-  const uint4 *arow = reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(min(ja, p.r - 1)) * p.K);
-  const uint4 *brow = reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(min(jb, p.r - 1)) * p.K);
-  for (int st = hs * GV_WARPS + warp; st < p.S; st += GV_WARPS * p.HS) {
-    const int kb = 4 * st + c;
-    const int kbc = min(kb, KB - 1);
-    const bool va = kb < KB && ja < p.r, vb = kb < KB && jb < p.r;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {   // half a block of each row in flight at once
-      uint4 ua[4], ub[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        ua[w] = __ldg(arow + kbc * 8 + 4 * h + w);
-        ub[w] = __ldg(brow + kbc * 8 + 4 * h + w);
-      }
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint4 a4 = va ? ua[w] : make_uint4(0, 0, 0, 0);
-        const uint4 b4 = vb ? ub[w] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const uint4 xv = x.load(t, kbc, 4 * h + w);
-          mma16816(acc[t], a4.x, b4.x, a4.y, b4.y, xv.x, xv.y);
-          mma16816(acc[t], a4.z, b4.z, a4.w, b4.w, xv.z, xv.w);
-        }
-      }
-    }
+    const uint4 xv = x.load(t, kb, w8);
+    mma16816(acc[t], h.a.x, h.b.x, h.a.y, h.b.y, xv.x, xv.y);
+    mma16816(acc[t], h.a.z, h.b.z, h.a.w, h.b.w, xv.z, xv.w);
   }
 #pragma unroll
   for (int t = 0; t < NT; ++t)
@@ -272,46 +272,59 @@ __device__ __forceinline__ void h_role(const GemvParams &p, const XSource<NT, XS
     for (int e = 0; e < 4; ++e) red[((warp * NT + t) * 4 + e) * 32 + lane] = acc[t][e];
   __syncthreads();
   if (warp == 0) {
+    float *dst = p.hpart + static_cast<int64_t>(i) * 8 * NT * 16;
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float h = 0.0f;
+        float v = 0.0f;
 #pragma unroll
-        for (int w = 0; w < GV_WARPS; ++w) h += red[((w * NT + t) * 4 + e) * 32 + lane];
-        if (p.HS == 1) {
-          write_sh<NT>(p, j0, t, e, lane, h);
-        } else {   // partial: [jt][hs][tok][16 j]
-          const int tok = 8 * t + 2 * c + (e & 1), jl = g + 8 * (e >> 1);
-          p.hpart[((static_cast<int64_t>(jt) * p.HS + hs) * 8 * NT + tok) * 16 + jl] = h;
-        }
+        for (int w = 0; w < GV_WARPS; ++w) v += red[((w * NT + t) * 4 + e) * 32 + lane];
+        // C fragment: H^T[j0 + g + 8 (e >> 1)][tok = 8 t + 2 c + (e & 1)]
+        __stcg(dst + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1), v);
       }
     }
   }
-}
-
-// Between the two grid barriers (HS > 1): warp jt of all warps adds the HS
-// partial sums of adapter tile jt in K-part order and writes s H.
-template <int NT>
-__device__ __forceinline__ void h_finish(const GemvParams &p) {
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int jt = blockIdx.x * GV_WARPS + (threadIdx.x >> 5);
-  if (jt >= p.JT) return;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = 8 * t + 2 * c + (e & 1), jl = g + 8 * (e >> 1);
-      float h = 0.0f;
-      for (int hs = 0; hs < p.HS; ++hs) h += __ldcg(p.hpart + ((static_cast<int64_t>(jt) * p.HS + hs) * 8 * NT + tok) * 16 + jl);
-      write_sh<NT>(p, jt * 16, t, e, lane, h);
-    }
+  __syncthreads();   // the part is stored, and red is free again
+  if (threadIdx.x == 0) {
+    __threadfence();
+    st_release_gpu_u64(p.hpflag + i, p.tag);
   }
 }
 
-// The code stream of one weight warp: lane 0 keeps GV_STAGES positions of the
-// warp's range in flight (issue cursor: position iu = it S + is).
+// CTA jt < JT: tile jt of H^T, the sum of its S parts in K order, once their
+// flags are up (one thread per flag), published under the tile's flag (and
+// stored as fp32 H when asked).
+template <int NT>
+__device__ __forceinline__ void h_tile(const GemvParams &p, int jt) {
+  for (int s = threadIdx.x; s < p.S; s += GV_THREADS)
+    if (!wait_flag(p.hpflag + jt * p.S + s, p.tag, p.wait_limit)) latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+  __syncthreads();
+  const int n = 8 * NT * 16;
+  for (int e = threadIdx.x; e < n; e += GV_THREADS) {
+    const float *src = p.hpart + static_cast<int64_t>(jt) * p.S * n + e;
+    float h = 0.0f;
+    for (int s0 = 0; s0 < p.S; s0 += 16) {   // sixteen loads in flight, added in order
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = s0 + u < p.S ? __ldcg(src + static_cast<int64_t>(s0 + u) * n) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (s0 + u < p.S) h += v[u];
+    }
+    __stcg(p.hsum + jt * n + e, h);
+    const int tok = e >> 4, j = jt * 16 + (e & 15);
+    if (p.H_out && tok < p.M && j < p.r) p.H_out[static_cast<int64_t>(tok) * p.r + j] = h;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    st_release_gpu_u64(p.hflag + jt, p.tag);
+  }
+}
+
+// The code stream of one weight warp: lane 0 keeps GV_STAGES units of the
+// warp's range in flight (issue cursor: unit iu = it S + is).
 struct CodeStream {
   uint8_t *ring;
   uint64_t *bar;
@@ -327,45 +340,64 @@ struct CodeStream {
   }
 };
 
-// Phase 1, weight warp gw: positions [a, b).  The sum over the warp's part of
-// each tile it touches is stored, as soon as that part is done, as the tile's
-// piece gw - g0 (g0: the first warp on the tile).
-template <int NT, bool XS>
-__device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvParams &p, const XSource<NT, XS> &x,
-                                            CodeStream &cs, int gw, int a, int b) {
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int S = p.S;
-  const int KB = static_cast<int>(p.K / kBlock);
-  const int N = static_cast<int>(p.N);
-  const int first_tile = a / S;
-  int g0 = range_owner(first_tile * S, p.U, p.G);   // first warp on the current tile
-
-  // Block constants one position ahead in registers.  Rows past N and blocks
-  // past K read a clamped, valid address and are marked in bit 8 of q, so
-  // their weights decode to (signed) zero.
-  const float mu = dq_offset(p.tab);
-  int ft = first_tile, fs = a - first_tile * S, fu = a;
-  auto fetch = [&](PosConst &f) {
+// Block constants of a warp's units, one unit ahead in registers.  Rows past
+// N and blocks past K read a clamped, valid address and are marked in bit 8 of
+// q, so their weights decode to (signed) zero.
+// With p.cs_rows > 0 the CTA's constants are in shared memory: the bytes of
+// its rows from row r0 = 16 ta on (cq) and the group scales from group g0 on
+// (cs), see stage_constants.
+struct ConstStream {
+  int ft, fs, fu, b;   // cursor: unit fu = ft S + fs; the range ends at b
+  const uint8_t *cq;
+  const float *cs;
+  int r0, g0;
+  __device__ __forceinline__ ConstStream(int S, int a, int b_, const uint8_t *cq_, const float *cs_, int r0_, int g0_)
+      : ft(a / S), fs(a - (a / S) * S), fu(a), b(b_), cq(cq_), cs(cs_), r0(r0_), g0(g0_) {}
+  __device__ __forceinline__ void fetch(const GemvParams &p, PosConst &f) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const int KB = static_cast<int>(p.K / kBlock);
+    const int N = static_cast<int>(p.N);
     const int kb = 4 * fs + c;
     const int kbc = min(kb, KB - 1);
     const int n0 = ft * 16 + g;
     const int bi0 = min(n0, N - 1) * KB + kbc, bi1 = min(n0 + 8, N - 1) * KB + kbc;   // < 2^31 (host check)
     const bool kv = kb < KB;
-    f.q0 = ldg_once_u8(p.absmax_q + bi0) | ((kv && n0 < N) ? 0u : 0x100u);
-    f.q1 = ldg_once_u8(p.absmax_q + bi1) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
-    f.S0 = ldg_once_f32(p.group_scale + (bi0 >> 8));
-    f.S1 = ldg_once_f32(p.group_scale + (bi1 >> 8));
-    if (fu + 1 < b) {   // advance, staying on the last position of the range
+    if (p.cs_rows > 0) {
+      const int o = r0 * KB;
+      f.q0 = static_cast<uint32_t>(cq[bi0 - o]) | ((kv && n0 < N) ? 0u : 0x100u);
+      f.q1 = static_cast<uint32_t>(cq[bi1 - o]) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
+      f.S0 = cs[(bi0 >> 8) - g0];
+      f.S1 = cs[(bi1 >> 8) - g0];
+    } else {
+      f.q0 = ldg_once_u8(p.absmax_q + bi0) | ((kv && n0 < N) ? 0u : 0x100u);
+      f.q1 = ldg_once_u8(p.absmax_q + bi1) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
+      f.S0 = ldg_once_f32(p.group_scale + (bi0 >> 8));
+      f.S1 = ldg_once_f32(p.group_scale + (bi1 >> 8));
+    }
+    if (fu + 1 < b) {   // advance, staying on the last unit of the range
       ++fu;
-      if (++fs == S) {
+      if (++fs == p.S) {
         fs = 0;
         ++ft;
       }
     }
-  };
-  PosConst q;
-  fetch(q);
+  }
+};
+
+// Phase 2, warp `warp` of CTA c: units [a, b), the constants of unit a already
+// in q (fetched as early as the kernel may read the weight).  The warp's sum
+// over its part of each tile it touches is stored, as soon as that part is
+// done, in the CTA's piece slot (tile - ta) + warp (ta: the CTA's first tile).
+template <int NT, bool XS>
+__device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvParams &p, const XSource<NT, XS> &x,
+                                            CodeStream &cs, ConstStream &cst, PosConst q, int cta, int ta, int a,
+                                            int b) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int S = p.S;
+  const int KB = static_cast<int>(p.K / kBlock);
+  const int first_tile = a / S;
+  const float mu = dq_offset(p.tab);
 
   float acc[NT][4];
 #pragma unroll
@@ -374,10 +406,10 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
     for (int e = 0; e < 4; ++e) acc[tt][e] = 0.0f;
 
   int t = first_tile, step = a - first_tile * S;
-  int ip = 0;   // index of position u within the range
+  int ip = 0;   // index of unit u within the range
   for (int u = a; u < b; ++u, ++ip) {
     const PosConst f = q;
-    fetch(q);
+    cst.fetch(p, q);
 
     const int kbc = min(4 * step + c, KB - 1);
     uint4 xv[2][NT];   // activation words, read one word ahead
@@ -423,7 +455,7 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
         mma16816(acc[tt], o0[2], o1[2], o0[3], o1[3], xw.z, xw.w);
       }
     }
-    // every lane has used its codes: the slot takes the position GV_STAGES ahead
+    // every lane has used its codes: the slot takes the unit GV_STAGES ahead
     __syncwarp();
     if (lane == 0 && cs.iu < b) {
       fence_proxy_async_smem();
@@ -437,15 +469,14 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
     } else if (u + 1 < b) {
       continue;   // the tile continues in this warp's range
     }
-    // this warp's part of the tile is done: piece gw - g0
-    float *pc = p.pieces + (static_cast<int64_t>(tile) * p.P + (gw - g0)) * 16 * p.M;
-    g0 = gw;   // every later tile of the range starts in this warp
+    // this warp's part of the tile is done: its piece
+    float *pc = p.pieces + (static_cast<int64_t>(cta) * p.SLOTS + (tile - ta) + warp) * 16 * p.M;
 #pragma unroll
     for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = tt * 8 + 2 * c + (e & 1);
-        if (tok < p.M) pc[tok * 16 + g + 8 * (e >> 1)] = acc[tt][e];
+        if (tok < p.M) __stcg(pc + tok * 16 + g + 8 * (e >> 1), acc[tt][e]);
       }
 #pragma unroll
     for (int tt = 0; tt < NT; ++tt)
@@ -455,8 +486,9 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
 }
 
 // acc += (s H) B^T for the 16 rows of tile t: the rows of B are the A operand
-// (the adapter index j is the reduction index), s H the B operand, hi part then
-// lo part.  The loads of four 16-wide adapter steps are issued together.
+// (the adapter index j is the reduction index), s H the B operand as a bf16
+// pair hi + lo (hi = bf16(s H), lo = bf16(s H - hi)), formed from the tiles of
+// H in L2; the loads of four 16-wide adapter steps are issued together.
 template <int NT>
 __device__ __forceinline__ void add_lora(const GemvParams &p, int t, float (&acc)[NT][4], int lane) {
   const int g = lane >> 2, c = lane & 3;
@@ -465,7 +497,8 @@ __device__ __forceinline__ void add_lora(const GemvParams &p, int t, float (&acc
   const uint32_t *B0 = reinterpret_cast<const uint32_t *>(p.B + min(n0, p.N - 1) * p.r);
   const uint32_t *B1 = reinterpret_cast<const uint32_t *>(p.B + min(n1, p.N - 1) * p.r);
   for (int j0 = 0; j0 < p.r; j0 += 64) {
-    uint32_t a[4][4], h[4][NT][2], l[4][NT][2];
+    uint32_t a[4][4];
+    float hv[4][NT][4];   // H at token 8 tt + g, adapter indices ja, ja + 1, jb, jb + 1
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int ja = j0 + 16 * q + 2 * c, jb = ja + 8;   // ja < r whenever j0 + 16 q < r (r % 8 == 0)
@@ -476,16 +509,13 @@ __device__ __forceinline__ void add_lora(const GemvParams &p, int t, float (&acc
       a[q][2] = (v0 && vb) ? __ldg(B0 + jbc / 2) : 0u;
       a[q][3] = (v1 && vb) ? __ldg(B1 + jbc / 2) : 0u;
 #pragma unroll
-      for (int tt = 0; tt < NT; ++tt) {   // s H is padded to r16 columns
-        const int ra = min(ja, p.r16 - 2), rb = min(jb, p.r16 - 2);
-        const uint32_t *hr = reinterpret_cast<const uint32_t *>(p.sh_hi + (tt * 8 + g) * p.r16);
-        const uint32_t *lr = reinterpret_cast<const uint32_t *>(p.sh_lo + (tt * 8 + g) * p.r16);
-        // s H is read by every finishing warp: L1-cached loads (no SM holds a line
-        // of it from before the grid barrier, so none can be stale)
-        h[q][tt][0] = hr[ra / 2];
-        h[q][tt][1] = hr[rb / 2];
-        l[q][tt][0] = lr[ra / 2];
-        l[q][tt][1] = lr[rb / 2];
+      for (int tt = 0; tt < NT; ++tt) {
+        const int tok = tt * 8 + g;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = (i < 2 ? ja : jb) + (i & 1);
+          hv[q][tt][i] = j < p.r ? __ldcg(p.hsum + ((j >> 4) * 8 * NT + tok) * 16 + (j & 15)) : 0.0f;
+        }
       }
     }
 #pragma unroll
@@ -493,8 +523,16 @@ __device__ __forceinline__ void add_lora(const GemvParams &p, int t, float (&acc
       if (j0 + 16 * q < p.r) {
 #pragma unroll
         for (int tt = 0; tt < NT; ++tt) {
-          mma16816(acc[tt], a[q][0], a[q][1], a[q][2], a[q][3], h[q][tt][0], h[q][tt][1]);
-          mma16816(acc[tt], a[q][0], a[q][1], a[q][2], a[q][3], l[q][tt][0], l[q][tt][1]);
+          uint32_t hi[2], lo[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const float s0 = __fmul_rn(p.s, hv[q][tt][2 * h2]), s1 = __fmul_rn(p.s, hv[q][tt][2 * h2 + 1]);
+            const __nv_bfloat16 b0 = __float2bfloat16_rn(s0), b1 = __float2bfloat16_rn(s1);
+            hi[h2] = pack_bf16x2(__bfloat162float(b0), __bfloat162float(b1));
+            lo[h2] = pack_bf16x2(__fsub_rn(s0, __bfloat162float(b0)), __fsub_rn(s1, __bfloat162float(b1)));
+          }
+          mma16816(acc[tt], a[q][0], a[q][1], a[q][2], a[q][3], hi[0], hi[1]);
+          mma16816(acc[tt], a[q][0], a[q][1], a[q][2], a[q][3], lo[0], lo[1]);
         }
       }
     }
@@ -519,104 +557,181 @@ __device__ __forceinline__ void store_y(const GemvParams &p, int t, const float 
   }
 }
 
-// Phase 3: warp w of all W warps finishes tiles w, w + W, ...: the tile's
-// pieces in warp order (a fixed order), then the adapter term, then Y.  The
-// loads of the pieces, of the tile's rows of B and of s H are issued together.
+// Phase 3, per warp: the tiles whose last unit lies in this warp's range
+// [aw, bw).  A tile's pieces are added CTA by CTA (CTA order is K order) and,
+// within a CTA, warp by warp; the warp first waits for the flags of every
+// other warp on the tile (lanes poll in parallel) and of the tiles of H.
 template <int NT>
-__device__ __forceinline__ void finish_role(const GemvParams &p) {
+__device__ __forceinline__ void finish_tiles(const GemvParams &p, const int *starts, int cta, int aw, int bw) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int W = gridDim.x * GV_WARPS;
-  for (int t = blockIdx.x * GV_WARPS + warp; t < p.T; t += W) {
-    const int np = range_owner((t + 1) * p.S - 1, p.U, p.G) - range_owner(t * p.S, p.U, p.G) + 1;
-    const float *src = p.pieces + static_cast<int64_t>(t) * p.P * 16 * p.M;
+  const int S = p.S;
+  bool h_ready = false;
+  for (int t = aw / S; t <= (bw - 1) / S; ++t) {
+    const int last = (t + 1) * S - 1;
+    if (last < aw || last >= bw) continue;    // finished by a later warp
+    if (!h_ready) {
+      for (int i = lane; i < p.JT; i += 32)
+        if (!wait_flag(p.hflag + i, p.tag, p.wait_limit)) latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+      h_ready = true;
+    }
     float acc[NT][4];
 #pragma unroll
     for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[tt][e] = 0.0f;
-    constexpr int GV_PIECE_BATCH = 16 / NT;   // pieces loaded together
-    for (int i0 = 0; i0 < np; i0 += GV_PIECE_BATCH) {
-      float v[GV_PIECE_BATCH][NT][4];
+    const int c_first = cta_owner(starts, p.G, t * S);
+    for (int cp = c_first; cp <= cta; ++cp) {
+      const int ap = starts[cp], bp = starts[cp + 1];
+      if (bp <= ap) continue;
+      const int Lp = bp - ap, tap = ap / S;
+      const int ulo = max(t * S, ap), uhi = min((t + 1) * S, bp) - 1;
+      const int w0 = warp_owner(ap, Lp, ulo), w1 = warp_owner(ap, Lp, uhi);
+      // lane w polls warp w's flag (this warp's own piece needs none)
+      if (lane >= w0 && lane <= w1 && lane < GV_WARPS && !(cp == cta && lane == warp) &&
+          warp_start(ap, Lp, lane) != warp_start(ap, Lp, lane + 1) &&
+          !wait_flag(p.wflag + cp * GV_WARPS + lane, p.tag, p.wait_limit))
+        latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+      __syncwarp();
+      // the CTA's pieces of tile t sit in consecutive slots: all loads in flight, then added in warp order
+      const float *src = p.pieces + (static_cast<int64_t>(cp) * p.SLOTS + (t - tap)) * 16 * p.M;
+      float v[GV_WARPS][NT][4];
 #pragma unroll
-      for (int i = 0; i < GV_PIECE_BATCH; ++i)
+      for (int w = 0; w < GV_WARPS; ++w) {
+        const bool live = w >= w0 && w <= w1 && warp_start(ap, Lp, w) != warp_start(ap, Lp, w + 1);
 #pragma unroll
         for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int tok = tt * 8 + 2 * c + (e & 1);
-            v[i][tt][e] = (i0 + i < np && tok < p.M) ? __ldcg(src + ((i0 + i) * p.M + tok) * 16 + g + 8 * (e >> 1)) : 0.0f;
+            v[w][tt][e] = (live && tok < p.M) ? __ldcg(src + w * 16 * p.M + tok * 16 + g + 8 * (e >> 1)) : 0.0f;
           }
+      }
 #pragma unroll
-      for (int i = 0; i < GV_PIECE_BATCH; ++i)
+      for (int w = 0; w < GV_WARPS; ++w) {
+        if (w < w0 || w > w1 || warp_start(ap, Lp, w) == warp_start(ap, Lp, w + 1)) continue;
 #pragma unroll
         for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[tt][e] += v[i][tt][e];
+          for (int e = 0; e < 4; ++e) acc[tt][e] += v[w][tt][e];
+      }
     }
     add_lora<NT>(p, t, acc, lane);
     store_y<NT>(p, t, acc, lane);
   }
 }
 
-#ifndef QLORA_GEMV_MAXNREG
-#define QLORA_GEMV_MAXNREG 128
-#endif
+// The CTA's block constants into shared memory: the bytes of rows [r0, r1)
+// (one bulk copy of the 16-byte-aligned part, counted on `bar`; plain loads for
+// the rest) and the group scales g0 .. g1.  r0 = 16 ta is a multiple of 16, so
+// the copy starts on a 16-byte boundary.
+__device__ __forceinline__ uint32_t constants_bulk_bytes(const GemvParams &p, int r0, int r1) {
+  return static_cast<uint32_t>((static_cast<int64_t>(r1 - r0) * (p.K / kBlock)) & ~int64_t(15));
+}
+__device__ __forceinline__ void stage_constants(const GemvParams &p, uint8_t *cq, float *cs, int r0, int r1, int g0,
+                                                int g1, uint64_t *bar) {
+  const int KB = static_cast<int>(p.K / kBlock);
+  const int64_t o = static_cast<int64_t>(r0) * KB, n = static_cast<int64_t>(r1 - r0) * KB;
+  const uint32_t bulk = constants_bulk_bytes(p, r0, r1);
+  if (threadIdx.x == 0 && bulk > 0) bulk_load(cq, p.absmax_q + o, bulk, bar);
+  if (threadIdx.x < static_cast<int>(n - bulk)) cq[bulk + threadIdx.x] = p.absmax_q[o + bulk + threadIdx.x];
+  for (int i = threadIdx.x; i <= g1 - g0; i += GV_THREADS) cs[i] = __ldg(p.group_scale + g0 + i);
+}
+
 template <int NT, bool XS>
-__global__ void __maxnreg__(QLORA_GEMV_MAXNREG) gemv_kernel(const __grid_constant__ CUtensorMap tm_codes,
-                                                          const GemvParams p) {
+__global__ void __launch_bounds__(GV_THREADS, GV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ CUtensorMap tm_codes,
+                                                          const GemvParams p, int aux_off, int xs_off, int cq_off,
+                                                          int cs_off) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  int *starts = reinterpret_cast<int *>(smem + GV_START_OFFSET);
+  fill_starts(p, starts);   // read after the first CTA barrier below
+  const int a = cta_start(p, cta), b = cta_start(p, cta + 1);
+  const int L = b - a;
+  const int aw = warp_start(a, L, warp), bw = warp_start(a, L, warp + 1);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + GV_BAR_OFFSET);
+  uint64_t *xbar = bars + GV_WARPS * GV_STAGES;
+  CodeStream cs{smem + warp * GV_STAGES * GV_STAGE_BYTES, bars + warp * GV_STAGES, aw / p.S, aw - (aw / p.S) * p.S,
+                aw};
+
+  // Barriers, and the warp's first units brought into L2, while the kernel
+  // before this one may still be running (the weight is not written by it;
+  // a prefetch only warms L2, which stays coherent either way).
+  if (lane == 0) {
+    for (int i = 0; i < GV_STAGES; ++i) mbar_init(&cs.bar[i], 1);
+    if (warp == 0) mbar_init(xbar, 1);
+    fence_mbar_init();
+    int pt = cs.it, ps = cs.is;
+    for (int u = aw; u < bw && u < aw + GV_PREFETCH_UNITS; ++u) {
+      tma_prefetch_2d(&tm_codes, ps * 128, pt * 16);
+      if (++ps == p.S) {
+        ps = 0;
+        ++pt;
+      }
+    }
+  }
   // The next kernel on the stream may be scheduled once every CTA has passed
-  // here; nothing is read before the previous kernel's writes are visible.
+  // here; nothing the previous kernel writes is read before its results are visible.
   griddep_launch_dependents();
   griddep_wait();
-  grid_barrier_open(p.bar, p.epoch);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool h_cta = static_cast<int>(blockIdx.x) < p.JT * p.HS;
-  const int gw = (static_cast<int>(blockIdx.x) - p.JT * p.HS) * GV_WARPS + warp;   // weight warp index
-  const bool weight = !h_cta && gw < p.G;
-  const int a = weight ? range_start(gw, p.U, p.G) : 0, b = weight ? range_start(gw + 1, p.U, p.G) : 0;
-  float *red = reinterpret_cast<float *>(smem + GV_RED_OFFSET);
 
-  // The activations first (every warp needs them before its first product),
-  // then the first code boxes.
-  const uint32_t xs = smem_addr(smem + GV_XS_OFFSET);
-  uint64_t *xbar = reinterpret_cast<uint64_t *>(smem + GV_RING_BYTES) + GV_WARPS * GV_STAGES;
+  // This CTA's first part of H is loaded first (its result is waited for by
+  // every tile), then the activations (every warp needs them before its first
+  // product), then the first code boxes.
+  HLoad hl{};
+  if (cta < p.HP) hl = h_load(p, cta);
+  const uint32_t xs = smem_addr(smem + xs_off);
+  // the CTA's block constants (when they fit) and the activations arrive on xbar
+  const int KB = static_cast<int>(p.K / kBlock);
+  const int r0 = (a / p.S) * 16, r1 = L > 0 ? static_cast<int>(min(p.N, static_cast<int64_t>((b - 1) / p.S + 1) * 16)) : r0;
+  const int g0 = static_cast<int>((static_cast<int64_t>(r0) * KB) >> 8);
+  const int g1 = r1 > r0 ? static_cast<int>((static_cast<int64_t>(r1) * KB - 1) >> 8) : g0 - 1;
+  uint8_t *cq = smem + cq_off;
+  float *csc = reinterpret_cast<float *>(smem + cs_off);
+  if (threadIdx.x == 0)   // every byte the copies below bring (possibly none: the phase then ends here)
+    mbar_arrive_expect_tx(xbar, (p.cs_rows > 0 ? constants_bulk_bytes(p, r0, r1) : 0u) +
+                                    (XS ? static_cast<uint32_t>(p.K * 2 * p.M) : 0u));
+  if (p.cs_rows > 0) stage_constants(p, cq, csc, r0, r1, g0, g1, xbar);
   if (XS && threadIdx.x == 0) {
-    mbar_init(xbar, 1);
-    fence_mbar_init();
     const uint32_t row = static_cast<uint32_t>(p.K * 2);
-    mbar_arrive_expect_tx(xbar, row * p.M);
     for (int m = 0; m < p.M; ++m)
-      bulk_load(smem + GV_XS_OFFSET + m * p.xs_row, p.X + static_cast<int64_t>(m) * p.K, row, xbar);
+      bulk_load(smem + xs_off + m * p.xs_row, p.X + static_cast<int64_t>(m) * p.K, row, xbar);
   }
-  CodeStream cs{smem + warp * GV_STAGES * GV_STAGE_BYTES,
-                reinterpret_cast<uint64_t *>(smem + GV_RING_BYTES) + warp * GV_STAGES, a / p.S, a - (a / p.S) * p.S, a};
-  if (weight && lane == 0) {
-    for (int i = 0; i < GV_STAGES; ++i) mbar_init(&cs.bar[i], 1);
-    fence_mbar_init();
-    for (int i = 0; i < GV_STAGES && cs.iu < b; ++i) cs.issue(&tm_codes, i, p.S);
+  if (lane == 0)
+    for (int i = 0; i < GV_STAGES && cs.iu < bw; ++i) cs.issue(&tm_codes, i, p.S);
+  // the rows of B of the tiles this CTA finishes (the adapter term reads them
+  // last) are brought into L2 now as well
+  ConstStream cst(p.S, aw, bw, cq, csc, r0, g0);
+  if (L > 0 && threadIdx.x < 8) {
+    const int t = (b - 1) / p.S - static_cast<int>(threadIdx.x);   // a tile of the range, from the last
+    const int last = (t + 1) * p.S - 1;
+    if (t >= a / p.S && last >= a && last < b) {
+      const int64_t rows = min(static_cast<int64_t>(16), p.N - static_cast<int64_t>(t) * 16);
+      bulk_prefetch_l2(p.B + static_cast<int64_t>(t) * 16 * p.r, static_cast<uint32_t>(rows * p.r * 2));
+    }
   }
-  if (XS) {
-    __syncthreads();   // the barrier is initialised
-    if (!mbar_wait(xbar, 0, p.wait_limit)) latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
-  }
-  __syncwarp();
+  __syncthreads();   // every barrier is initialised, the plain constant loads are in shared memory
+  if (!mbar_wait(xbar, 0, p.wait_limit)) latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+  PosConst q0{};
+  if (aw < bw) cst.fetch(p, q0);
   const XSource<NT, XS> x(p, xs, lane >> 2);
 
-  if (h_cta) {
-    h_role<NT, XS>(p, x, red);
-  } else {
-    if (weight) weight_role<NT, XS>(&tm_codes, p, x, cs, gw, a, b);
+  for (int i = cta; i < p.HP; i += p.G) {
+    if (i != cta) hl = h_load(p, i);
+    h_part<NT, XS>(p, x, hl, i, reinterpret_cast<float *>(smem + aux_off));
   }
-
-  grid_barrier(p.bar, p.epoch, 1, p.status, p.wait_limit);   // pieces (and s H or its partial sums) complete and visible
-  if (p.HS > 1) {
-    h_finish<NT>(p);
-    grid_barrier(p.bar, p.epoch, 2, p.status, p.wait_limit);
+  if (cta < p.JT) h_tile<NT>(p, cta);
+  if (aw >= bw) return;
+  weight_role<NT, XS>(&tm_codes, p, x, cs, cst, q0, cta, a / p.S, aw, bw);
+  // this warp's pieces are stored: publish them
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    st_release_gpu_u64(p.wflag + cta * GV_WARPS + warp, p.tag);
   }
-  finish_role<NT>(p);
+  finish_tiles<NT>(p, starts, cta, aw, bw);
 }
 
 int device_sm_count() {
@@ -631,13 +746,15 @@ int device_sm_count() {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Work split and workspace carve-up shared by the size query and the launch.
-// The piece slots per tile are sized for the largest weight-warp count the
-// device can hold, so the layout does not depend on the occupancy found at launch.
+// The piece slots are sized for the longest CTA range of a launch with one CTA
+// per SM (more CTAs only shorten the ranges), and the per-CTA arrays for the
+// most CTAs a launch can have, so the layout does not depend on the occupancy
+// found at launch.
 struct GemvLayout {
-  int NT, r16, JT, HS, P;
-  int64_t T, S, U, G_max;
-  bool fits32;
-  size_t off_pieces, off_hpart, off_hi, off_lo, off_bar, total;
+  int NT, r16, JT, G_max, SLOTS;
+  int64_t T, S, U, HP;
+  bool ok;
+  size_t off_pieces, off_hpart, off_hsum, off_hpflag, off_hflag, off_wflag, total;
 };
 
 GemvLayout gemv_layout(int64_t M, int64_t N, int64_t K, int r) {
@@ -648,33 +765,38 @@ GemvLayout gemv_layout(int64_t M, int64_t N, int64_t K, int r) {
   L.T = ceil_div(N, int64_t(16));
   L.S = ceil_div(K / kBlock, int64_t(4));
   L.U = L.T * L.S;
-  // K parts of the adapter product: at most two 256-wide steps per H warp, at most ~32 H CTAs
-  L.HS = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(L.S, int64_t(2 * GV_WARPS)),
-                                                                  std::max(1, 32 / L.JT))));
-  const int64_t slots = static_cast<int64_t>(GV_CTAS_PER_SM) * device_sm_count() - static_cast<int64_t>(L.JT) * L.HS;
-  L.G_max = std::min<int64_t>(L.U, std::max<int64_t>(slots, 1) * GV_WARPS);
-  const int64_t lmin = std::max<int64_t>(L.U / L.G_max, 1);   // shortest weight-warp range
-  L.P = static_cast<int>(std::min<int64_t>(L.G_max, ceil_div(L.S, lmin) + 1));
-  L.fits32 = L.U <= INT32_MAX && N * (K / kBlock) <= INT32_MAX && L.T * L.P * 16 * M <= INT32_MAX;
+  L.HP = static_cast<int64_t>(L.JT) * L.S;   // parts of H
+  const int sms = device_sm_count();
+  L.G_max = GV_CTAS_PER_SM * sms;
+  const int64_t g_min = sms;   // fewest CTAs a launch runs with (one per SM)
+  L.ok = g_min > L.JT && L.G_max <= GV_MAX_CTAS && L.U < (int64_t(1) << 27) && L.HP <= INT32_MAX &&
+         N * (K / kBlock) <= INT32_MAX;
+  if (!L.ok) return L;
+  // longest CTA range at g_min CTAs or more: at most ceil(total / G) with total <=
+  // U + G pc + JT hc (pc, hc as the launch sets them)
+  const int64_t maxlen = ceil_div(L.U + static_cast<int64_t>(L.JT) * (QLORA_GEMV_HC + L.S / 16), g_min) + QLORA_GEMV_PC;
+  L.SLOTS = static_cast<int>(ceil_div(maxlen, L.S) + 1 + (GV_WARPS - 1));
+  L.ok = static_cast<int64_t>(L.G_max) * L.SLOTS * 16 * M <= INT32_MAX;
   size_t off = 0;
   L.off_pieces = off;
-  off += align256(static_cast<size_t>(L.T) * L.P * 16 * M * sizeof(float));
+  off += align256(static_cast<size_t>(L.G_max) * L.SLOTS * 16 * M * sizeof(float));
   L.off_hpart = off;
-  off += align256(static_cast<size_t>(L.JT) * L.HS * 8 * L.NT * 16 * sizeof(float));
-  const size_t sh = static_cast<size_t>(8 * L.NT) * L.r16 * sizeof(uint16_t);
-  L.off_hi = off;
-  off += align256(sh);
-  L.off_lo = off;
-  off += align256(sh);
-  L.off_bar = off;
-  off += 256;
+  off += align256(static_cast<size_t>(L.HP) * 8 * L.NT * 16 * sizeof(float));
+  L.off_hsum = off;
+  off += align256(static_cast<size_t>(L.JT) * 8 * L.NT * 16 * sizeof(float));
+  L.off_hpflag = off;
+  off += align256(static_cast<size_t>(L.HP) * sizeof(unsigned long long));
+  L.off_hflag = off;
+  off += align256(static_cast<size_t>(L.JT) * sizeof(unsigned long long));
+  L.off_wflag = off;
+  off += align256(static_cast<size_t>(L.G_max) * GV_WARPS * sizeof(unsigned long long));
   L.total = off;
   return L;
 }
 
-// A tag for each launch's barrier word: consecutive from a random start.
-uint32_t next_epoch() {
-  static std::atomic<uint32_t> next{static_cast<uint32_t>(std::random_device{}())};
+// A tag for each launch's flags: consecutive from a random 64-bit start.
+uint64_t next_tag() {
+  static std::atomic<uint64_t> next{(static_cast<uint64_t>(std::random_device{}()) << 32) ^ std::random_device{}()};
   return next.fetch_add(1);
 }
 
@@ -690,9 +812,21 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
     return QLORA_ERR_CUDA;
 
   const int KB = static_cast<int>(a.wK / kBlock);
+  // shared memory: ring, barriers and CTA starts, the H reduction, then (when they
+  // fit the per-CTA budget) the CTA's block constants and the activations
+  const int aux = GV_WARPS * NT * 4 * 32 * 4;
+  const int xs_off = GV_AUX_OFFSET + aux;
+  const int budget = smem_sm / GV_CTAS_PER_SM - 1024 - 1024;   // per-CTA reserve and alignment slack
+  const int cs_rows = 16 * (L.SLOTS - (GV_WARPS - 1));          // rows of the most tiles a CTA touches
+  const int64_t cq_bytes = (static_cast<int64_t>(cs_rows) * KB + 15) / 16 * 16 + 16;
+  const int64_t cs_bytes = ((static_cast<int64_t>(cs_rows) * KB / 256 + 2) * 4 + 15) / 16 * 16;
+  const bool cs_on = xs_off + cq_bytes + cs_bytes <= budget;
+  const int64_t c_total = cs_on ? cq_bytes + cs_bytes : 0;
   const int64_t xs_bytes = a.M * static_cast<int64_t>(xs_row_bytes(KB));
-  const bool xs = xs_bytes <= GV_XS_MAX;
-  const int smem = GV_SMEM_BASE + (xs ? static_cast<int>(xs_bytes) : 0);
+  const bool xs = xs_off + c_total + xs_bytes <= budget;
+  const int cq_off = xs_off + (xs ? static_cast<int>(xs_bytes) : 0);
+  const int cs_off = cq_off + (cs_on ? static_cast<int>(cq_bytes) : 0);
+  const int smem = static_cast<int>(cq_off + c_total) + 1024;
   auto kern = xs ? gemv_kernel<NT, true> : gemv_kernel<NT, false>;
   const int64_t need = static_cast<int64_t>(GV_CTAS_PER_SM) * (smem + 1024);
   const int pct = static_cast<int>(std::min<int64_t>(100, (need * 100 + smem_sm - 1) / smem_sm));
@@ -702,26 +836,57 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
   int occ = 0;   // every CTA must be resident at once (cooperative launch)
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, GV_THREADS, smem) != cudaSuccess || occ < 1)
     return QLORA_ERR_CUDA;
-  const int64_t hctas = static_cast<int64_t>(L.JT) * L.HS;
-  const int64_t resident = static_cast<int64_t>(std::min(occ, GV_CTAS_PER_SM)) * sms;
-  if (resident <= hctas) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  const int64_t ctas = std::min<int64_t>(hctas + ceil_div(L.U, int64_t(GV_WARPS)), resident);
-  const int64_t G = std::min<int64_t>(L.U, (ctas - hctas) * GV_WARPS);
-  if (G > L.G_max) return QLORA_ERR_CUDA;   // the piece slots were sized for at most G_max warps
+  const int G = std::min(occ, GV_CTAS_PER_SM) * sms;
+  if (G > L.G_max || G <= L.JT) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  // weight units given up for a part of H (one round trip for 16 bytes of A per thread)
+  // and for adding a tile of H (waiting for its parts, S loads per element), capped so
+  // the CTA ranges stay ordered
+  const int64_t per = L.U / G;
+  const int64_t pc = std::min<int64_t>(QLORA_GEMV_PC, per);
+  const int64_t hc = std::min<int64_t>(QLORA_GEMV_HC + L.S / 16, per - pc);
 
   CUtensorMap tm;   // codes as [N rows][K/2 bytes], boxes of 16 rows x 128 bytes
   if (!make_tmap_2d(&tm, a.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<uint64_t>(a.wK / 2),
                     static_cast<uint64_t>(a.wN), static_cast<uint64_t>(a.wK / 2), 128, 16,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return QLORA_ERR_CUDA;
-  GemvParams p{a.X, a.absmax_q, a.group_scale, a.A, a.B, a.s, a.Y, a.H_out,
-               reinterpret_cast<uint16_t *>(ws + L.off_hi), reinterpret_cast<uint16_t *>(ws + L.off_lo),
-               reinterpret_cast<float *>(ws + L.off_pieces), reinterpret_cast<float *>(ws + L.off_hpart),
-               reinterpret_cast<unsigned long long *>(ws + L.off_bar), next_epoch(), static_cast<int>(a.M), a.r, L.r16, L.JT, L.HS, static_cast<int>(G), static_cast<int>(L.S),
-               static_cast<int>(L.U), static_cast<int>(L.T), L.P, xs ? xs_row_bytes(KB) : 0, a.wN, a.wK, status,
-               wait_limit(), a.tab};
+  GemvParams p{};
+  p.X = a.X;
+  p.absmax_q = a.absmax_q;
+  p.group_scale = a.group_scale;
+  p.A = a.A;
+  p.B = a.B;
+  p.s = a.s;
+  p.Y = a.Y;
+  p.H_out = a.H_out;
+  p.pieces = reinterpret_cast<float *>(ws + L.off_pieces);
+  p.hpart = reinterpret_cast<float *>(ws + L.off_hpart);
+  p.hsum = reinterpret_cast<float *>(ws + L.off_hsum);
+  p.hpflag = reinterpret_cast<unsigned long long *>(ws + L.off_hpflag);
+  p.hflag = reinterpret_cast<unsigned long long *>(ws + L.off_hflag);
+  p.wflag = reinterpret_cast<unsigned long long *>(ws + L.off_wflag);
+  p.tag = next_tag();
+  p.M = static_cast<int>(a.M);
+  p.r = a.r;
+  p.r16 = L.r16;
+  p.JT = L.JT;
+  p.HP = static_cast<int>(L.HP);
+  p.pc = static_cast<int>(pc);
+  p.G = G;
+  p.S = static_cast<int>(L.S);
+  p.U = static_cast<int>(L.U);
+  p.T = static_cast<int>(L.T);
+  p.SLOTS = L.SLOTS;
+  p.hc = static_cast<int>(hc);
+  p.xs_row = xs ? xs_row_bytes(KB) : 0;
+  p.cs_rows = cs_on ? cs_rows : 0;
+  p.N = a.wN;
+  p.K = a.wK;
+  p.status = status;
+  p.wait_limit = wait_limit();
+  p.tab = a.tab;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
   cfg.blockDim = dim3(GV_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -732,7 +897,8 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, kern, tm, p) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, tm, p, GV_AUX_OFFSET, xs_off, cq_off, cs_off) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
 
@@ -740,12 +906,15 @@ qlora_status launch_gemv_nt(const GemvArgs &a, const GemvLayout &L, cudaStream_t
 
 bool gemv_enabled() { return true; }
 
-size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) { return gemv_layout(M, N, K, r).total; }
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  const GemvLayout L = gemv_layout(M, N, K, r);
+  return L.ok ? L.total : 256;
+}
 
 qlora_status launch_gemv(const GemvArgs &a, cudaStream_t st) {
   if (a.M < 1 || a.M > kGemvMaxTokens) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const GemvLayout L = gemv_layout(a.M, a.wN, a.wK, a.r);
-  if (!L.fits32) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!L.ok) return QLORA_ERR_UNSUPPORTED_SHAPE;
   prof_mark(kProfGemv, true, st);
   const qlora_status s = L.NT == 1 ? launch_gemv_nt<1>(a, L, st) : launch_gemv_nt<2>(a, L, st);
   prof_mark(kProfGemv, false, st);
