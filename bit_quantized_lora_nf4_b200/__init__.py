@@ -18,6 +18,10 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqlora.so")
+# The debug build: the same library with the kernels' global-memory indices
+# checked against their buffers (a miss latches QLORA_ERR_BOUNDS, no trap).
+# QLORA_DEBUG_BOUNDS=1 in the environment makes load() pick it.
+DEBUG_LIB_PATH = os.path.join(_HERE, "libqlora_debug.so")
 
 QLORA_OP_FWD = 0
 QLORA_OP_BWD = 1
@@ -29,6 +33,7 @@ STREAM_K_OFF, STREAM_K_AUTO, STREAM_K_ALWAYS = 0, 1, 2
 STATUS_NAMES = {
     0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED_SHAPE", 3: "QLORA_ERR_MISALIGNED",
     4: "QLORA_ERR_NONFINITE", 5: "QLORA_ERR_DEVICE_TIMEOUT", 6: "QLORA_ERR_CUDA", 7: "QLORA_ERR_WORKSPACE",
+    8: "QLORA_ERR_BOUNDS",
 }
 
 # Every symbol include/qlora.h declares.
@@ -79,14 +84,21 @@ MATERIALIZE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
                                   ctypes.c_void_p)
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libqlora.so once and declare the C signatures."""
-    global _lib
+_lib_path = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the library once (libqlora.so, or libqlora_debug.so when
+    QLORA_DEBUG_BOUNDS=1) and declare the C signatures."""
+    global _lib, _lib_path
     if _lib is not None:
         return _lib
+    if path is None:
+        path = DEBUG_LIB_PATH if os.environ.get("QLORA_DEBUG_BOUNDS") == "1" else LIB_PATH
     if not os.path.exists(path):
-        raise ImportError(f"libqlora.so not built at {path}; run python -m bit_quantized_lora_nf4_b200.build")
+        raise ImportError(f"{os.path.basename(path)} not built at {path}; run python -m bit_quantized_lora_nf4_b200.build")
     lib = ctypes.CDLL(path)
+    _lib_path = path
     vp, i64, sz, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
     wp = ctypes.POINTER(Nf4WeightC)
     sig = {
@@ -129,6 +141,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn.argtypes = args
     _lib = lib
     return lib
+
+
+def loaded_path() -> str | None:
+    """Path of the library load() opened (None before the first load)."""
+    return _lib_path
 
 
 def _check(code: int, where: str):

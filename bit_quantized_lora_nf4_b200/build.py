@@ -39,9 +39,16 @@ def sources():
     return sorted(f for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(OBJDIR, src.replace(".cu", ".o"))
-    cmd = [_nvcc()] + COMMON + (["-fmad=false"] if src in NO_FMAD else []) + [
+DEBUG_OBJDIR = os.path.join(OBJDIR, "debug")
+DEBUG_LIB = os.path.join(PKG, "libqlora_debug.so")
+# The debug build: global-memory indices of the quantizer, dequantizer and
+# few-token kernels checked against their buffers (QLORA_ERR_BOUNDS, no trap).
+DEBUG_FLAGS = ["-DQLORA_BOUNDS_CHECK"]
+
+
+def _compile(src: str, verbose: bool, debug: bool = False) -> str:
+    obj = os.path.join(DEBUG_OBJDIR if debug else OBJDIR, src.replace(".cu", ".o"))
+    cmd = [_nvcc()] + COMMON + (DEBUG_FLAGS if debug else []) + (["-fmad=false"] if src in NO_FMAD else []) + [
         "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -53,28 +60,30 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build libqlora.so (or, with debug=True, libqlora_debug.so) if a source is newer."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    os.makedirs(DEBUG_OBJDIR if debug else OBJDIR, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), sources()))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose, debug), sources()))
+    tmp = lib + ".tmp"
     cmd = [_nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcuda"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

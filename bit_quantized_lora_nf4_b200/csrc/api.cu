@@ -447,6 +447,7 @@ const char *qlora_status_string(qlora_status st) {
     case QLORA_ERR_DEVICE_TIMEOUT: return "QLORA_ERR_DEVICE_TIMEOUT";
     case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
     case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE";
+    case QLORA_ERR_BOUNDS: return "QLORA_ERR_BOUNDS";
   }
   return "QLORA_ERR_UNKNOWN";
 }

@@ -44,6 +44,20 @@ __device__ __forceinline__ void latch_status(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Bounds checks of the debug build (compiled with QLORA_BOUNDS_CHECK): an index
+// outside its buffer latches QLORA_ERR_BOUNDS and the caller skips the access
+// (no trap).  In the release build the check is compiled out.
+#ifdef QLORA_BOUNDS_CHECK
+__device__ __forceinline__ bool ql_in_bounds(int *status, int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  latch_status(status, QLORA_ERR_BOUNDS);
+  return false;
+}
+#define QL_IN_BOUNDS(status, idx, n) ::qlora::ql_in_bounds((status), static_cast<int64_t>(idx), static_cast<int64_t>(n))
+#else
+#define QL_IN_BOUNDS(status, idx, n) true
+#endif
+
 // ------------------------------------------------------------------ smem / mbarrier
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -281,14 +281,16 @@ __device__ __forceinline__ void h_part(const GemvParams &p, const XSource<NT, XS
 #pragma unroll
         for (int w = 0; w < GV_WARPS; ++w) v += red[((w * NT + t) * 4 + e) * 32 + lane];
         // C fragment: H^T[j0 + g + 8 (e >> 1)][tok = 8 t + 2 c + (e & 1)]
-        __stcg(dst + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1), v);
+        const int64_t o = static_cast<int64_t>(i) * 8 * NT * 16 + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1);
+        if (QL_IN_BOUNDS(p.status, o, static_cast<int64_t>(p.HP) * 8 * NT * 16))
+          __stcg(dst + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1), v);
       }
     }
   }
   __syncthreads();   // the part is stored, and red is free again
   if (threadIdx.x == 0) {
     __threadfence();
-    st_release_gpu_u64(p.hpflag + i, p.tag);
+    if (QL_IN_BOUNDS(p.status, i, p.HP)) st_release_gpu_u64(p.hpflag + i, p.tag);
   }
 }
 
@@ -307,19 +309,24 @@ __device__ __forceinline__ void h_tile(const GemvParams &p, int jt) {
     for (int s0 = 0; s0 < p.S; s0 += 16) {   // sixteen loads in flight, added in order
       float v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = s0 + u < p.S ? __ldcg(src + static_cast<int64_t>(s0 + u) * n) : 0.0f;
+      for (int u = 0; u < 16; ++u)
+        v[u] = (s0 + u < p.S && QL_IN_BOUNDS(p.status, (static_cast<int64_t>(jt) * p.S + s0 + u) * n + e,
+                                             static_cast<int64_t>(p.HP) * n))
+                   ? __ldcg(src + static_cast<int64_t>(s0 + u) * n)
+                   : 0.0f;
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         if (s0 + u < p.S) h += v[u];
     }
-    __stcg(p.hsum + jt * n + e, h);
+    if (QL_IN_BOUNDS(p.status, jt * n + e, p.JT * n)) __stcg(p.hsum + jt * n + e, h);
     const int tok = e >> 4, j = jt * 16 + (e & 15);
-    if (p.H_out && tok < p.M && j < p.r) p.H_out[static_cast<int64_t>(tok) * p.r + j] = h;
+    if (p.H_out && tok < p.M && j < p.r && QL_IN_BOUNDS(p.status, tok * p.r + j, p.M * p.r))
+      p.H_out[static_cast<int64_t>(tok) * p.r + j] = h;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    st_release_gpu_u64(p.hflag + jt, p.tag);
+    if (QL_IN_BOUNDS(p.status, jt, p.JT)) st_release_gpu_u64(p.hflag + jt, p.tag);
   }
 }
 
@@ -364,10 +371,15 @@ struct ConstStream {
     const bool kv = kb < KB;
     if (p.cs_rows > 0) {
       const int o = r0 * KB;
-      f.q0 = static_cast<uint32_t>(cq[bi0 - o]) | ((kv && n0 < N) ? 0u : 0x100u);
-      f.q1 = static_cast<uint32_t>(cq[bi1 - o]) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
-      f.S0 = cs[(bi0 >> 8) - g0];
-      f.S1 = cs[(bi1 >> 8) - g0];
+      const int64_t nq = static_cast<int64_t>(p.cs_rows) * KB, ns = nq / 256 + 2;
+      (void)nq;
+      (void)ns;
+      const bool in = QL_IN_BOUNDS(p.status, bi0 - o, nq) && QL_IN_BOUNDS(p.status, bi1 - o, nq) &&
+                      QL_IN_BOUNDS(p.status, (bi0 >> 8) - g0, ns) && QL_IN_BOUNDS(p.status, (bi1 >> 8) - g0, ns);
+      f.q0 = (in ? static_cast<uint32_t>(cq[bi0 - o]) : 0u) | ((kv && n0 < N) ? 0u : 0x100u);
+      f.q1 = (in ? static_cast<uint32_t>(cq[bi1 - o]) : 0u) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
+      f.S0 = in ? cs[(bi0 >> 8) - g0] : 0.0f;
+      f.S1 = in ? cs[(bi1 >> 8) - g0] : 0.0f;
     } else {
       f.q0 = ldg_once_u8(p.absmax_q + bi0) | ((kv && n0 < N) ? 0u : 0x100u);
       f.q1 = ldg_once_u8(p.absmax_q + bi1) | ((kv && n0 + 8 < N) ? 0u : 0x100u);
@@ -470,13 +482,16 @@ __device__ __forceinline__ void weight_role(const CUtensorMap *tm, const GemvPar
       continue;   // the tile continues in this warp's range
     }
     // this warp's part of the tile is done: its piece
-    float *pc = p.pieces + (static_cast<int64_t>(cta) * p.SLOTS + (tile - ta) + warp) * 16 * p.M;
+    const int64_t pbase = (static_cast<int64_t>(cta) * p.SLOTS + (tile - ta) + warp) * 16 * p.M;
+    float *pc = p.pieces + pbase;
 #pragma unroll
     for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = tt * 8 + 2 * c + (e & 1);
-        if (tok < p.M) __stcg(pc + tok * 16 + g + 8 * (e >> 1), acc[tt][e]);
+        if (tok < p.M &&
+            QL_IN_BOUNDS(p.status, pbase + tok * 16 + g + 8 * (e >> 1), static_cast<int64_t>(p.G) * p.SLOTS * 16 * p.M))
+          __stcg(pc + tok * 16 + g + 8 * (e >> 1), acc[tt][e]);
       }
 #pragma unroll
     for (int tt = 0; tt < NT; ++tt)
@@ -514,7 +529,9 @@ __device__ __forceinline__ void add_lora(const GemvParams &p, int t, float (&acc
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int j = (i < 2 ? ja : jb) + (i & 1);
-          hv[q][tt][i] = j < p.r ? __ldcg(p.hsum + ((j >> 4) * 8 * NT + tok) * 16 + (j & 15)) : 0.0f;
+          hv[q][tt][i] = (j < p.r && QL_IN_BOUNDS(p.status, ((j >> 4) * 8 * NT + tok) * 16 + (j & 15), p.JT * 8 * NT * 16))
+                             ? __ldcg(p.hsum + ((j >> 4) * 8 * NT + tok) * 16 + (j & 15))
+                             : 0.0f;
         }
       }
     }
@@ -549,7 +566,7 @@ __device__ __forceinline__ void store_y(const GemvParams &p, int t, const float 
     for (int e = 0; e < 4; ++e) {
       const int tok = tt * 8 + 2 * c + (e & 1);
       const int64_t n = n0 + 8 * (e >> 1);
-      if (tok < p.M && n < p.N) {
+      if (tok < p.M && n < p.N && QL_IN_BOUNDS(p.status, tok * p.N + n, p.M * p.N)) {
         const __nv_bfloat16 y = __float2bfloat16_rn(acc[tt][e]);
         p.Y[static_cast<int64_t>(tok) * p.N + n] = *reinterpret_cast<const uint16_t *>(&y);
       }
@@ -604,7 +621,12 @@ __device__ __forceinline__ void finish_tiles(const GemvParams &p, const int *sta
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int tok = tt * 8 + 2 * c + (e & 1);
-            v[w][tt][e] = (live && tok < p.M) ? __ldcg(src + w * 16 * p.M + tok * 16 + g + 8 * (e >> 1)) : 0.0f;
+            v[w][tt][e] = (live && tok < p.M &&
+                           QL_IN_BOUNDS(p.status, (static_cast<int64_t>(cp) * p.SLOTS + (t - tap) + w) * 16 * p.M +
+                                                      tok * 16 + g + 8 * (e >> 1),
+                                        static_cast<int64_t>(p.G) * p.SLOTS * 16 * p.M))
+                              ? __ldcg(src + w * 16 * p.M + tok * 16 + g + 8 * (e >> 1))
+                              : 0.0f;
           }
       }
 #pragma unroll
@@ -729,7 +751,8 @@ __global__ void __launch_bounds__(GV_THREADS, GV_CTAS_PER_SM) gemv_kernel(const 
   __syncwarp();
   if (lane == 0) {
     __threadfence();
-    st_release_gpu_u64(p.wflag + cta * GV_WARPS + warp, p.tag);
+    if (QL_IN_BOUNDS(p.status, cta * GV_WARPS + warp, p.G * GV_WARPS))
+      st_release_gpu_u64(p.wflag + cta * GV_WARPS + warp, p.tag);
   }
   finish_tiles<NT>(p, starts, cta, aw, bw);
 }

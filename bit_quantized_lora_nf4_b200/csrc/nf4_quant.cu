@@ -161,6 +161,9 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
   const int64_t g = blockIdx.x;
   const int64_t base = g * kGroupElems;
   const int64_t nblocks = (numel + kBlock - 1) / kBlock;
+  const int64_t code_bytes = (numel + 1) / 2, ngroups = (nblocks + kGroup - 1) / kGroup;
+  (void)code_bytes;
+  (void)ngroups;
   bool bad = false;
 
   if (base + kGroupElems <= numel && (reinterpret_cast<uintptr_t>(W) & 15u) == 0) {
@@ -180,7 +183,8 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
       const uint32_t c1 = encode_nf4(block_norm(x.y, m), s_thr);
       const uint32_t c2 = encode_nf4(block_norm(x.z, m), s_thr);
       const uint32_t c3 = encode_nf4(block_norm(x.w, m), s_thr);
-      C2[it * kQuantThreads + t] = static_cast<uint16_t>(c0 | (c1 << 4) | (c2 << 8) | (c3 << 12));
+      if (QL_IN_BOUNDS(status, base / 2 + 2 * (it * kQuantThreads + t) + 1, code_bytes))
+        C2[it * kQuantThreads + t] = static_cast<uint16_t>(c0 | (c1 << 4) | (c2 << 8) | (c3 << 12));
     }
   } else {
     const int64_t blk = g * kGroup + t;
@@ -196,7 +200,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
       for (int64_t e = e0; e < e1; e += 2) {
         const uint32_t lo = encode_nf4(block_norm(load_weight(W, e), a), s_thr);
         const uint32_t hi = (e + 1 < e1) ? encode_nf4(block_norm(load_weight(W, e + 1), a), s_thr) : 0u;
-        codes[e / 2] = static_cast<uint8_t>(lo | (hi << 4));
+        if (QL_IN_BOUNDS(status, e / 2, code_bytes)) codes[e / 2] = static_cast<uint8_t>(lo | (hi << 4));
       }
     }
     s_abs[t] = a;
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
     // Signed constants: keep a_b for the second pass and add it to the exact sum.
     const float a = s_abs[t];
     const int64_t blk = g * kGroup + t;
-    if (blk < nblocks) dq_abs[blk] = a;
+    if (blk < nblocks && QL_IN_BOUNDS(status, blk, nblocks)) dq_abs[blk] = a;
     warp_exact_add(a, s_acc);
     __syncthreads();
     if (t < kSumDigits && s_acc[t] != 0) atomicAdd(dq_acc + t, s_acc[t]);
@@ -230,9 +234,9 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const TW *_
   if (blk < nblocks) {
     uint32_t q = 0;
     if (S != 0.0f) q = static_cast<uint32_t>(fminf(rintf(__fdiv_rn(a, S)), 255.0f));
-    absmax_q[blk] = static_cast<uint8_t>(q);
+    if (QL_IN_BOUNDS(status, blk, nblocks)) absmax_q[blk] = static_cast<uint8_t>(q);
   }
-  if (t == 0) group_scale[g] = S;
+  if (t == 0 && QL_IN_BOUNDS(status, g, ngroups)) group_scale[g] = S;
   if (bad) latch_status(status, QLORA_ERR_NONFINITE);
 }
 
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_dq_signed_kernel(const floa
                                                                       const unsigned long long *__restrict__ dq_acc,
                                                                       int64_t nblocks, uint8_t *__restrict__ absmax_q,
                                                                       float *__restrict__ group_scale,
-                                                                      float *__restrict__ mu_out) {
+                                                                      float *__restrict__ mu_out, int *status) {
   __shared__ float s_mu;
   __shared__ float s_wmax[kQuantThreads / 32];
   const int t = threadIdx.x;
@@ -264,9 +268,10 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_dq_signed_kernel(const floa
   if (blk < nblocks) {
     int q = 0;
     if (S != 0.0f) q = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(c, S)), -127.0f), 127.0f));
-    absmax_q[blk] = static_cast<uint8_t>(q & 0xFF);
+    if (QL_IN_BOUNDS(status, blk, nblocks)) absmax_q[blk] = static_cast<uint8_t>(q & 0xFF);
   }
-  if (t == 0) group_scale[g] = S;
+  if (t == 0 && QL_IN_BOUNDS(status, g, (nblocks + kGroup - 1) / kGroup)) group_scale[g] = S;
+  (void)status;
   if (g == 0 && t == 0) *mu_out = mu;
 }
 
@@ -279,7 +284,8 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
                                                                      const uint8_t *__restrict__ absmax_q,
                                                                      const float *__restrict__ group_scale,
                                                                      int64_t numel, uint16_t *__restrict__ out,
-                                                                     Nf4Table tab) {
+                                                                     Nf4Table tab, int *status) {
+  (void)status;
   const int64_t nchunk = (numel + 31) / 32;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const float mu = dq_offset(tab);
@@ -297,14 +303,14 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
       for (int w = 0; w < 4; ++w) {
         uint32_t o[4];
         nf4_lut8(words[w], LO, HI, o);
-        __stcs(dst + w, make_uint4(o[0], o[1], o[2], o[3]));
+        if (QL_IN_BOUNDS(status, e0 + 8 * w + 7, numel)) __stcs(dst + w, make_uint4(o[0], o[1], o[2], o[3]));
       }
     } else {
       for (int64_t e = e0; e < numel; ++e) {
         const uint32_t cd = (codes[e >> 1] >> (4 * (e & 1))) & 15u;
         uint32_t o[4];
         nf4_lut8(cd, LO, HI, o);                 // code in nibble 0 -> T[cd] in the low half of o[0]
-        out[e] = static_cast<uint16_t>(o[0] & 0xFFFFu);
+        if (QL_IN_BOUNDS(status, e, numel)) out[e] = static_cast<uint16_t>(o[0] & 0xFFFFu);
       }
     }
   }
@@ -333,8 +339,9 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
                                                                           const uint8_t *__restrict__ absmax_q,
                                                                           const float *__restrict__ group_scale,
                                                                           int64_t nchunks, uint16_t *__restrict__ out,
-                                                                          Nf4Table tab, int *status,
+                                                                          int64_t out_elems, Nf4Table tab, int *status,
                                                                           uint64_t wait_limit) {
+  (void)out_elems;
   extern __shared__ __align__(128) uint8_t dq_smem[];
   uint8_t *cbuf = dq_smem;                                         // [kDqStages][kDqStageBytes]
   uint8_t *obuf = dq_smem + kDqStages * kDqStageBytes;             // [2][kDqOutBytes]
@@ -385,7 +392,8 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
     fence_proxy_async_smem();
     __syncthreads();   // stage ls is consumed and obuf[ob] is written
     if (t == 0) {
-      bulk_store(out + ch * kDqChunk, obuf + ob * kDqOutBytes, kDqOutBytes);
+      if (QL_IN_BOUNDS(status, (ch + 1) * kDqChunk - 1, out_elems))
+        bulk_store(out + ch * kDqChunk, obuf + ob * kDqOutBytes, kDqOutBytes);
       bulk_commit();
       if (first + issued * step < nchunks) issue(issued++);   // refill stage ls, kDqStages chunks ahead
     }
@@ -428,7 +436,7 @@ cudaError_t launch_quantize(const void *W, int dtype, int64_t numel, uint8_t *co
         static_cast<const float *>(W), numel, codes, absmax_q, group_scale, tab, abs_ws, acc, status);
   if (sgn)
     nf4_dq_signed_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, st>>>(
-        abs_ws, acc, nblocks, absmax_q, group_scale, const_cast<float *>(tab.offset));
+        abs_ws, acc, nblocks, absmax_q, group_scale, const_cast<float *>(tab.offset), status);
   prof_mark(kProfQuant, false, st);
   return cudaGetLastError();
 }
@@ -445,7 +453,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
                                          kDqSmem);
     if (e != cudaSuccess) return e;
     nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, kDqSmem, st>>>(
-        codes, absmax_q, group_scale, nfull, out, tab, status, wait_limit());
+        codes, absmax_q, group_scale, nfull, out, numel, tab, status, wait_limit());
   }
   const int64_t done = nfull * kDqChunk;
   if (done < numel) {
@@ -455,7 +463,8 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
     const int64_t nchunk = (rest + 31) / 32;
     int64_t blocks = (nchunk + kDeqThreads - 1) / kDeqThreads;
     nf4_dequantize_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, 0, st>>>(
-        codes + done / 2, absmax_q + done / kBlock, group_scale + done / (kBlock * kGroup), rest, out + done, tab);
+        codes + done / 2, absmax_q + done / kBlock, group_scale + done / (kBlock * kGroup), rest, out + done, tab,
+        device_status_ptr());
   }
   prof_mark(kProfDequant, false, st);
   return cudaGetLastError();

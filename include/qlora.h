@@ -36,6 +36,10 @@
  *     the quantizer, a pipeline wait that exceeded its bound) are latched in a
  *     device status word; read and clear it with qlora_device_status().
  *   - Outputs are overwritten, never accumulated into.
+ *   - The debug build of the library (libqlora_debug.so, compiled with
+ *     QLORA_BOUNDS_CHECK) checks the global-memory indices of the quantizer,
+ *     the dequantizer and the few-token forward against their buffers; a miss
+ *     latches QLORA_ERR_BOUNDS and skips the access instead of trapping.
  *   - The library caches per-device state on first use (the device addresses
  *     of its status word and scratch array, its side streams and events); do
  *     not reset a device (cudaDeviceReset) after calling the library on it.
@@ -62,7 +66,9 @@ typedef enum {
   QLORA_ERR_NONFINITE = 4,         /* device: non-finite weight seen by quantizer  */
   QLORA_ERR_DEVICE_TIMEOUT = 5,    /* device: a pipeline wait exceeded its bound   */
   QLORA_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed            */
-  QLORA_ERR_WORKSPACE = 7          /* workspace missing or smaller than required   */
+  QLORA_ERR_WORKSPACE = 7,         /* workspace missing or smaller than required   */
+  QLORA_ERR_BOUNDS = 8             /* device, debug build only: an index outside its
+                                      buffer was caught and the access skipped     */
 } qlora_status;
 
 /* The frozen base weight W [rows=N (out), cols=K (in)] in NF4 + double quant.

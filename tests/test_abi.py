@@ -252,3 +252,14 @@ def test_noalloc_scratch_size_and_documented_limits():
         assert lib.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 863, N, K, 256) > lim
         # the stream-K tail never fits beside the forward
         assert lib.qlora_workspace_bytes(q.QLORA_OP_FWD, 256, N, K, 64) > lim
+
+
+def test_debug_library_exports_every_declared_symbol():
+    """The bounds-checked debug build (built beside the release library) loads
+    and exports the same C ABI."""
+    assert os.path.exists(q.DEBUG_LIB_PATH), "libqlora_debug.so not built"
+    dbg = ctypes.CDLL(q.DEBUG_LIB_PATH)
+    for name in _declared():
+        assert hasattr(dbg, name), name
+    dbg.qlora_status_string.restype = ctypes.c_char_p
+    assert dbg.qlora_status_string(8).decode() == "QLORA_ERR_BOUNDS"
