@@ -280,14 +280,15 @@ Plan make_plan(int op, int64_t M, int64_t N, int64_t K, int r, bool packed = tru
     return p;
   }
   skinny_plan(M, r, K, &p.spH, &p.kpsH);
-  size_t part = static_cast<size_t>(p.spH) * Mr;
+  size_t part = skinny_part_floats(M, r, p.spH);
   if (op == QLORA_OP_BWD) {
     skinny_plan(M, r, N, &p.spG, &p.kpsG);
-    skinny_plan(N, 2 * r, M, &p.spB, &p.kpsB);
-    skinny_plan(2 * r, K, M, &p.spA, &p.kpsA);
-    part = std::max(part, static_cast<size_t>(p.spG) * Mr);
-    part = std::max(part, static_cast<size_t>(p.spB) * N * 2 * r);
-    part = std::max(part, static_cast<size_t>(p.spA) * 2 * r * K);
+    // dB and dA share one launch (one split count over their tiles together)
+    skinny_plan_pair(N, 2 * r, 2 * r, K, M, &p.spB, &p.kpsB);
+    p.spA = p.spB;
+    p.kpsA = p.kpsB;
+    part = std::max(part, skinny_part_floats(M, r, p.spG));
+    part = std::max(part, skinny_part_floats(N, 2 * r, p.spB) + skinny_part_floats(2 * r, K, p.spA));
   }
   p.part = take(part * 4);
   p.H = take(Mr * 4);
@@ -647,20 +648,24 @@ qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint
                 p.kpsA, part};
   aA.ep.kind = kSkinnyRows;
   aA.ep.out_f = dA;
-  // Both finishing in-kernel (no shared partial buffer): they run on the side
-  // stream, beside the dgrad GEMM.
+  // Both finishing in-kernel (no shared partial buffer): one launch of the two,
+  // on the side stream beside the dgrad GEMM.
   // (Off while the timing hook records, so that every kernel's events time it alone.)
-  SideStream *side = (skinny_fused_ok(aB) && skinny_fused_ok(aA) && !prof_on()) ? side_stream() : nullptr;
+  const bool paired = skinny_pair_ok(aB, aA);
+  SideStream *side = (paired && !prof_on()) ? side_stream() : nullptr;
   if (side) {
     QL_CUDA(cudaEventRecord(side->fork, st));
     QL_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
     // dX = dY W' + Gb A first, so that its CTAs are dispatched ahead of the products'
     const qlora_status gst = launch_qgemm(dgrad, st);
-    QL_CUDA(launch_skinny(aB, side->s));
-    QL_CUDA(launch_skinny(aA, side->s));
+    QL_CUDA(launch_skinny_pair(aB, aA, side->s));
     QL_CUDA(cudaEventRecord(side->join, side->s));
     QL_CUDA(cudaStreamWaitEvent(st, side->join, 0));
     return gst;
+  }
+  if (paired) {
+    QL_CUDA(launch_skinny_pair(aB, aA, st));
+    return launch_qgemm(dgrad, st);
   }
   if (skinny_fused_ok(aB)) {
     QL_CUDA(launch_skinny(aB, st));

@@ -142,8 +142,18 @@ struct SkinnyArgs {
 // Whether the product can finish inside the kernel (cluster of its splits).
 bool skinny_fused_ok(const SkinnyArgs &a);
 cudaError_t launch_skinny(const SkinnyArgs &a, cudaStream_t st);
-// Pick the split count for a skinny product (deterministic in the sizes).
+// fp32 partial sums a product's launch may write (part): the larger of the
+// fused layout [tile][split][128 x min(128, J)] and the plain [split][I][J].
+// Two products in one launch take the first's floats and then the second's.
+size_t skinny_part_floats(int64_t I, int64_t J, int splits);
+// Two fused products in one launch: same operand layouts and split count.
+bool skinny_pair_ok(const SkinnyArgs &a, const SkinnyArgs &b);
+cudaError_t launch_skinny_pair(const SkinnyArgs &a, const SkinnyArgs &b, cudaStream_t st);
+// Pick the split count for a skinny product, or for two sharing one launch
+// and one reduction length (deterministic in the sizes).
 void skinny_plan(int64_t I, int64_t J, int64_t Kred, int *splits, int64_t *k_per_split);
+void skinny_plan_pair(int64_t I0, int64_t J0, int64_t I1, int64_t J1, int64_t Kred, int *splits,
+                      int64_t *k_per_split);
 
 // Epilogues of the skinny products.
 //   H  = sum_z part            -> H (fp32 [M,r]); sH = bf16(s*H) [M,r]; Hs = [bf16 hi | bf16 lo] [M,2r] (optional)

@@ -23,7 +23,7 @@
 // call (a reset reloads the module, and the array may move).
 //
 // The array covers the forward's minimum workspace only: the minimum grows
-// with M r (about 2.4 KB per token at r = 64, so M <= 3449 there), and the
+// with M r (about 2.4 KB per token at r = 64, so M <= 3413 there), and the
 // fused GEMM's optional stream-K region (about 80 MB for M > 128) never fits,
 // so the GEMM always runs without the stream-K split of a partial last wave.
 #include <mutex>

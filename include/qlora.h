@@ -277,7 +277,8 @@ qlora_status qlora_linear_bwd_materialized(qlora_materialize_fn materialize, voi
  *   Returns QLORA_ERR_WORKSPACE (nothing enqueued) when
  *   qlora_workspace_min_bytes(QLORA_OP_FWD, M, N, K, r) exceeds
  *   QLORA_STATIC_SCRATCH_BYTES.  That minimum grows with M r and does not
- *   depend on N or K: at r = 64 it is about 2.4 KB per token, so M <= 3449 fits
+ *   depend on N or K: at r = 64 it is about 2.4 KB per token (the adapter
+ *   product's fp32 partial sums, in whole 128-token tiles), so M <= 3413 fits
  *   (M = 2048, r = 64 fits; M = 4096, r = 64 does not); at r = 256, M <= 862.
  *   The fused GEMM always runs without its stream-K tail here (that optional
  *   workspace region is about 80 MB for M > 128), so a partial last wave of

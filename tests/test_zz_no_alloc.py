@@ -68,8 +68,8 @@ def test_noalloc_documented_size_limits(lib):
     lib_ = q.load()
     limit = q.QLORA_STATIC_SCRATCH_BYTES
     assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 2048, 4096, 4096, 64) <= limit
-    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3449, 4096, 4096, 64) <= limit
-    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3450, 4096, 4096, 64) > limit
+    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3413, 4096, 4096, 64) <= limit
+    assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 3414, 4096, 4096, 64) > limit
     assert lib_.qlora_workspace_min_bytes(q.QLORA_OP_FWD, 4096, 4096, 4096, 64) > limit
     # fits: runs, and equals the ordinary entry point within the parity tolerance
     _check_case(qi.LinearCase("noalloc_fits", 2048, 4096, 4096, 64, 16.0, 73))
