@@ -96,7 +96,11 @@ constexpr int MAX_D_STAGES = 8;
 static_assert(Cfg<1>::D_STAGES >= 2 && Cfg<2>::D_STAGES <= MAX_D_STAGES, "operand ring depth");
 constexpr uint64_t kDrainLimit = 4000000000ull;
 constexpr int kFwdLanes = 2;                // odd CTA: lanes forwarding readiness, steps in turn
-constexpr int kGroupM = 8;                  // M-pairs per raster group
+constexpr int kGroupM = 8;                  // M-pairs per raster group (default)
+// Raster per launch (compile-time switch for comparisons: 0 keeps kGroupM).
+#ifndef QLORA_PAIR_RASTER_AUTO
+#define QLORA_PAIR_RASTER_AUTO 1
+#endif
 // Stream-K tail: the tiles left after the last full wave have their K-steps
 // split evenly over the cluster slots; a workspace provides for kSkMaxUnits
 // such clusters, and none takes fewer than kSkMinSteps K-steps.  Measured on
@@ -125,6 +129,7 @@ struct Params {
   int nkb;           // weight K-steps (of 128)
   int nls;           // adapter K-steps (of 128)
   int num_m, num_n;  // pair tiles along M and along the output columns
+  int group_m;       // M-pairs per raster group
   uint16_t *out;
   int *status;
   uint64_t wait_limit;
@@ -155,12 +160,12 @@ constexpr int SMEM_BYTES = A_STAGES * A_BYTES + D_RING + 1024 + static_cast<int>
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(A_STAGES * A_BYTES >= NUM_DEC_WARPS * 16384, "epilogue staging fits the activation ring");
 
-// Tile t of the grouped raster: consecutive tiles walk kGroupM M-pairs before
+// Tile t of the grouped raster: consecutive tiles walk group_m M-pairs before
 // moving to the next N tile, so a wave reuses both operands from L2.
 __device__ __forceinline__ void tile_coords(const Params &p, int t, int &pm, int &pn) {
-  const int in_group = kGroupM * p.num_n;
-  const int first_m = (t / in_group) * kGroupM;
-  const int gsz = min(p.num_m - first_m, kGroupM);
+  const int in_group = p.group_m * p.num_n;
+  const int first_m = (t / in_group) * p.group_m;
+  const int gsz = min(p.num_m - first_m, p.group_m);
   pm = first_m + (t % in_group) % gsz;
   pn = (t % in_group) / gsz;
 }
@@ -905,6 +910,14 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
   p.num_n = static_cast<int>(ceil_div(n_out, BN));
   const int tiles = p.num_m * p.num_n;
   p.dp_tiles = tiles;
+  // Raster: a wave of kGroupM-row groups touches every M-pair, so an activation
+  // too large to stay in L2 is read from DRAM once per round of tiles (about
+  // 2.6 times for the 90 MB operands at 1.73 rounds), while each weight tile is
+  // read about once.  Walking one M-pair's tiles at a time reads the activation
+  // about once and the (packed, smaller) weight once per round instead.
+  const double act_bytes = static_cast<double>(a.M) * static_cast<double>(kred) * 2.0;
+  const double w_bytes = static_cast<double>(a.wN) * static_cast<double>(a.wK) * (a.wdense ? 2.0 : 0.5);
+  p.group_m = QLORA_PAIR_RASTER_AUTO && act_bytes >= 64.0 * (1 << 20) && act_bytes > 2.0 * w_bytes ? 1 : kGroupM;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);        // set per launch below (the occupancy query reads the rest)
