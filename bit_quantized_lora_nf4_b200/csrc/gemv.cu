@@ -23,12 +23,13 @@
 //      m16n8k16 A fragments (tokens are the 8-column B operand; two column
 //      tiles when M > 8).  For every tile it touches it stores its fp32 sum
 //      as a piece in the CTA's slot (tile - first tile of the CTA) + warp.
-//   3. The CTA stamps its flag once all its pieces are stored, gathers s H
-//      from the JT tiles of H into shared memory, and finishes
-//      the tiles whose last unit it holds: the pieces of every CTA on the
-//      tile, in CTA order and warp order within a CTA (a fixed order, so
-//      results do not depend on timing), waiting only for the flags of the
-//      earlier CTAs on that tile; then (s H) B^T and bf16 Y.
+//   3. Each warp stamps its own flag once its pieces are stored and finishes
+//      the tiles whose last unit lies in its range: the pieces of every CTA
+//      on the tile, in CTA order and warp order within a CTA (a fixed order,
+//      so results do not depend on timing), waiting only for the flags of
+//      the warps holding those pieces (lanes poll in parallel) and of the
+//      tiles of H; then (s H) B^T on mma.sync (s H as a bf16 hi/lo pair
+//      formed from the tiles of H in L2) and bf16 Y.
 // Nothing waits before it has published what others wait for, so the waits
 // form no cycle.  Flags carry a 64-bit tag unique to the launch (consecutive
 // from a random start), so no word needs clearing between launches.
