@@ -425,13 +425,14 @@ def measure_dq_signed(q, dev, pk, barrier):
     return out
 
 
-FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x fp32 lanes x 2 flops x max SM clock
+TF32_OVER_BF16 = 1.1 / 2.25   # nominal dense tf32 / bf16 tensor throughput of the B200
 
 
 def measure_lq(q, dev, pk, barrier):
     """Low-rank plus quantized decomposition of the 4096 x 4096 q-projection-shaped weight with a
     planted rank-64 part (r = 64, test matrix width 72, 2 power rounds, 2 alternation rounds):
-    time per decomposition and the residual products' fp32 rate against the CUDA-core peak."""
+    time per decomposition, and the residual products (tcgen05 tf32, three products per tile) against
+    HBM (they read W and the packed weight once per launch) and against the tf32 tensor peak."""
     N = K = 4096
     r, l, power, iters = 64, 72, 2, 2
     W = qi.make_lowrank_weight(N, K, r, seed=99).to(dev)
@@ -455,14 +456,25 @@ def measure_lq(q, dev, pk, barrier):
     q.profile_enable(False)
     flops = pn * 2 * N * K * l
     tf = flops / (pms * 1e-3) / 1e12
+    # algorithmic bytes: the first rank-r step (6 launches) reads W alone (4 B per element), the later
+    # ones (12) W and the packed weight (4 + 0.5 + 1/64 + 4/16384 B); every launch reads its l-wide
+    # small operand and writes its l-wide result (4 l (N + K) bytes)
+    n_plain = 6 if pn >= 6 else pn
+    per_elem = n_plain * 4.0 + (pn - n_plain) * (4.0 + 0.5 + 1.0 / 64 + 4.0 / 16384)
+    prod_bytes = per_elem * N * K + pn * 4.0 * l * (N + K)
+    gbs = prod_bytes / (pms * 1e-3) / 1e9
+    tf32_peak = pk["bf16"] * TF32_OVER_BF16
     plain = q.quantize_nf4(W)
     plain_err = float((q.dequantize(plain).double() - W.double()).norm() / W.double().norm())
     e = err.cpu().numpy()
     out = {"ms_per_decomposition": round(ms, 3),
-           "products": {"launches": int(pn), "ms": round(pms, 3), "achieved": round(tf, 2), "unit": "TFLOP/s",
-                        "bound": "alu", "peak": round(FP32_FMA_PEAK_TFLOPS, 1),
-                        "frac": round(tf / FP32_FMA_PEAK_TFLOPS, 4), "share": round(pms / ms, 3),
-                        "flops_per_launch": 2 * N * K * l},
+           "products": {"launches": int(pn), "ms": round(pms, 3), "bound": "hbm", "achieved": round(gbs, 1),
+                        "unit": "GB/s", "peak": pk["hbm"], "frac": round(gbs / pk["hbm"], 4),
+                        "bytes_per_launch_avg": round(prod_bytes / max(pn, 1)),
+                        "tflops": round(tf, 2), "tf32_peak": round(tf32_peak, 1),
+                        "frac_of_tf32_peak": round(tf / tf32_peak, 4),
+                        "tf32_peak_kind": "measured bf16 burst x nominal tf32/bf16 (1.1 / 2.25)",
+                        "share": round(pms / ms, 3), "flops_per_launch": 2 * N * K * l},
            "ms_by_kernel_kind": parts,
            "rel_error": {"plain_nf4": round(plain_err, 5), "after_quantization": [round(x, 5) for x in e[:, 0]],
                          "after_rank_r_step": [round(x, 5) for x in e[:, 1]]},

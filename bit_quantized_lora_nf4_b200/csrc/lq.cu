@@ -210,143 +210,222 @@ __device__ __forceinline__ void raw8_decode(const Raw8 &r, const LqQuant &q, con
   }
 }
 
-// ---- Y = R M: tall-skinny product over K -------------------------------------
-// CTA (bx, split): 32 rows of R x all l (<= 96) columns over the split's range
-// of K, walked in chunks of 64 (one NF4 block per row); writes
-// part[split][n][c].  Thread (tx, ty): rows 4 ty .. 4 ty + 3, columns tx + 32 m.
-// Tile fill: thread t decodes row t / 8, columns 8 (t % 8) .. + 7.
-constexpr int kRmRows = 32, kRmChunk = 64;
+// ---- Y = R M and Z = R^T Y on tensor cores ------------------------------------
+// One CTA: a 128-row tile of the output (rows n of R for Y = R M, columns k of
+// R for Z = R^T Y) over one split of the reduction, walked 32 deep per step.
+// In each step the 8 producer warps load 128 x 32 elements of W with their
+// codes and block constants, form R = fl32(W - W') and split it exactly as
+// R = Rh + Rl (Rh: R with the low 13 mantissa bits cleared, a tf32 value; Rl
+// = R - Rh, exact in fp32), and split the 32 x l tile of the small operand (M
+// or Y) the same way.  One thread issues tcgen05.mma kind::tf32 (M = 128, N =
+// l rounded up to 16, K = 8) for Rh Bh + Rh Bl + Rl Bh into an fp32 TMEM
+// accumulator: the dropped Rl Bl term and the tensor core's truncation of the
+// low parts to tf32 leave about 2^-20 of |R| |B| per product term, the level
+// of an fp32 multiply-add.  Both operands are K-major 128-byte-swizzled tiles
+// in shared memory; the producers write them transposed where the source is
+// not (Z's R^T tile and the small operand, lane = reduction index, so the
+// 4-byte stores of a warp hit 32 banks).  The tile's rows go to
+// part[split][row][c]; lq_sum_splits_kernel adds the splits in order.
+constexpr int kTcRows = 128, kTcRed = 32, kTcStages = 2, kTcProducers = 256;
+constexpr int kTcThreads = 32 + kTcProducers;
+constexpr int kTcATile = kTcRows * kTcRed * 4;          // 16 KB: one component of the R tile
+__host__ __device__ constexpr int lq_tc_stage_bytes(int nl) { return 2 * kTcATile + 2 * nl * kTcRed * 4; }
+__host__ __device__ constexpr int lq_tc_smem(int nl) { return kTcStages * lq_tc_stage_bytes(nl) + 1024 + 128; }
+constexpr uint64_t kTcDrain = 4000000000ull;
 
-__global__ void __launch_bounds__(kLqThreads) lq_rmul_kernel(const float *__restrict__ W, int64_t N, int64_t K,
-                                                             LqQuant q, const float *__restrict__ M, int l,
-                                                             int64_t k_per, float *__restrict__ part) {
-  __shared__ __align__(16) float Rs[kRmRows][kRmChunk + 4];
-  __shared__ float Ms[kRmChunk][kLqMaxL];
-  __shared__ float lv[16];
-  __shared__ float mu_s;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int fr = threadIdx.x >> 3, fc = (threadIdx.x & 7) * 8;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kRmRows;
-  lq_load_levels(q, lv, &mu_s);
-  __syncthreads();
-  const float mu = mu_s;
-  float acc[4][3];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int m = 0; m < 3; ++m) acc[i][m] = 0.0f;
-  const int64_t ka = static_cast<int64_t>(blockIdx.y) * k_per, kb = min(K, ka + k_per);
-  Raw8 raw;
-  raw8_load(W, q, n0 + fr, N, ka + fc, kb, K, raw);
-  for (int64_t k0 = ka; k0 < kb; k0 += kRmChunk) {
-    float rv[8];
-    raw8_decode(raw, q, lv, mu, rv);
-    *reinterpret_cast<float4 *>(&Rs[fr][fc]) = make_float4(rv[0], rv[1], rv[2], rv[3]);
-    *reinterpret_cast<float4 *>(&Rs[fr][fc + 4]) = make_float4(rv[4], rv[5], rv[6], rv[7]);
-    for (int idx = threadIdx.x; idx < kRmChunk * l; idx += kLqThreads) {
-      const int kk = idx / l, c = idx % l;
-      Ms[kk][c] = (k0 + kk < kb) ? __ldg(M + (k0 + kk) * l + c) : 0.0f;
-    }
-    raw8_load(W, q, n0 + fr, N, k0 + kRmChunk + fc, kb, K, raw);   // next chunk, in flight meanwhile
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kRmChunk; kk += 4) {
-      float4 a[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4 *>(&Rs[4 * ty + i][kk]);
-#pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        const int c = tx + 32 * m;
-        if (c < l) {
-          const float b0 = Ms[kk][c], b1 = Ms[kk + 1][c], b2 = Ms[kk + 2][c], b3 = Ms[kk + 3][c];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[i][m] = fmaf(a[i].x, b0, acc[i][m]);
-            acc[i][m] = fmaf(a[i].y, b1, acc[i][m]);
-            acc[i][m] = fmaf(a[i].z, b2, acc[i][m]);
-            acc[i][m] = fmaf(a[i].w, b3, acc[i][m]);
-          }
-        }
-      }
-    }
-    __syncthreads();
-  }
-  float *Y = part + static_cast<int64_t>(blockIdx.y) * N * l;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t n = n0 + 4 * ty + i;
-#pragma unroll
-    for (int m = 0; m < 3; ++m) {
-      const int c = tx + 32 * m;
-      if (n < N && c < l) Y[n * l + c] = acc[i][m];
+// Byte offset of element (row, c), c < 32, in a K-major 128-byte-swizzled tile of 32-bit elements.
+__device__ __forceinline__ uint32_t tc_off(int row, int c) {
+  return static_cast<uint32_t>(row * 128 + ((((c >> 2) ^ row) & 7) << 4) + (c & 3) * 4);
+}
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+__device__ __forceinline__ bool lq_wait(uint64_t *bar, uint32_t parity, uint64_t limit, volatile int *abort_flag,
+                                        int *status) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (static_cast<uint64_t>(clock64() - t0) > limit) {
+      *abort_flag = 1;
+      latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
+      return false;
     }
   }
 }
 
-// ---- Z = R^T Y: tall-skinny product over N, split over row ranges ------------
-// CTA (bx, split): columns 64 bx .. 64 bx + 63 of R x all l columns of Y, rows
-// [rows_per * split, ...) walked 32 at a time.  Thread (tx, ty): R columns
-// 8 ty .. 8 ty + 7, Y columns tx + 32 m.  Writes part[split][k][c].
-constexpr int kRtCols = 64, kRtRows = 32;
-
-__global__ void __launch_bounds__(kLqThreads) lq_rtmul_kernel(const float *__restrict__ W, int64_t N, int64_t K,
-                                                              LqQuant q, const float *__restrict__ Y, int l,
-                                                              int64_t rows_per, float *__restrict__ part) {
-  __shared__ __align__(16) float Rs[kRtRows][kRtCols + 4];
-  __shared__ float Ys[kRtRows][kLqMaxL];
+template <bool TRANS>
+__global__ void __launch_bounds__(kTcThreads, 2)   // two CTAs per SM (the split plan counts on it)
+    lq_tc_kernel(const float *__restrict__ W, int64_t N, int64_t K, LqQuant q, const float *__restrict__ Bsrc,
+                 int l, int nl, int64_t red_per, float *__restrict__ part, int *status, uint64_t wait_limit) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int stage_bytes = lq_tc_stage_bytes(nl);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcStages * stage_bytes);
+  uint64_t *full = bars, *empty = bars + kTcStages, *acc_full = bars + 2 * kTcStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kTcStages + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   __shared__ float lv[16];
   __shared__ float mu_s;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int fr = threadIdx.x >> 3, fc = (threadIdx.x & 7) * 8;
-  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kRtCols;
-  const int64_t na = static_cast<int64_t>(blockIdx.y) * rows_per, nb = min(N, na + rows_per);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rows_total = TRANS ? K : N;   // output rows
+  const int64_t o0 = static_cast<int64_t>(blockIdx.x) * kTcRows;
+  const int64_t ra = static_cast<int64_t>(blockIdx.y) * red_per;
+  const int64_t rb = min(TRANS ? N : K, ra + red_per);
+  const int nsteps = rb > ra ? static_cast<int>((rb - ra + kTcRed - 1) / kTcRed) : 0;
   lq_load_levels(q, lv, &mu_s);
-  __syncthreads();
-  const float mu = mu_s;
-  float acc[8][3];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int m = 0; m < 3; ++m) acc[i][m] = 0.0f;
-  Raw8 raw;
-  raw8_load(W, q, na + fr, nb, k0 + fc, K, K, raw);
-  for (int64_t n0 = na; n0 < nb; n0 += kRtRows) {
-    float rv[8];
-    raw8_decode(raw, q, lv, mu, rv);
-    *reinterpret_cast<float4 *>(&Rs[fr][fc]) = make_float4(rv[0], rv[1], rv[2], rv[3]);
-    *reinterpret_cast<float4 *>(&Rs[fr][fc + 4]) = make_float4(rv[4], rv[5], rv[6], rv[7]);
-    for (int idx = threadIdx.x; idx < kRtRows * l; idx += kLqThreads) {
-      const int rr = idx / l, c = idx % l;
-      Ys[rr][c] = (n0 + rr < nb) ? __ldg(Y + (n0 + rr) * l + c) : 0.0f;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], kTcProducers);
+      mbar_init(&empty[s], 1);
     }
-    raw8_load(W, q, n0 + kRtRows + fr, nb, k0 + fc, K, K, raw);   // next rows, in flight meanwhile
-    __syncthreads();
-#pragma unroll 2
-    for (int rr = 0; rr < kRtRows; ++rr) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&Rs[rr][8 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&Rs[rr][8 * ty + 4]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // rows l .. nl - 1 of the small operand's tiles stay zero (never written below)
+  for (int idx = threadIdx.x; idx < kTcStages * 2 * (nl - l) * kTcRed; idx += blockDim.x) {
+    const int per = (nl - l) * kTcRed;
+    const int sc = idx / per, e = idx - sc * per;
+    const int j = l + e / kTcRed, c = e % kTcRed;
+    *reinterpret_cast<float *>(smem + (sc >> 1) * stage_bytes + 2 * kTcATile + (sc & 1) * nl * kTcRed * 4 +
+                               tc_off(j, c)) = 0.0f;
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float mu = mu_s;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_tf32_f32(kTcRows, nl);
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % kTcStages;
+        if (!lq_wait(&full[s], (i / kTcStages) & 1, wait_limit, abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t ah = smem_addr(smem + s * stage_bytes), al = ah + kTcATile;
+        const uint32_t bh = ah + 2 * kTcATile, bl = bh + nl * kTcRed * 4;
+        for (int kk = 0; kk < kTcRed / 8; ++kk) {   // K = 8 tf32 = 32 bytes per MMA
+          const uint64_t dah = sdesc_sw128(ah + kk * 32, 16, 1024), dal = sdesc_sw128(al + kk * 32, 16, 1024);
+          const uint64_t dbh = sdesc_sw128(bh + kk * 32, 16, 1024), dbl = sdesc_sw128(bl + kk * 32, 16, 1024);
+          tc_mma_tf32(tmem, dah, dbh, idesc, (i | kk) != 0 ? 1u : 0u);
+          tc_mma_tf32(tmem, dah, dbl, idesc, 1u);
+          tc_mma_tf32(tmem, dal, dbh, idesc, 1u);
+        }
+        tc_commit(&empty[s]);
+      }
+      tc_commit(acc_full);
+    }
+  } else {
+    const int pt = threadIdx.x - 32, pw = pt >> 5;
+    const int nb = (kTcRed * l + kTcProducers - 1) / kTcProducers;   // small-operand elements per thread (<= 12)
+    for (int i = 0; i < nsteps; ++i) {
+      const int s = i % kTcStages;
+      const int64_t r0 = ra + static_cast<int64_t>(i) * kTcRed;
+      // this step's loads first: they overlap the wait for the slot
+      Raw8 raw[2];
 #pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        const int c = tx + 32 * m;
-        if (c < l) {
-          const float b = Ys[rr][c];
+      for (int u = 0; u < 2; ++u) {
+        if (!TRANS) {
+          const int id = pt + kTcProducers * u, row = id >> 2, rr = id & 3;   // 8 rows x 4 runs per warp
+          raw8_load(W, q, o0 + row, N, r0 + 8 * rr, rb, K, raw[u]);
+        } else {
+          const int g = pw + 8 * u;                                             // lane = row n of R
+          raw8_load(W, q, r0 + lane, rb, o0 + 8 * g, K, K, raw[u]);
+        }
+      }
+      float bv[(kTcRed * kLqMaxL + kTcProducers - 1) / kTcProducers];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i][m] = fmaf(a[i], b, acc[i][m]);
+      for (int v = 0; v < (kTcRed * kLqMaxL + kTcProducers - 1) / kTcProducers; ++v) {
+        const int e = pt + kTcProducers * v;
+        bv[v] = 0.0f;
+        if (v < nb && e < kTcRed * l) {
+          const int rl = e / l, j = e - rl * l;
+          if (r0 + rl < rb) bv[v] = __ldg(Bsrc + (r0 + rl) * l + j);
+        }
+      }
+      if (i >= kTcStages && !lq_wait(&empty[s], ((i / kTcStages) & 1) ^ 1, wait_limit, abort_flag, status)) break;
+      uint8_t *ah = smem + s * stage_bytes, *al = ah + kTcATile;
+      uint8_t *bh = ah + 2 * kTcATile, *bl = bh + nl * kTcRed * 4;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float rv[8];
+        raw8_decode(raw[u], q, lv, mu, rv);
+        float hv[8], lo[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          hv[t] = tf32_hi(rv[t]);
+          lo[t] = __fsub_rn(rv[t], hv[t]);
+        }
+        if (!TRANS) {
+          const int id = pt + kTcProducers * u, row = id >> 2, c = 8 * (id & 3);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t off = tc_off(row, c + 4 * h);
+            *reinterpret_cast<float4 *>(ah + off) = make_float4(hv[4 * h], hv[4 * h + 1], hv[4 * h + 2], hv[4 * h + 3]);
+            *reinterpret_cast<float4 *>(al + off) = make_float4(lo[4 * h], lo[4 * h + 1], lo[4 * h + 2], lo[4 * h + 3]);
+          }
+        } else {
+          const int g = pw + 8 * u;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const uint32_t off = tc_off(8 * g + t, lane);
+            *reinterpret_cast<float *>(ah + off) = hv[t];
+            *reinterpret_cast<float *>(al + off) = lo[t];
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < (kTcRed * kLqMaxL + kTcProducers - 1) / kTcProducers; ++v) {
+        const int e = pt + kTcProducers * v;
+        if (v < nb && e < kTcRed * l) {
+          const int rl = e / l, j = e - rl * l;
+          const float h = tf32_hi(bv[v]);
+          const uint32_t off = tc_off(j, rl);
+          *reinterpret_cast<float *>(bh + off) = h;
+          *reinterpret_cast<float *>(bl + off) = __fsub_rn(bv[v], h);
+        }
+      }
+      fence_proxy_async_smem();   // generic-proxy writes visible to the tensor core
+      mbar_arrive(&full[s]);
+    }
+    // epilogue: warps 1..4 hold TMEM lanes 32 (warp % 4) .. + 31 = output rows of the tile
+    if (warp <= 4) {
+      const bool ok = mbar_wait(acc_full, 0, kTcDrain);
+      tc_fence_after();
+      const bool live = __all_sync(0xffffffffu, ok && *abort_flag == 0 && nsteps > 0);
+      const int quarter = warp & 3;
+      const int64_t orow = o0 + quarter * 32 + lane;
+      float *out = part + static_cast<int64_t>(blockIdx.y) * rows_total * l + orow * l;
+      if (!ok) latch_status(status, QLORA_ERR_DEVICE_TIMEOUT);
+      for (int c0 = 0; c0 < nl; c0 += 16) {
+        uint32_t v[16];
+        if (live) {
+          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c0, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = 0u;   // empty or aborted split: zero
+        }
+        if (orow < rows_total) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (c0 + e < l) out[c0 + e] = __uint_as_float(v[e]);
         }
       }
     }
-    __syncthreads();
   }
-  float *out = part + static_cast<int64_t>(blockIdx.y) * K * l;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t k = k0 + 8 * ty + i;
-#pragma unroll
-    for (int m = 0; m < 3; ++m) {
-      const int c = tx + 32 * m;
-      if (k < K && c < l) out[k * l + c] = acc[i][m];
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -691,14 +770,14 @@ LqPlan lq_plan(int64_t N, int64_t K, int r, int l, int dq) {
   p.K = K;
   p.r = r;
   p.l = l;
-  // both products aim at about four CTAs per SM
-  const int64_t col_tiles = ceil_div(K, kRtCols);
-  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(ceil_div(4 * 148, col_tiles), ceil_div(N, kRtRows)));
-  p.rt_rows = ceil_div(ceil_div(N, splits), kRtRows) * kRtRows;
+  // both products: about two CTAs per SM, splits of the reduction at least four steps deep
+  const int64_t col_tiles = ceil_div(K, kTcRows);
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(2 * 148 / col_tiles, ceil_div(N, 4 * kTcRed)));
+  p.rt_rows = ceil_div(ceil_div(N, splits), kTcRed) * kTcRed;
   p.rt_splits = ceil_div(N, p.rt_rows);
-  const int64_t row_tiles = ceil_div(N, kRmRows);
-  splits = std::max<int64_t>(1, std::min<int64_t>(ceil_div(4 * 148, row_tiles), ceil_div(K, kRmChunk)));
-  p.rm_cols = ceil_div(ceil_div(K, splits), kRmChunk) * kRmChunk;
+  const int64_t row_tiles = ceil_div(N, kTcRows);
+  splits = std::max<int64_t>(1, std::min<int64_t>(2 * 148 / row_tiles, ceil_div(K, 4 * kTcRed)));
+  p.rm_cols = ceil_div(ceil_div(K, splits), kTcRed) * kTcRed;
   p.rm_splits = ceil_div(K, p.rm_cols);
   p.res_ctas = ceil_div(K, kResCols) * ceil_div(N, kResRows);
   p.gram_parts_max = kGramMaxParts;
@@ -755,13 +834,25 @@ struct LqRun {
     lq_sum_kernel<<<1, kLqThreads, 0, st>>>(part, n, norm2, out);
     check();
   }
-  void rmul(const LqQuant &q, const float *M, float *Y) {
-    const dim3 grid(static_cast<unsigned>(ceil_div(p.N, kRmRows)), static_cast<unsigned>(p.rm_splits));
-    float *part = wsp<float>(ws, p.Zpart);
+  // one tensor-core product launch: out-rows tiles x splits CTAs
+  template <bool TRANS>
+  void tc_product(const LqQuant &q, const float *B, int64_t red_per, int64_t splits, float *part) {
+    const int nl = static_cast<int>(ceil_div(p.l, 16) * 16);
+    const int smem = lq_tc_smem(nl);
+    if (err == cudaSuccess) err = cudaFuncSetAttribute(lq_tc_kernel<TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int *status = device_status_ptr();
+    if (err == cudaSuccess && !status) err = cudaErrorInvalidValue;
+    if (err != cudaSuccess) return;
+    const dim3 grid(static_cast<unsigned>(ceil_div(TRANS ? p.K : p.N, kTcRows)), static_cast<unsigned>(splits));
     prof_mark(kProfLqProduct, true, st);
-    lq_rmul_kernel<<<grid, kLqThreads, 0, st>>>(W, p.N, p.K, q, M, p.l, p.rm_cols, part);
+    lq_tc_kernel<TRANS><<<grid, kTcThreads, smem, st>>>(W, p.N, p.K, q, B, p.l, nl, red_per, part, status,
+                                                         wait_limit());
     prof_mark(kProfLqProduct, false, st);
     check();
+  }
+  void rmul(const LqQuant &q, const float *M, float *Y) {
+    float *part = wsp<float>(ws, p.Zpart);
+    tc_product<false>(q, M, p.rm_cols, p.rm_splits, part);
     sum_splits(part, static_cast<int>(p.rm_splits), p.N * p.l, Y);
   }
   void sum_splits(const float *part, int ns, int64_t n, float *out) {
@@ -772,12 +863,8 @@ struct LqRun {
     check();
   }
   void rtmul(const LqQuant &q, const float *Y, float *Z) {
-    const dim3 grid(static_cast<unsigned>(ceil_div(p.K, kRtCols)), static_cast<unsigned>(p.rt_splits));
     float *part = wsp<float>(ws, p.Zpart);
-    prof_mark(kProfLqProduct, true, st);
-    lq_rtmul_kernel<<<grid, kLqThreads, 0, st>>>(W, p.N, p.K, q, Y, p.l, p.rt_rows, part);
-    prof_mark(kProfLqProduct, false, st);
-    check();
+    tc_product<true>(q, Y, p.rt_rows, p.rt_splits, part);
     sum_splits(part, static_cast<int>(p.rt_splits), p.K * p.l, Z);
   }
   // G = X^T X (fp64, l x l) of X [rows, l]
