@@ -162,75 +162,54 @@ __global__ void lq_sum_kernel(const double *__restrict__ part, int64_t n, const 
   if (threadIdx.x == 0) *out = norm2 ? (*norm2 > 0.0 ? sqrt(tot / *norm2) : 0.0) : tot;
 }
 
-// ---- residual tiles: 8 consecutive elements of one row per thread -------------
-// K % 64 == 0, so a run of 8 never leaves its 64-element block and its codes
-// are one aligned 32-bit word.  The raw loads are issued one chunk ahead and
-// decoded after the current chunk's arithmetic.
-struct Raw8 {
-  float4 w0, w1;
-  uint32_t codes, q;
-  float S;
-  bool valid;   // false past the matrix or the CTA's range: the run decodes to 0
-};
-
-__device__ __forceinline__ void raw8_load(const float *W, const LqQuant &q, int64_t n, int64_t N, int64_t k,
-                                          int64_t kend, int64_t K, Raw8 &r) {
-  r.valid = n < N && k < kend;
-  if (r.valid) {
-    const int64_t e = n * K + k;
-    r.w0 = __ldg(reinterpret_cast<const float4 *>(W + e));
-    r.w1 = __ldg(reinterpret_cast<const float4 *>(W + e) + 1);
-    if (q.codes) {
-      r.codes = __ldg(reinterpret_cast<const uint32_t *>(q.codes + (e >> 1)));
-      r.q = __ldg(q.absmax_q + (e >> 6));
-      r.S = __ldg(q.group_scale + (e >> 14));
-    }
-  } else {
-    r.w0 = r.w1 = make_float4(0.f, 0.f, 0.f, 0.f);
-    r.codes = 0;
-    r.q = 0;
-    r.S = 0.0f;
-  }
-}
-
-// R = fl32(W - W') for the 8 elements (0 for an invalid run).
-__device__ __forceinline__ void raw8_decode(const Raw8 &r, const LqQuant &q, const float *lv, float mu,
-                                            float (&out)[8]) {
-  const float w[8] = {r.w0.x, r.w0.y, r.w0.z, r.w0.w, r.w1.x, r.w1.y, r.w1.z, r.w1.w};
-  if (!q.codes || !r.valid) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) out[i] = w[i];   // W itself; zeros for an invalid run
-    return;
-  }
-  const float ap = block_constant(r.q, r.S, q.tab.qx, mu);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(r.codes >> (4 * i)) & 15u], ap)));
-    out[i] = __fsub_rn(w[i], wq);
-  }
-}
-
 // ---- Y = R M and Z = R^T Y on tensor cores ------------------------------------
-// One CTA: a 128-row tile of the output (rows n of R for Y = R M, columns k of
-// R for Z = R^T Y) over one split of the reduction, walked 32 deep per step.
-// In each step the 8 producer warps load 128 x 32 elements of W with their
-// codes and block constants, form R = fl32(W - W') and split it exactly as
-// R = Rh + Rl (Rh: R with the low 13 mantissa bits cleared, a tf32 value; Rl
-// = R - Rh, exact in fp32), and split the 32 x l tile of the small operand (M
-// or Y) the same way.  One thread issues tcgen05.mma kind::tf32 (M = 128, N =
-// l rounded up to 16, K = 8) for Rh Bh + Rh Bl + Rl Bh into an fp32 TMEM
-// accumulator: the dropped Rl Bl term and the tensor core's truncation of the
-// low parts to tf32 leave about 2^-20 of |R| |B| per product term, the level
-// of an fp32 multiply-add.  Both operands are K-major 128-byte-swizzled tiles
-// in shared memory; the producers write them transposed where the source is
-// not (Z's R^T tile and the small operand, lane = reduction index, so the
-// 4-byte stores of a warp hit 32 banks).  The tile's rows go to
-// part[split][row][c]; lq_sum_splits_kernel adds the splits in order.
-constexpr int kTcRows = 128, kTcRed = 32, kTcStages = 2, kTcProducers = 256;
-constexpr int kTcThreads = 32 + kTcProducers;
-constexpr int kTcATile = kTcRows * kTcRed * 4;          // 16 KB: one component of the R tile
-__host__ __device__ constexpr int lq_tc_stage_bytes(int nl) { return 2 * kTcATile + 2 * nl * kTcRed * 4; }
-__host__ __device__ constexpr int lq_tc_smem(int nl) { return kTcStages * lq_tc_stage_bytes(nl) + 1024 + 128; }
+// One CTA per SM: a 128-row tile of the output (rows n of R for Y = R M,
+// columns k of R for Z = R^T Y) over one split of the reduction, walked 32
+// deep per step.
+//   warp 1   loader: lane 0 brings the step's 128 x 32 tile of W (128B-
+//            swizzled), its codes and the small operand's two 32-deep tiles
+//            (below) by TMA into a 3- or 4-stage ring (as shared memory
+//            allows); all lanes fetch the block
+//            constants (8-bit code, group scale) three steps ahead into
+//            registers and store them beside the tile (their row stride,
+//            K / 64 bytes, is not TMA-able in general).
+//   warps 2-17 form R = fl32(W - W') from the ring (one run of 8 elements per
+//            thread and step) and split it exactly as
+//            R = Rh + Rl (Rh: R with the low 13 mantissa bits cleared, a tf32
+//            value; Rl = R - Rh, exact in fp32), and write it K-major and
+//            128-byte-swizzled into a 2-stage operand ring (transposed for Z's
+//            R^T tile, lane = reduction index, so a warp's 4-byte stores hit
+//            32 banks).  Elements outside the matrix or the split are zero (a
+//            zero-filled code would decode as a level).
+// The small operand (M or Y, [reduction, l]) is split the same way once per
+// product by lq_tc_split_kernel into the layout the MMA reads: per 32-deep
+// block, an hi and a lo tile of nl rows (l rounded up to 16; the extra rows
+// zero) x 32 fp32, which the loader's TMA swizzles as it lands.
+//   warp 0   one thread issues tcgen05.mma kind::tf32 (M = 128, N = l rounded
+//            up to 16, K = 8) for Rh Bh + Rh Bl + Rl Bh into an fp32 TMEM
+//            accumulator: the dropped Rl Bl term and the tensor core's
+//            truncation of the low parts to tf32 leave about 2^-20 of |R| |B|
+//            per product term, the level of an fp32 multiply-add.
+// Warps 2-5 then write the tile's rows to part[split][row][c], and
+// lq_sum_splits_kernel adds the splits in order.
+constexpr int kTcRows = 128, kTcRed = 32, kTcMaxRawStages = 4, kTcOpStages = 2, kTcProducers = 512;
+constexpr int kTcThreads = 64 + kTcProducers;
+constexpr int kTcATile = kTcRows * kTcRed * 4;          // 16 KB: one component of the R tile (and W's raw tile)
+// raw stage: W tile (16 KB), codes (2 KB), the small operand's hi and lo tiles (nl x 128 B each, 1024-
+// aligned for the swizzle), 8-bit constants, group scales
+constexpr int kTcRawCodes = kTcATile, kTcRawB = kTcRawCodes + 2048;
+__host__ __device__ constexpr int lq_tc_raw_q(int nl) { return kTcRawB + 2 * nl * kTcRed * 4; }
+__host__ __device__ constexpr int lq_tc_raw_s(int nl) { return lq_tc_raw_q(nl) + 128; }
+__host__ __device__ constexpr int lq_tc_raw_bytes(int nl) { return (lq_tc_raw_s(nl) + 128 * 4 + 1023) / 1024 * 1024; }
+// raw stages that fit beside the operand ring in 227 KB
+__host__ __device__ constexpr int lq_tc_raw_stages(int nl) {
+  return (232448 - kTcOpStages * 2 * kTcATile - 1024 - 160) / lq_tc_raw_bytes(nl) >= kTcMaxRawStages
+             ? kTcMaxRawStages
+             : 3;
+}
+__host__ __device__ constexpr int lq_tc_smem(int nl) {
+  return lq_tc_raw_stages(nl) * lq_tc_raw_bytes(nl) + kTcOpStages * 2 * kTcATile + 1024 + 160;
+}
 constexpr uint64_t kTcDrain = 4000000000ull;
 
 // Byte offset of element (row, c), c < 32, in a K-major 128-byte-swizzled tile of 32-bit elements.
@@ -255,16 +234,79 @@ __device__ __forceinline__ bool lq_wait(uint64_t *bar, uint32_t parity, uint64_t
   }
 }
 
+// The small operand [red, l] split for the products: Bt[(b * 2 + h) * nl + j][c]
+// = component h (0: tf32-exact high part, 1: remainder) of B[32 b + c][j], zero
+// for j >= l or 32 b + c >= red.  One thread per four consecutive c (16-byte
+// stores of both components); the reads hit L2 (B is a few MB at most).
+__global__ void __launch_bounds__(256) lq_tc_split_kernel(const float *__restrict__ B, int64_t red, int l, int nl,
+                                                          int nblk, float *__restrict__ Bt) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= nblk * nl * (kTcRed / 4)) return;
+  const int c4 = e & 7, bj = e >> 3;
+  const int b = bj / nl, j = bj - b * nl;
+  float x[4], hv[4], lo[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int64_t r = static_cast<int64_t>(b) * kTcRed + 4 * c4 + t;
+    x[t] = (j < l && r < red) ? __ldg(B + r * l + j) : 0.0f;
+    hv[t] = tf32_hi(x[t]);
+    lo[t] = __fsub_rn(x[t], hv[t]);
+  }
+  float *hi_row = Bt + (static_cast<int64_t>(b * 2) * nl + j) * kTcRed + 4 * c4;
+  *reinterpret_cast<float4 *>(hi_row) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+  *reinterpret_cast<float4 *>(hi_row + static_cast<int64_t>(nl) * kTcRed) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+}
+
+// The block constants a loader lane fetches for one step: rows lane + 32 j
+// (Y = R M, one 64-block per row) or row lane, blocks 0 and 1 (Z = R^T Y).
+struct TcConst {
+  uint32_t q[4];
+  float S[4];
+};
+
 template <bool TRANS>
-__global__ void __launch_bounds__(kTcThreads, 2)   // two CTAs per SM (the split plan counts on it)
-    lq_tc_kernel(const float *__restrict__ W, int64_t N, int64_t K, LqQuant q, const float *__restrict__ Bsrc,
-                 int l, int nl, int64_t red_per, float *__restrict__ part, int *status, uint64_t wait_limit) {
+__device__ __forceinline__ TcConst tc_const_load(const LqQuant &q, int64_t N, int64_t K, int64_t o0, int64_t r0,
+                                                 int64_t rb, int lane) {
+  TcConst c{};
+  if (!q.codes) return c;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    int64_t n, k;
+    bool ok;
+    if (!TRANS) {
+      n = o0 + lane + 32 * j;
+      k = r0;
+      ok = n < N && r0 < rb;
+    } else {
+      n = r0 + lane;
+      k = o0 + 64 * j;
+      ok = j < 2 && n < rb && k < K;
+    }
+    if (ok) {
+      const int64_t blk = (n * K + k) >> 6;
+      c.q[j] = __ldg(q.absmax_q + blk);
+      c.S[j] = __ldg(q.group_scale + (blk >> 8));
+    }
+  }
+  return c;
+}
+
+template <bool TRANS>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    lq_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmC,
+                 const __grid_constant__ CUtensorMap tmB, int64_t N, int64_t K, LqQuant q, int l, int nl,
+                 int64_t red_per, float *__restrict__ part, int *status, uint64_t wait_limit) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int stage_bytes = lq_tc_stage_bytes(nl);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcStages * stage_bytes);
-  uint64_t *full = bars, *empty = bars + kTcStages, *acc_full = bars + 2 * kTcStages;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kTcStages + 1);
+  const int op_bytes = 2 * kTcATile;
+  const int raw_bytes = lq_tc_raw_bytes(nl), raw_q = lq_tc_raw_q(nl), raw_s = lq_tc_raw_s(nl);
+  const int RS = lq_tc_raw_stages(nl);
+  uint8_t *raw_ring = smem;
+  uint8_t *op_ring = smem + RS * raw_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(op_ring + kTcOpStages * op_bytes);
+  uint64_t *raw_full = bars, *raw_empty = bars + kTcMaxRawStages;
+  uint64_t *op_full = bars + 2 * kTcMaxRawStages, *op_empty = op_full + kTcOpStages, *acc_full = op_empty + kTcOpStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   __shared__ float lv[16];
   __shared__ float mu_s;
@@ -274,23 +316,23 @@ __global__ void __launch_bounds__(kTcThreads, 2)   // two CTAs per SM (the split
   const int64_t ra = static_cast<int64_t>(blockIdx.y) * red_per;
   const int64_t rb = min(TRANS ? N : K, ra + red_per);
   const int nsteps = rb > ra ? static_cast<int>((rb - ra + kTcRed - 1) / kTcRed) : 0;
+  const bool quant = q.codes != nullptr;
   lq_load_levels(q, lv, &mu_s);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], kTcProducers);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&raw_full[s], 1 + 32);           // the TMA lane's expect-tx arrival + every loader lane's constants
+      mbar_init(&raw_empty[s], kTcProducers + 1);   // + the MMAs' commit (they read the small tiles there)
+    }
+    for (int s = 0; s < kTcOpStages; ++s) {
+      mbar_init(&op_full[s], kTcProducers);
+      mbar_init(&op_empty[s], 1);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  // rows l .. nl - 1 of the small operand's tiles stay zero (never written below)
-  for (int idx = threadIdx.x; idx < kTcStages * 2 * (nl - l) * kTcRed; idx += blockDim.x) {
-    const int per = (nl - l) * kTcRed;
-    const int sc = idx / per, e = idx - sc * per;
-    const int j = l + e / kTcRed, c = e % kTcRed;
-    *reinterpret_cast<float *>(smem + (sc >> 1) * stage_bytes + 2 * kTcATile + (sc & 1) * nl * kTcRed * 4 +
-                               tc_off(j, c)) = 0.0f;
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmB);
+    if (quant) tma_prefetch_desc(&tmC);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 128);
@@ -303,14 +345,17 @@ __global__ void __launch_bounds__(kTcThreads, 2)   // two CTAs per SM (the split
   const float mu = mu_s;
 
   if (warp == 0) {
+    // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_tf32_f32(kTcRows, nl);
       for (int i = 0; i < nsteps; ++i) {
-        const int s = i % kTcStages;
-        if (!lq_wait(&full[s], (i / kTcStages) & 1, wait_limit, abort_flag, status)) break;
+        const int s = i % kTcOpStages, sr = i % RS;
+        if (!lq_wait(&op_full[s], (i / kTcOpStages) & 1, wait_limit, abort_flag, status) ||
+            !lq_wait(&raw_full[sr], (i / RS) & 1, wait_limit, abort_flag, status))
+          break;
         tc_fence_after();
-        const uint32_t ah = smem_addr(smem + s * stage_bytes), al = ah + kTcATile;
-        const uint32_t bh = ah + 2 * kTcATile, bl = bh + nl * kTcRed * 4;
+        const uint32_t ah = smem_addr(op_ring + s * op_bytes), al = ah + kTcATile;
+        const uint32_t bh = smem_addr(raw_ring + sr * raw_bytes + kTcRawB), bl = bh + nl * kTcRed * 4;
         for (int kk = 0; kk < kTcRed / 8; ++kk) {   // K = 8 tf32 = 32 bytes per MMA
           const uint64_t dah = sdesc_sw128(ah + kk * 32, 16, 1024), dal = sdesc_sw128(al + kk * 32, 16, 1024);
           const uint64_t dbh = sdesc_sw128(bh + kk * 32, 16, 1024), dbl = sdesc_sw128(bl + kk * 32, 16, 1024);
@@ -318,45 +363,108 @@ __global__ void __launch_bounds__(kTcThreads, 2)   // two CTAs per SM (the split
           tc_mma_tf32(tmem, dah, dbl, idesc, 1u);
           tc_mma_tf32(tmem, dal, dbh, idesc, 1u);
         }
-        tc_commit(&empty[s]);
+        tc_commit(&op_empty[s]);
+        tc_commit(&raw_empty[sr]);
       }
       tc_commit(acc_full);
     }
-  } else {
-    const int pt = threadIdx.x - 32, pw = pt >> 5;
-    const int nb = (kTcRed * l + kTcProducers - 1) / kTcProducers;   // small-operand elements per thread (<= 12)
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- loader
+    const uint32_t bytes = static_cast<uint32_t>(kTcATile + (quant ? 2048 : 0) + 2 * nl * kTcRed * 4);
+    TcConst c0 = tc_const_load<TRANS>(q, N, K, o0, ra, rb, lane);
+    TcConst c1 = tc_const_load<TRANS>(q, N, K, o0, ra + kTcRed, rb, lane);
+    TcConst c2 = tc_const_load<TRANS>(q, N, K, o0, ra + 2 * kTcRed, rb, lane);
     for (int i = 0; i < nsteps; ++i) {
-      const int s = i % kTcStages;
+      const int s = i % RS;
       const int64_t r0 = ra + static_cast<int64_t>(i) * kTcRed;
-      // this step's loads first: they overlap the wait for the slot
-      Raw8 raw[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      if (i >= RS && !lq_wait(&raw_empty[s], ((i / RS) & 1) ^ 1, wait_limit, abort_flag, status))
+        break;
+      uint8_t *st = raw_ring + s * raw_bytes;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&raw_full[s], bytes);
         if (!TRANS) {
-          const int id = pt + kTcProducers * u, row = id >> 2, rr = id & 3;   // 8 rows x 4 runs per warp
-          raw8_load(W, q, o0 + row, N, r0 + 8 * rr, rb, K, raw[u]);
+          tma_load_2d(st, &tmW, &raw_full[s], static_cast<int>(r0), static_cast<int>(o0));
+          if (quant) tma_load_2d(st + kTcRawCodes, &tmC, &raw_full[s], static_cast<int>(r0 / 2), static_cast<int>(o0));
         } else {
-          const int g = pw + 8 * u;                                             // lane = row n of R
-          raw8_load(W, q, r0 + lane, rb, o0 + 8 * g, K, K, raw[u]);
+          for (int b = 0; b < 4; ++b)
+            tma_load_2d(st + 4096 * b, &tmW, &raw_full[s], static_cast<int>(o0) + 32 * b, static_cast<int>(r0));
+          if (quant) tma_load_2d(st + kTcRawCodes, &tmC, &raw_full[s], static_cast<int>(o0 / 2), static_cast<int>(r0));
+        }
+        const int blk = static_cast<int>(r0 / kTcRed);   // the small operand's hi and lo tiles of this block
+        tma_load_2d(st + kTcRawB, &tmB, &raw_full[s], 0, 2 * blk * nl);
+        tma_load_2d(st + kTcRawB + nl * kTcRed * 4, &tmB, &raw_full[s], 0, (2 * blk + 1) * nl);
+      }
+      uint8_t *qs = st + raw_q;
+      float *ss = reinterpret_cast<float *>(st + raw_s);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int idx = TRANS ? lane * 2 + j : lane + 32 * j;
+        if (!TRANS || j < 4) {
+          if (TRANS && j >= 2) continue;
+          qs[idx] = static_cast<uint8_t>(c0.q[j]);
+          ss[idx] = c0.S[j];
         }
       }
-      float bv[(kTcRed * kLqMaxL + kTcProducers - 1) / kTcProducers];
-#pragma unroll
-      for (int v = 0; v < (kTcRed * kLqMaxL + kTcProducers - 1) / kTcProducers; ++v) {
-        const int e = pt + kTcProducers * v;
-        bv[v] = 0.0f;
-        if (v < nb && e < kTcRed * l) {
-          const int rl = e / l, j = e - rl * l;
-          if (r0 + rl < rb) bv[v] = __ldg(Bsrc + (r0 + rl) * l + j);
+      mbar_arrive(&raw_full[s]);
+      c0 = c1;
+      c1 = c2;
+      c2 = tc_const_load<TRANS>(q, N, K, o0, r0 + 3 * kTcRed, rb, lane);
+    }
+  } else {
+    // ---------------------------------------------------------------- producers
+    const int pt = threadIdx.x - 64, pw = pt >> 5;
+    for (int i = 0; i < nsteps; ++i) {
+      const int sr = i % RS, so = i % kTcOpStages;
+      const int64_t r0 = ra + static_cast<int64_t>(i) * kTcRed;
+      if (!lq_wait(&raw_full[sr], (i / RS) & 1, wait_limit, abort_flag, status)) break;
+      if (i >= kTcOpStages && !lq_wait(&op_empty[so], ((i / kTcOpStages) & 1) ^ 1, wait_limit, abort_flag, status))
+        break;
+      const uint8_t *st = raw_ring + sr * raw_bytes;
+      const uint8_t *qs = st + raw_q;
+      const float *ss = reinterpret_cast<const float *>(st + raw_s);
+      uint8_t *ah = op_ring + so * op_bytes, *al = ah + kTcATile;
+      {
+        // this thread's run of 8 elements: (tile row, reduction offset) for Y = R M,
+        // (reduction row = lane, tile column 8 g) for Z = R^T Y
+        int row, col, ci;
+        uint32_t w_off, c_off;
+        bool ok;
+        if (!TRANS) {
+          row = pt >> 2;                         // 8 rows x 4 runs per warp
+          col = 8 * (pt & 3);
+          w_off = static_cast<uint32_t>(row * 128);
+          c_off = static_cast<uint32_t>(row * 16 + (pt & 3) * 4);
+          ci = row;
+          ok = o0 + row < N && r0 + col < rb;
+        } else {
+          const int g = pw;                      // 16 groups of 8 tile columns, lane = reduction row
+          row = lane;
+          col = 8 * g;
+          w_off = static_cast<uint32_t>(4096 * (g >> 2) + lane * 128);
+          c_off = static_cast<uint32_t>(lane * 64 + g * 4);
+          ci = lane * 2 + (g >> 3);
+          ok = r0 + lane < rb && o0 + col < K;
         }
-      }
-      if (i >= kTcStages && !lq_wait(&empty[s], ((i / kTcStages) & 1) ^ 1, wait_limit, abort_flag, status)) break;
-      uint8_t *ah = smem + s * stage_bytes, *al = ah + kTcATile;
-      uint8_t *bh = ah + 2 * kTcATile, *bl = bh + nl * kTcRed * 4;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
+        const int cc = TRANS ? 8 * ((col >> 3) & 3) : col;   // column within the 32-wide swizzled raw tile
+        const float4 wa = *reinterpret_cast<const float4 *>(st + w_off + ((((cc >> 2) ^ row) & 7) << 4));
+        const float4 wb = *reinterpret_cast<const float4 *>(st + w_off + (((((cc >> 2) + 1) ^ row) & 7) << 4));
+        const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
         float rv[8];
-        raw8_decode(raw[u], q, lv, mu, rv);
+        if (!ok) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) rv[t] = 0.0f;
+        } else if (!quant) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) rv[t] = w[t];
+        } else {
+          const uint32_t codes = *reinterpret_cast<const uint32_t *>(st + kTcRawCodes + c_off);
+          const float ap = block_constant(qs[ci], ss[ci], q.tab.qx, mu);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(codes >> (4 * t)) & 15u], ap)));
+            rv[t] = __fsub_rn(w[t], wq);
+          }
+        }
         float hv[8], lo[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
@@ -364,39 +472,27 @@ __global__ void __launch_bounds__(kTcThreads, 2)   // two CTAs per SM (the split
           lo[t] = __fsub_rn(rv[t], hv[t]);
         }
         if (!TRANS) {
-          const int id = pt + kTcProducers * u, row = id >> 2, c = 8 * (id & 3);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const uint32_t off = tc_off(row, c + 4 * h);
+            const uint32_t off = tc_off(row, col + 4 * h);
             *reinterpret_cast<float4 *>(ah + off) = make_float4(hv[4 * h], hv[4 * h + 1], hv[4 * h + 2], hv[4 * h + 3]);
             *reinterpret_cast<float4 *>(al + off) = make_float4(lo[4 * h], lo[4 * h + 1], lo[4 * h + 2], lo[4 * h + 3]);
           }
         } else {
-          const int g = pw + 8 * u;
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const uint32_t off = tc_off(8 * g + t, lane);
+            const uint32_t off = tc_off(col + t, lane);
             *reinterpret_cast<float *>(ah + off) = hv[t];
             *reinterpret_cast<float *>(al + off) = lo[t];
           }
         }
       }
-#pragma unroll
-      for (int v = 0; v < (kTcRed * kLqMaxL + kTcProducers - 1) / kTcProducers; ++v) {
-        const int e = pt + kTcProducers * v;
-        if (v < nb && e < kTcRed * l) {
-          const int rl = e / l, j = e - rl * l;
-          const float h = tf32_hi(bv[v]);
-          const uint32_t off = tc_off(j, rl);
-          *reinterpret_cast<float *>(bh + off) = h;
-          *reinterpret_cast<float *>(bl + off) = __fsub_rn(bv[v], h);
-        }
-      }
       fence_proxy_async_smem();   // generic-proxy writes visible to the tensor core
-      mbar_arrive(&full[s]);
+      mbar_arrive(&op_full[so]);
+      mbar_arrive(&raw_empty[sr]);
     }
-    // epilogue: warps 1..4 hold TMEM lanes 32 (warp % 4) .. + 31 = output rows of the tile
-    if (warp <= 4) {
+    // epilogue: warps 2..5 hold TMEM lanes 32 (warp % 4) .. + 31 = output rows of the tile
+    if (warp <= 5) {
       const bool ok = mbar_wait(acc_full, 0, kTcDrain);
       tc_fence_after();
       const bool live = __all_sync(0xffffffffu, ok && *abort_flag == 0 && nsteps > 0);
@@ -752,7 +848,7 @@ struct LqPlan {
   int64_t rm_cols, rm_splits;      // K range per split and number of splits of R M
   int64_t res_ctas;                // CTAs of the residual kernel (error parts)
   int64_t gram_parts_max;
-  size_t E, qws, Ya, Yb, Za, Zb, Zpart, Gpart, G, T, M1, M2, sv, errpart, norm2, total;
+  size_t E, qws, Ya, Yb, Za, Zb, Zpart, Bt, Gpart, G, T, M1, M2, sv, errpart, norm2, total;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -770,13 +866,13 @@ LqPlan lq_plan(int64_t N, int64_t K, int r, int l, int dq) {
   p.K = K;
   p.r = r;
   p.l = l;
-  // both products: about two CTAs per SM, splits of the reduction at least four steps deep
+  // both products: one CTA per SM in one wave, splits of the reduction at least four steps deep
   const int64_t col_tiles = ceil_div(K, kTcRows);
-  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(2 * 148 / col_tiles, ceil_div(N, 4 * kTcRed)));
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(148 / col_tiles, ceil_div(N, 4 * kTcRed)));
   p.rt_rows = ceil_div(ceil_div(N, splits), kTcRed) * kTcRed;
   p.rt_splits = ceil_div(N, p.rt_rows);
   const int64_t row_tiles = ceil_div(N, kTcRows);
-  splits = std::max<int64_t>(1, std::min<int64_t>(2 * 148 / row_tiles, ceil_div(K, 4 * kTcRed)));
+  splits = std::max<int64_t>(1, std::min<int64_t>(148 / row_tiles, ceil_div(K, 4 * kTcRed)));
   p.rm_cols = ceil_div(ceil_div(K, splits), kTcRed) * kTcRed;
   p.rm_splits = ceil_div(K, p.rm_cols);
   p.res_ctas = ceil_div(K, kResCols) * ceil_div(N, kResRows);
@@ -794,6 +890,8 @@ LqPlan lq_plan(int64_t N, int64_t K, int r, int l, int dq) {
   p.Za = take(4 * static_cast<size_t>(K) * l);
   p.Zb = take(4 * static_cast<size_t>(K) * l);
   p.Zpart = take(4 * std::max(static_cast<size_t>(p.rt_splits) * K, static_cast<size_t>(p.rm_splits) * N) * l);
+  // the products' split small operand: hi and lo tiles of (l rounded up to 16) x 32 per 32-deep block
+  p.Bt = take(4 * 2 * static_cast<size_t>(ceil_div(std::max(N, K), kTcRed)) * kTcRed * ceil_div(l, 16) * 16);
   p.Gpart = take(8 * static_cast<size_t>(p.gram_parts_max) * l * l);
   p.G = take(8 * static_cast<size_t>(l) * l);
   p.T = take(8 * static_cast<size_t>(l) * l);
@@ -843,9 +941,31 @@ struct LqRun {
     int *status = device_status_ptr();
     if (err == cudaSuccess && !status) err = cudaErrorInvalidValue;
     if (err != cudaSuccess) return;
+    CUtensorMap tmW, tmC, tmB;
+    // W [N, K] fp32: 32 x 128 (Y) or four 32 x 32 (Z) boxes, 128B-swizzled; codes [N, K/2] bytes:
+    // 16 x 128 (Y) or 64 x 32 (Z) boxes; the small operand [reduction, l] fp32: l x 32 boxes
+    bool ok = make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.K, p.N, static_cast<uint64_t>(p.K) * 4, 32,
+                           TRANS ? 32 : kTcRows, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (q.codes)
+      ok = ok && make_tmap_2d(&tmC, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.K / 2, p.N, static_cast<uint64_t>(p.K) / 2,
+                              TRANS ? 64 : 16, TRANS ? 32 : kTcRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+      tmC = tmW;
+    // the small operand, split into hi / lo tiles of nl x 32 per 32-deep block
+    const int64_t red = TRANS ? p.N : p.K, nblk = ceil_div(red, kTcRed);
+    if (nblk * nl * (kTcRed / 4) >= (int64_t(1) << 31)) ok = false;   // the split kernel indexes with 32 bits
+    float *Bt = wsp<float>(ws, p.Bt);
+    ok = ok && make_tmap_2d(&tmB, Bt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kTcRed, static_cast<uint64_t>(2 * nblk * nl),
+                            kTcRed * 4, kTcRed, static_cast<uint32_t>(nl), CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) {
+      err = cudaErrorInvalidValue;
+      return;
+    }
     const dim3 grid(static_cast<unsigned>(ceil_div(TRANS ? p.K : p.N, kTcRows)), static_cast<unsigned>(splits));
     prof_mark(kProfLqProduct, true, st);
-    lq_tc_kernel<TRANS><<<grid, kTcThreads, smem, st>>>(W, p.N, p.K, q, B, p.l, nl, red_per, part, status,
+    lq_tc_split_kernel<<<static_cast<unsigned>(ceil_div(nblk * nl * (kTcRed / 4), 256)), 256, 0, st>>>(
+        B, red, p.l, nl, static_cast<int>(nblk), Bt);
+    lq_tc_kernel<TRANS><<<grid, kTcThreads, smem, st>>>(tmW, tmC, tmB, p.N, p.K, q, p.l, nl, red_per, part, status,
                                                          wait_limit());
     prof_mark(kProfLqProduct, false, st);
     check();
@@ -962,7 +1082,8 @@ qlora_status lq_args(const float *W, int64_t N, int64_t K, int r, int l, int dq,
                      LqPlan *plan) {
   if (!W || N < 1 || K < 1) return QLORA_ERR_INVALID_ARG;
   const int lc = l == 0 ? r : l;
-  if (r < 1 || lc < r || lc > kLqMaxL || (lc & 1)) return QLORA_ERR_INVALID_ARG;
+  // l a multiple of 4: the test matrix's rows are 16-byte runs for the products' tensor maps
+  if (r < 1 || lc < r || lc > kLqMaxL || (l != 0 && (l & 3))) return QLORA_ERR_INVALID_ARG;
   if (N < lc || K < lc) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (l != 0 && K % kBlock != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;   // the products walk whole blocks
   if (dq == QLORA_DQ_SIGNED && N * K >= (int64_t(1) << 38)) return QLORA_ERR_UNSUPPORTED_SHAPE;

@@ -329,7 +329,8 @@ qlora_status qlora_format_codebook(int format, float *levels, float *thresh);
  *           (sized for Q->dq, as for qlora_quantize_nf4).
  *   L1    : device fp32 [N, r];  L2 : device fp32 [r, K]  (outputs).
  *   Omega : device fp32 [K, l] Gaussian test matrix (the random numbers the
- *           method draws; the caller supplies them).  r <= l <= 96, l even,
+ *           method draws; the caller supplies them).  r <= l <= 96, l a
+ *           multiple of 4 (16-byte rows),
  *           N >= l, K >= l.  0 <= power <= 16, 1 <= iters <= 1000.
  *   err   : device fp64 [2 iters]: err[2t] = ||W - W' - L1 L2||_F / ||W||_F
  *           after round t's quantization, err[2t+1] after its rank-r step.

@@ -204,6 +204,7 @@ def test_lq_sizes_and_argument_errors():
     assert lib.qlora_lq_lowrank(FAKE, 256, 512, ctypes.byref(q.Nf4WeightC(256, 256, FAKE, FAKE, FAKE, 0, 0)),
                                 FAKE, 24, 2, 16, FAKE, FAKE, FAKE, big, None) == 1       # shape mismatch
     assert lib.qlora_lq_lowrank(FAKE, 10, 512, None, FAKE, 24, 2, 16, FAKE, FAKE, FAKE, big, None) == 2
+    assert lib.qlora_lq_lowrank(FAKE, 256, 512, None, FAKE, 26, 2, 16, FAKE, FAKE, FAKE, big, None) == 1   # l % 4
     assert lib.qlora_lq_quantize_residual(FAKE, None, FAKE, 16, ctypes.byref(w), FAKE, big, None) == 1
     assert lib.qlora_lq_quantize_residual(FAKE, FAKE, FAKE, 16, ctypes.byref(w), FAKE, 64, None) == 7
 
