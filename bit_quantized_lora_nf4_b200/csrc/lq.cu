@@ -371,44 +371,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- loader
     const uint32_t bytes = static_cast<uint32_t>(kTcATile + (quant ? 2048 : 0) + 2 * nl * kTcRed * 4);
-    TcConst c0 = tc_const_load<TRANS>(q, N, K, o0, ra, rb, lane);
-    TcConst c1 = tc_const_load<TRANS>(q, N, K, o0, ra + kTcRed, rb, lane);
-    TcConst c2 = tc_const_load<TRANS>(q, N, K, o0, ra + 2 * kTcRed, rb, lane);
-    for (int i = 0; i < nsteps; ++i) {
-      const int s = i % RS;
-      const int64_t r0 = ra + static_cast<int64_t>(i) * kTcRed;
-      if (i >= RS && !lq_wait(&raw_empty[s], ((i / RS) & 1) ^ 1, wait_limit, abort_flag, status))
-        break;
-      uint8_t *st = raw_ring + s * raw_bytes;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&raw_full[s], bytes);
-        if (!TRANS) {
-          tma_load_2d(st, &tmW, &raw_full[s], static_cast<int>(r0), static_cast<int>(o0));
-          if (quant) tma_load_2d(st + kTcRawCodes, &tmC, &raw_full[s], static_cast<int>(r0 / 2), static_cast<int>(o0));
-        } else {
-          for (int b = 0; b < 4; ++b)
-            tma_load_2d(st + 4096 * b, &tmW, &raw_full[s], static_cast<int>(o0) + 32 * b, static_cast<int>(r0));
-          if (quant) tma_load_2d(st + kTcRawCodes, &tmC, &raw_full[s], static_cast<int>(o0 / 2), static_cast<int>(r0));
-        }
-        const int blk = static_cast<int>(r0 / kTcRed);   // the small operand's hi and lo tiles of this block
-        tma_load_2d(st + kTcRawB, &tmB, &raw_full[s], 0, 2 * blk * nl);
-        tma_load_2d(st + kTcRawB + nl * kTcRed * 4, &tmB, &raw_full[s], 0, (2 * blk + 1) * nl);
-      }
-      uint8_t *qs = st + raw_q;
-      float *ss = reinterpret_cast<float *>(st + raw_s);
+    // three register slots used in place (slot u of step i is reloaded for step i + 3 right after it
+    // is stored), so no instruction ever waits on a constant load still in flight
+    TcConst c[3];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int idx = TRANS ? lane * 2 + j : lane + 32 * j;
-        if (!TRANS || j < 4) {
-          if (TRANS && j >= 2) continue;
-          qs[idx] = static_cast<uint8_t>(c0.q[j]);
-          ss[idx] = c0.S[j];
+    for (int u = 0; u < 3; ++u) c[u] = tc_const_load<TRANS>(q, N, K, o0, ra + u * kTcRed, rb, lane);
+    bool stop = false;
+#pragma unroll 1
+    for (int i0 = 0; i0 < nsteps && !stop; i0 += 3) {
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int i = i0 + u;
+        if (i >= nsteps || stop) break;
+        const int s = i % RS;
+        const int64_t r0 = ra + static_cast<int64_t>(i) * kTcRed;
+        if (i >= RS && !lq_wait(&raw_empty[s], ((i / RS) & 1) ^ 1, wait_limit, abort_flag, status)) {
+          stop = true;
+          break;
         }
+        uint8_t *st = raw_ring + s * raw_bytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&raw_full[s], bytes);
+          if (!TRANS) {
+            tma_load_2d(st, &tmW, &raw_full[s], static_cast<int>(r0), static_cast<int>(o0));
+            if (quant)
+              tma_load_2d(st + kTcRawCodes, &tmC, &raw_full[s], static_cast<int>(r0 / 2), static_cast<int>(o0));
+          } else {
+            for (int b = 0; b < 4; ++b)
+              tma_load_2d(st + 4096 * b, &tmW, &raw_full[s], static_cast<int>(o0) + 32 * b, static_cast<int>(r0));
+            if (quant)
+              tma_load_2d(st + kTcRawCodes, &tmC, &raw_full[s], static_cast<int>(o0 / 2), static_cast<int>(r0));
+          }
+          const int blk = static_cast<int>(r0 / kTcRed);   // the small operand's hi and lo tiles of this block
+          tma_load_2d(st + kTcRawB, &tmB, &raw_full[s], 0, 2 * blk * nl);
+          tma_load_2d(st + kTcRawB + nl * kTcRed * 4, &tmB, &raw_full[s], 0, (2 * blk + 1) * nl);
+        }
+        uint8_t *qs = st + raw_q;
+        float *ss = reinterpret_cast<float *>(st + raw_s);
+#pragma unroll
+        for (int j = 0; j < (TRANS ? 2 : 4); ++j) {
+          const int idx = TRANS ? lane * 2 + j : lane + 32 * j;
+          qs[idx] = static_cast<uint8_t>(c[u].q[j]);
+          ss[idx] = c[u].S[j];
+        }
+        mbar_arrive(&raw_full[s]);
+        c[u] = tc_const_load<TRANS>(q, N, K, o0, r0 + 3 * kTcRed, rb, lane);
       }
-      mbar_arrive(&raw_full[s]);
-      c0 = c1;
-      c1 = c2;
-      c2 = tc_const_load<TRANS>(q, N, K, o0, r0 + 3 * kTcRed, rb, lane);
     }
   } else {
     // ---------------------------------------------------------------- producers
