@@ -282,7 +282,8 @@ __device__ __forceinline__ void h_part(const GemvParams &p, const XSource<NT, XS
 #pragma unroll
         for (int w = 0; w < GV_WARPS; ++w) v += red[((w * NT + t) * 4 + e) * 32 + lane];
         // C fragment: H^T[j0 + g + 8 (e >> 1)][tok = 8 t + 2 c + (e & 1)]
-        const int64_t o = static_cast<int64_t>(i) * 8 * NT * 16 + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1);
+        [[maybe_unused]] const int64_t o =   // checked in the bounds-checked build only
+            static_cast<int64_t>(i) * 8 * NT * 16 + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1);
         if (QL_IN_BOUNDS(p.status, o, static_cast<int64_t>(p.HP) * 8 * NT * 16))
           __stcg(dst + (8 * t + 2 * c + (e & 1)) * 16 + g + 8 * (e >> 1), v);
       }

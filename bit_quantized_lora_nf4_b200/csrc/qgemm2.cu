@@ -657,7 +657,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int acc = NACC == 1 ? 0 : (dwarp >> 2);
       const int col_begin = NACC == 1 ? (dwarp >> 2) * 128 : 0;
       const int nchunk = NACC == 1 ? 4 : 8;
-      const int arow = quarter * 32 + lane;     // row of this CTA's accumulator
       // A piece is laid out by thread: float4 group g (columns 4g .. 4g + 3) of
       // lane l of warp quarter q of accumulator a at float4 index
       // ((a * 4 + q) * 64 + g) * 32 + l, so that a warp writes and reads 512
