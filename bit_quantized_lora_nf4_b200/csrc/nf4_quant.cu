@@ -28,6 +28,8 @@
 // the fp32 a_b and an exact, order-free sum of the a_b (integer digits added
 // with 64-bit atomics); a second kernel turns the sum into mu and codes every
 // group's constants against it.
+#include <atomic>
+
 #include "decode.cuh"
 #include "internal.h"
 
@@ -316,6 +318,26 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_kernel(const uint8
   }
 }
 
+// SMs of the current device, looked up once per device (148 when no device
+// answers: sizing only).
+int device_sm_count_cached() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  int v = cache[dev].load();
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      return 148;
+    }
+    cache[dev].store(v);
+  }
+  return v;
+}
+
 // Persistent dequantizer for whole chunks of 8192 weights (128 blocks): the
 // 4 KB of codes and the chunk's 128 block constants arrive by 1-D bulk copies
 // into a ring of kDqStages stages issued kDqStages - 1 chunks ahead, 256
@@ -351,6 +373,11 @@ __global__ void __launch_bounds__(kDeqThreads) nf4_dequantize_bulk_kernel(const 
   const int64_t first = blockIdx.x;
   const int64_t step = gridDim.x;
   int issued = 0;   // chunks whose load thread 0 has issued
+  // The next kernel on the stream may be scheduled now (its launch overlaps this
+  // one's tail); no global memory is touched before the previous kernel's
+  // writes are visible.
+  griddep_launch_dependents();
+  griddep_wait();
   auto issue = [&](int j) {   // the load of this CTA's chunk number j into stage j % kDqStages
     const int64_t ch = first + j * step;
     uint8_t *dst = cbuf + (j % kDqStages) * kDqStageBytes;
@@ -448,12 +475,27 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *absmax_q, con
   prof_mark(kProfDequant, true, st);
   if (nfull > 0) {
     int *status = device_status_ptr();
-    int64_t blocks = nfull < 148 * QLORA_DQ_CTAS_PER_SM ? nfull : 148 * QLORA_DQ_CTAS_PER_SM;
+    // as many CTAs as are co-resident, each taking the same number of chunks (so no
+    // last round runs with a part of the grid idle)
+    const int64_t slots = static_cast<int64_t>(device_sm_count_cached()) * QLORA_DQ_CTAS_PER_SM;
+    const int64_t per = (nfull + slots - 1) / slots;
+    const int64_t blocks = (nfull + per - 1) / per;
     cudaError_t e = cudaFuncSetAttribute(nf4_dequantize_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kDqSmem);
     if (e != cudaSuccess) return e;
-    nf4_dequantize_bulk_kernel<<<static_cast<unsigned>(blocks), kDeqThreads, kDqSmem, st>>>(
-        codes, absmax_q, group_scale, nfull, out, numel, tab, status, wait_limit());
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(kDeqThreads);
+    cfg.dynamicSmemBytes = kDqSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the previous kernel's tail
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, nf4_dequantize_bulk_kernel, codes, absmax_q, group_scale, nfull, out, numel, tab,
+                           status, wait_limit());
+    if (e != cudaSuccess) return e;
   }
   const int64_t done = nfull * kDqChunk;
   if (done < numel) {
