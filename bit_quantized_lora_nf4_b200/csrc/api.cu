@@ -586,9 +586,11 @@ qlora_status linear_fwd_impl(const WeightSrc &src, const uint16_t *X, int64_t M,
                weight_table(w)};
     return launch_gemv(g, st);
   }
-  QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
   QGemmArgs g = gemm_args(src, false, M, X, at<uint16_t>(ws, p.sH), B, r, Y);
   g.sk_ws = p.sk_region(ws, ws_bytes);
+  // the GEMM's stream-K counters are cleared before H, so the GEMM follows H directly
+  QL_TRY(qgemm_prepare_split(g, st, &g.sk_zeroed));
+  QL_TRY(run_h(p, ws, X, A, M, K, r, s, H, at<uint16_t>(ws, p.sH), nullptr, st));
   return launch_qgemm(g, st);
 }
 
@@ -603,6 +605,8 @@ qlora_status linear_bwd_impl(const WeightSrc &src, const uint16_t *X, const uint
   dgrad.sk_ws = p.sk_region(ws, ws_bytes);
   if (H_saved && !aligned16(H_saved)) return QLORA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the dgrad GEMM's stream-K counters are cleared before the products it depends on
+  QL_TRY(qgemm_prepare_split(dgrad, st, &dgrad.sk_zeroed));
   float *part = at<float>(ws, p.part);
   uint16_t *Hs = at<uint16_t>(ws, p.Hs);
   uint16_t *Gb = at<uint16_t>(ws, p.Gb);

@@ -73,6 +73,7 @@ struct QGemmArgs {
   Nf4Table tab;        // weight_table() of the weight
   const uint16_t *wdense = nullptr;   // dense bf16 W' [wN, wK] instead of the packed weight (pair kernel only)
   void *sk_ws = nullptr;              // pair kernel: pair_sk_workspace_bytes(M) for its stream-K tail (null: none)
+  bool sk_zeroed = false;             // qgemm_prepare_split already cleared the tail's counters on the stream
 };
 // Workspace of the pair kernel's stream-K tail (fp32 pieces of shared tiles and their counters).
 size_t pair_sk_workspace_bytes(int64_t M);
@@ -83,6 +84,11 @@ qlora_status launch_qgemm(const QGemmArgs &a, cudaStream_t st);
 // for M > kPairMinRows and for a dense W'.
 constexpr int64_t kPairMinRows = 128;
 qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st);
+// Clears the stream-K tail's counters on `st` now when the launch of `a` will
+// split its last round (the same decision the launch makes), so that the
+// launch can follow the kernel before it with programmatic dependent launch;
+// sets *zeroed accordingly.  Issue it before the products the GEMM depends on.
+qlora_status qgemm_prepare_split(const QGemmArgs &a, cudaStream_t st, bool *zeroed);
 
 // Few-token forward: Y[M, N] = X W'^T + (s X A^T) B^T for M <= 16.
 struct GemvArgs {

@@ -862,7 +862,63 @@ int cluster_slots(Kern kern, cudaLaunchConfig_t cfg) {
   return v > 0 ? v : 0;
 }
 
+// Whether a launch splits the K-steps of its last, partial round of tiles over
+// all cluster slots (stream-K), and how.
+struct SplitPlan {
+  bool split = false;
+  int tail = 0, units = 0;
+  int64_t sk_steps = 0;
+};
+SplitPlan split_plan(const QGemmArgs &a, int tiles, int ns, int slots) {
+  SplitPlan sp;
+  const int mode = stream_k_mode();
+  sp.tail = slots > 0 && a.sk_ws && mode != QLORA_STREAM_K_OFF ? tiles % slots : 0;
+  sp.sk_steps = static_cast<int64_t>(sp.tail) * ns;
+  sp.units = static_cast<int>(std::min<int64_t>(slots, std::max<int64_t>(1, sp.sk_steps / kSkMinSteps)));
+  sp.split = sp.tail > 0 && (mode == QLORA_STREAM_K_ALWAYS ||
+                             ceil_div(sp.sk_steps, sp.units) + kSkCostSteps < ns + kTileCostSteps);
+  return sp;
+}
+
+// Tiles and K-steps per tile of a pair launch (as launch_qgemm_pair sets them).
+void pair_shape(const QGemmArgs &a, int *tiles, int *ns) {
+  const int64_t kred = a.dgrad ? a.wN : a.wK;
+  const int64_t n_out = a.dgrad ? a.wK : a.wN;
+  const int nacc = a.M > 2 * BM ? 2 : 1;
+  const int bk = nacc == 2 ? Cfg<2>::BK : Cfg<1>::BK;
+  *ns = static_cast<int>(ceil_div(kred, bk) + ceil_div(a.r, bk));
+  *tiles = static_cast<int>(ceil_div(a.M, 2 * BM * nacc) * ceil_div(n_out, BN));
+}
+
 }  // namespace
+
+qlora_status qgemm_prepare_split(const QGemmArgs &a, cudaStream_t st, bool *zeroed) {
+  *zeroed = false;
+  if (!(a.M > kPairMinRows || a.wdense) || !a.sk_ws) return QLORA_OK;   // no stream-K tail on this launch
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // every instance of the pair kernel has the same shape of resources; the slot count is cached
+  if (cudaFuncSetAttribute(qgemm2_kernel<false, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      cudaSuccess)
+    return QLORA_ERR_CUDA;
+  const int slots = std::min(cluster_slots(qgemm2_kernel<false, 2, false>, cfg), kSkMaxUnits);
+  int tiles, ns;
+  pair_shape(a, &tiles, &ns);
+  if (!split_plan(a, tiles, ns, slots).split) return QLORA_OK;
+  if (cudaMemsetAsync(a.sk_ws, 0, kSkCounterBytes, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  *zeroed = true;
+  return QLORA_OK;
+}
 
 size_t pair_sk_workspace_bytes(int64_t M) {
   const int64_t nacc = M > 2 * BM ? 2 : 1;
@@ -943,22 +999,19 @@ qlora_status launch_qgemm_pair(const QGemmArgs &a, cudaStream_t st) {
     // all clusters (stream-K), so that no cluster idles while others finish.
     const int slots = std::min(cluster_slots(kern, cfg), kSkMaxUnits);
     int clusters = slots > 0 ? std::min(tiles, slots) : tiles;
-    const int mode = stream_k_mode();
-    const int tail = slots > 0 && a.sk_ws && mode != QLORA_STREAM_K_OFF ? tiles % slots : 0;
-    const int64_t sk_steps = static_cast<int64_t>(tail) * p.ns;
-    const int units = static_cast<int>(std::min<int64_t>(slots, std::max<int64_t>(1, sk_steps / kSkMinSteps)));
-    const bool split = tail > 0 && (mode == QLORA_STREAM_K_ALWAYS ||
-                                    ceil_div(sk_steps, units) + kSkCostSteps < p.ns + kTileCostSteps);
-    if (split) {
-      p.dp_tiles = tiles - tail;
-      p.sk_steps = sk_steps;
-      p.sk_units = units;
+    const SplitPlan sp = split_plan(a, tiles, p.ns, slots);
+    if (sp.split) {
+      p.dp_tiles = tiles - sp.tail;
+      p.sk_steps = sp.sk_steps;
+      p.sk_units = sp.units;
       p.sk_count = static_cast<int *>(a.sk_ws);
       p.sk_ready = p.sk_count + 2 * kSkMaxUnits;
       p.sk_part = reinterpret_cast<float *>(static_cast<char *>(a.sk_ws) + kSkCounterBytes);
-      clusters = p.dp_tiles > 0 ? slots : units;
-      e = cudaMemsetAsync(a.sk_ws, 0, kSkCounterBytes, st);
-      if (e != cudaSuccess) return e;
+      clusters = p.dp_tiles > 0 ? slots : sp.units;
+      if (!a.sk_zeroed) {
+        e = cudaMemsetAsync(a.sk_ws, 0, kSkCounterBytes, st);
+        if (e != cudaSuccess) return e;
+      }
     }
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
     prof_mark(kind, true, st);
