@@ -502,15 +502,22 @@ int64_t skinny_tiles(int64_t I, int64_t J) {
   const int64_t t = ceil_div(I, TBM) * ceil_div(J, tc_bn(J));
   return t < 1 ? 1 : t;
 }
+// Clusters of z CTAs that are co-resident: a cluster sits in one GPC, so each
+// of the 8 GPCs (at least 18 SMs, TCTAS_PER_SM CTAs per SM) holds
+// floor(36 / z) of them (32 clusters of 8 measured on B200).  A fixed bound,
+// so that workspace sizes do not depend on the device a query runs on.
+int64_t coresident_clusters(int64_t z) { return 8 * ((18 * TCTAS_PER_SM) / z); }
+
 // Splits of the reduction for `tiles` tiles sharing one launch: every split of
-// every tile in one wave, at least four 64-deep steps per split, at most a
-// portable cluster.
+// every tile in one wave of co-resident clusters, at least four 64-deep steps
+// per split, at most a portable cluster.
 void plan_splits(int64_t tiles, int64_t Kred, int *splits, int64_t *k_per_split) {
   if (Kred < 1) Kred = 1;
   int64_t sp = 148 * TCTAS_PER_SM / tiles;
   const int64_t max_sp = Kred / (4 * TBK) > 0 ? Kred / (4 * TBK) : 1;
   if (sp > max_sp) sp = max_sp;
   if (sp > kMaxSkinnyCluster) sp = kMaxSkinnyCluster;   // the splits of a tile form one cluster
+  while (sp > 1 && tiles > coresident_clusters(sp)) --sp;
   if (sp < 1) sp = 1;
   const int64_t kps = ceil_div(ceil_div(Kred, sp), TBK) * TBK;
   *splits = static_cast<int>(ceil_div(Kred, kps));
