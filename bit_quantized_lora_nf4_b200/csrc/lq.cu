@@ -192,7 +192,11 @@ __global__ void lq_sum_kernel(const double *__restrict__ part, int64_t n, const 
 //            per product term, the level of an fp32 multiply-add.
 // Warps 2-5 then write the tile's rows to part[split][row][c], and
 // lq_sum_splits_kernel adds the splits in order.
-constexpr int kTcRows = 128, kTcRed = 32, kTcMaxRawStages = 4, kTcOpStages = 2, kTcProducers = 512;
+// Operand-ring depth (compile-time tunable; three stages measured slightly slower than two).
+#ifndef QLORA_LQ_OP_STAGES
+#define QLORA_LQ_OP_STAGES 2
+#endif
+constexpr int kTcRows = 128, kTcRed = 32, kTcMaxRawStages = 4, kTcOpStages = QLORA_LQ_OP_STAGES, kTcProducers = 512;
 constexpr int kTcThreads = 64 + kTcProducers;
 constexpr int kTcATile = kTcRows * kTcRed * 4;          // 16 KB: one component of the R tile (and W's raw tile)
 // raw stage: W tile (16 KB), codes (2 KB), the small operand's hi and lo tiles (nl x 128 B each, 1024-
