@@ -24,12 +24,13 @@
 //      tiles when M > 8).  For every tile it touches it stores its fp32 sum
 //      as a piece in the CTA's slot (tile - first tile of the CTA) + warp.
 //   3. Each warp stamps its own flag once its pieces are stored and finishes
-//      the tiles whose last unit lies in its range: the pieces of every CTA
-//      on the tile, in CTA order and warp order within a CTA (a fixed order,
-//      so results do not depend on timing), waiting only for the flags of
-//      the warps holding those pieces (lanes poll in parallel) and of the
-//      tiles of H; then (s H) B^T on mma.sync (s H as a bf16 hi/lo pair
-//      formed from the tiles of H in L2) and bf16 Y.
+//      the tiles whose last unit lies in its range: once the tiles of H are
+//      in, (s H) B^T on mma.sync (s H as a bf16 hi/lo pair formed from the
+//      tiles of H in L2; its loads overlap the wait for the pieces), then the
+//      pieces of every CTA on the tile, in CTA order and warp order within a
+//      CTA (a fixed order, so results do not depend on timing), waiting only
+//      for the flags of the warps holding those pieces (lanes poll in
+//      parallel); then bf16 Y.
 // Nothing waits before it has published what others wait for, so the waits
 // form no cycle.  Flags carry a 64-bit tag unique to the launch (consecutive
 // from a random start), so no word needs clearing between launches.
@@ -577,9 +578,10 @@ __device__ __forceinline__ void store_y(const GemvParams &p, int t, const float 
 }
 
 // Phase 3, per warp: the tiles whose last unit lies in this warp's range
-// [aw, bw).  A tile's pieces are added CTA by CTA (CTA order is K order) and,
-// within a CTA, warp by warp; the warp first waits for the flags of every
-// other warp on the tile (lanes poll in parallel) and of the tiles of H.
+// [aw, bw).  The adapter term comes first (the tiles of H are waited for once
+// per warp), then the tile's pieces CTA by CTA (CTA order is K order) and,
+// within a CTA, warp by warp, each CTA's after the flags of its warps on the
+// tile (lanes poll in parallel).
 template <int NT>
 __device__ __forceinline__ void finish_tiles(const GemvParams &p, const int *starts, int cta, int aw, int bw) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -592,6 +594,7 @@ __device__ __forceinline__ void finish_tiles(const GemvParams &p, const int *sta
     if (!h_ready) {
       for (int i = lane; i < p.JT; i += 32)
         if (!wait_flag(p.hflag + i, p.tag, p.wait_limit)) latch_status(p.status, QLORA_ERR_DEVICE_TIMEOUT);
+      __syncwarp();   // orders each lane's acquire before every lane's reads of H
       h_ready = true;
     }
     float acc[NT][4];
@@ -599,6 +602,7 @@ __device__ __forceinline__ void finish_tiles(const GemvParams &p, const int *sta
     for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[tt][e] = 0.0f;
+    add_lora<NT>(p, t, acc, lane);   // its loads are in flight while the pieces are waited for
     const int c_first = cta_owner(starts, p.G, t * S);
     for (int cp = c_first; cp <= cta; ++cp) {
       const int ap = starts[cp], bp = starts[cp + 1];
@@ -640,7 +644,6 @@ __device__ __forceinline__ void finish_tiles(const GemvParams &p, const int *sta
           for (int e = 0; e < 4; ++e) acc[tt][e] += v[w][tt][e];
       }
     }
-    add_lora<NT>(p, t, acc, lane);
     store_y<NT>(p, t, acc, lane);
   }
 }
