@@ -32,7 +32,10 @@
 //      for the flags of the warps holding those pieces (lanes poll in
 //      parallel); then bf16 Y.
 // Nothing waits before it has published what others wait for, so the waits
-// form no cycle.  Flags carry a 64-bit tag unique to the launch (consecutive
+// form no cycle.  A flag is published by one thread with a release store after
+// a CTA or warp barrier (which orders the other threads' stores before it) and
+// read with acquire loads, whose thread then meets the others at a warp or CTA barrier
+// before any of them reads what the flag covers.  Flags carry a 64-bit tag unique to the launch (consecutive
 // from a random start), so no word needs clearing between launches.
 #include <algorithm>
 #include <atomic>
@@ -290,11 +293,8 @@ __device__ __forceinline__ void h_part(const GemvParams &p, const XSource<NT, XS
       }
     }
   }
-  __syncthreads();   // the part is stored, and red is free again
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (QL_IN_BOUNDS(p.status, i, p.HP)) st_release_gpu_u64(p.hpflag + i, p.tag);
-  }
+  __syncthreads();   // the part is stored (and ordered before the release below), and red is free again
+  if (threadIdx.x == 0 && QL_IN_BOUNDS(p.status, i, p.HP)) st_release_gpu_u64(p.hpflag + i, p.tag);
 }
 
 // CTA jt < JT: tile jt of H^T, the sum of its S parts in K order, once their
@@ -326,11 +326,8 @@ __device__ __forceinline__ void h_tile(const GemvParams &p, int jt) {
     if (p.H_out && tok < p.M && j < p.r && QL_IN_BOUNDS(p.status, tok * p.r + j, p.M * p.r))
       p.H_out[static_cast<int64_t>(tok) * p.r + j] = h;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (QL_IN_BOUNDS(p.status, jt, p.JT)) st_release_gpu_u64(p.hflag + jt, p.tag);
-  }
+  __syncthreads();   // every thread's stores are ordered before the release below
+  if (threadIdx.x == 0 && QL_IN_BOUNDS(p.status, jt, p.JT)) st_release_gpu_u64(p.hflag + jt, p.tag);
 }
 
 // The code stream of one weight warp: lane 0 keeps GV_STAGES units of the
@@ -752,13 +749,11 @@ __global__ void __launch_bounds__(GV_THREADS, GV_CTAS_PER_SM) gemv_kernel(const 
   if (cta < p.JT) h_tile<NT>(p, cta);
   if (aw >= bw) return;
   weight_role<NT, XS>(&tm_codes, p, x, cs, cst, q0, cta, a / p.S, aw, bw);
-  // this warp's pieces are stored: publish them
+  // this warp's pieces are stored: publish them (the warp barrier orders every
+  // lane's stores before lane 0's release)
   __syncwarp();
-  if (lane == 0) {
-    __threadfence();
-    if (QL_IN_BOUNDS(p.status, cta * GV_WARPS + warp, p.G * GV_WARPS))
-      st_release_gpu_u64(p.wflag + cta * GV_WARPS + warp, p.tag);
-  }
+  if (lane == 0 && QL_IN_BOUNDS(p.status, cta * GV_WARPS + warp, p.G * GV_WARPS))
+    st_release_gpu_u64(p.wflag + cta * GV_WARPS + warp, p.tag);
   finish_tiles<NT>(p, starts, cta, aw, bw);
 }
 
