@@ -67,9 +67,11 @@ constexpr int GV_BAR_OFFSET = GV_RING_BYTES;               // ring barriers, the
 constexpr int GV_MAX_CTAS = 511;                            // CTA starts kept in shared memory
 constexpr int GV_START_OFFSET = GV_RING_BYTES + 512;        // int starts[GV_MAX_CTAS + 1]
 constexpr int GV_AUX_OFFSET = GV_RING_BYTES + 512 + 2048 + 512;   // H reduction, then s H (hi, lo); 1024-aligned
-// Units a warp brings into L2 before the previous kernel's results are waited for.
+// Units a warp brings into L2 before the previous kernel's results are waited for
+// (its TMA ring asks for the next ones right after the wait; prefetching the
+// whole range queues the activation copies behind it: 2 measured best on B200).
 #ifndef QLORA_GEMV_PREFETCH_UNITS
-#define QLORA_GEMV_PREFETCH_UNITS 64
+#define QLORA_GEMV_PREFETCH_UNITS 2
 #endif
 constexpr int GV_PREFETCH_UNITS = QLORA_GEMV_PREFETCH_UNITS;
 // Weight units a CTA gives up for a part of H and for adding a tile of H (tuned on B200).
