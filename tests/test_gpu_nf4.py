@@ -106,7 +106,9 @@ def _tie_weight(levels: np.ndarray) -> torch.Tensor:
 
 @pytest.mark.parametrize("fmt,fid", [("nf4", q.FORMAT_NF4), ("fp4", q.FORMAT_FP4), ("int4", q.FORMAT_INT4)])
 def test_ties_break_to_the_lower_index(lib, fmt, fid):
-    """The benchmark spec: the nearest level, ties broken to the lower code index.  Every
+    """Each normalized weight takes the nearest level ("QLoRA: fine-tuning a 65B
+    model on one GPU", section "NormalFloat, double quantization, paged
+    optimizers"), an exact tie going to the lower code index.  Every
     threshold of every table is hit exactly (the midpoints that are fp32 values
     give true ties: e.g. half of the first level above zero) and one to three
     fp32 steps either side; the codes must equal the oracle's bit for bit."""
