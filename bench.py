@@ -43,7 +43,7 @@ WORKLOAD = "llama7b_projections_q4096x4096_up11008x4096_down4096x11008_m4096_r64
 
 def peaks():
     """Roofline denominators: the measured HBM copy bandwidth and cuBLAS bf16
-    GEMM rate of this machine's B200s (burst: a kernel timed alone, at the full
+    GEMM rate measured on B200s of this kind (burst: a kernel timed alone, at the full
     clock; sustained: seconds of back-to-back GEMMs under the power cap, at the
     median clock recorded with it), else the recipe's fallback figures."""
     try:

@@ -1,5 +1,5 @@
 """Canary-padded output buffers for the GPU tests (stand-in for a memory
-sanitizer, which is not available on this machine).
+sanitizer, which these tests do not run).
 
 Every output of a library call is carved from a larger buffer with PAD bytes
 of a fixed byte pattern on both sides (PAD is a multiple of 16, so the carved

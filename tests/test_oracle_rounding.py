@@ -16,9 +16,9 @@ Each test recomputes the step from the exact rational value of its operands
 (Python ``Fraction``), rounds with tests/exact.py's own rounding routines, and
 compares bit patterns, on at least 10^5 elements over several groups
 (partial groups, sub-normal constants, signed zeros included).  Each test
-also feeds its checker a copy of the oracle step with one rounding slip
+also feeds its check a copy of the oracle step with one rounding slip
 planted (reciprocal-multiply, a fused multiply-add, one rounding where the
-reading has two, a wrong group index) and requires that the checker rejects it,
+reading has two, a wrong group index) and requires that the check rejects it,
 so a pin that could not see such a slip would fail here.
 """
 
