@@ -201,7 +201,10 @@ void prof_mark(int kind, bool begin, cudaStream_t st) {
   if (!P.on || kind <= 0 || kind >= kProfKinds) return;
   cudaEvent_t e = prof_event();
   if (!e) return;
-  cudaEventRecord(e, st);
+  if (cudaEventRecord(e, st) != cudaSuccess) {   // no timing for this launch (the error is left for the next check)
+    if (!begin) P.open[kind] = nullptr;
+    return;
+  }
   if (begin) {
     P.open[kind] = e;
   } else if (P.open[kind]) {
